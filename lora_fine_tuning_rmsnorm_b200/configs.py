@@ -1,0 +1,22 @@
+"""The LoRA-MLP workloads: shapes only (tokens T, hidden d, intermediate f, rank r).
+
+The shapes stand in for the pages' fine-tuning workloads: Llama-3-8B / Llama-3.2-1B
+LoRA/QLoRA SFT at sequence 2048 and batch 4 ("Unsloth提速秘诀：Triton内核如何加速反向传播",
+§4.1; "Unsloth 深度实战", §3.2), with alpha = 16 and eps = 1e-6.
+"""
+from .synth import Shape
+
+TINY = Shape(T=64, d=128, f=344, r=8, alpha=16.0)            # batch 2 x seq 32
+LLAMA32_1B = Shape(T=8192, d=2048, f=8192, r=16, alpha=16.0)  # batch 4 x seq 2048
+LLAMA3_8B = Shape(T=8192, d=4096, f=14336, r=16, alpha=16.0)  # batch 4 x seq 2048
+
+# rank / length sweep at the 8B width (batch 1, long rows); alpha = 16 throughout
+SWEEP = [Shape(T=T, d=4096, f=14336, r=r, alpha=16.0)
+         for r in (8, 16, 32, 64, 128) for T in (512, 2048, 8192, 32768)]
+
+QBLOCK = 64  # 4-bit blockwise quantisation block size
+
+
+def algorithmic_flops(s: Shape) -> float:
+    """Dense 12*T*d*f (6 fwd + 6 bwd, frozen W gets no gradient) + LoRA 18*T*r*(d+f)."""
+    return 12.0 * s.T * s.d * s.f + 18.0 * s.T * s.r * (s.d + s.f)

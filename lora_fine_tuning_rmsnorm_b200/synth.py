@@ -1,0 +1,120 @@
+"""Seeded synthetic inputs for the LoRA-MLP sub-block.
+
+This module is shared by the CUDA path's tests/bench and by the fp64 oracle's
+tests.  It draws random numbers and rounds them to bf16; it contains none of the
+method's arithmetic (no norm, no projection, no activation).
+
+Recipe (one stream per tensor, fixed order):
+  base seed 3407 (the seed the pages use in their training scripts,
+  "Unsloth 深度实战", §3.2 and "【编译】结合 Unsloth 与 🤗 TRL", §三);
+  tensor k in the order X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, dY draws from
+  numpy Generator(PCG64(SeedSequence([3407, k]))).
+
+Distributions (the workload descriptions of the LoRA-MLP configs):
+  X ~ N(0,1) [T x d];  w ~ 1 + N(0, 0.1) [d];
+  Wg, Wu ~ N(0, 0.02) [f x d];  Wd ~ N(0, 0.02) [d x f];
+  A ~ kaiming-uniform(a=sqrt(5)) on [r x in] = U(-1/sqrt(in), 1/sqrt(in))
+      ("Unsloth 深度实战", §1.3: A random Kaiming-uniform, B zero at init);
+  B ~ N(0, 0.01) [out x r] (non-zero so the adapter gradients are non-trivial);
+  dY ~ N(0, 1) [T x d].
+Every value is drawn in fp64, rounded to fp32, then to bf16 with
+round-to-nearest-even on the bit pattern; the same bits go to both sides.
+"""
+from __future__ import annotations
+
+import dataclasses
+import numpy as np
+
+BASE_SEED = 3407
+TENSOR_ORDER = ("X", "w", "Wg", "Wu", "Wd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd", "dY")
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (round-to-nearest-even), returned as uint16 bits."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32).astype(np.uint64)
+    nan = np.isnan(a)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    if nan.any():
+        r[nan] = 0x7FC0
+    return r
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+@dataclasses.dataclass(frozen=True)
+class Shape:
+    T: int
+    d: int
+    f: int
+    r: int
+    alpha: float = 16.0
+    eps: float = 1e-6
+
+    @property
+    def scale(self) -> float:
+        # the LoRA scaling alpha / r ("Unsloth 深度实战", §1.3, LoRALayer)
+        return self.alpha / self.r
+
+
+def _rng(k: int, seed: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, k])))
+
+
+def _normal(k, seed, shape, mean, std):
+    return mean + std * _rng(k, seed).standard_normal(size=shape, dtype=np.float64)
+
+
+def _uniform(k, seed, shape, bound):
+    return _rng(k, seed).uniform(-bound, bound, size=shape)
+
+
+def tensor_f64(name: str, s: Shape, seed: int = BASE_SEED) -> np.ndarray:
+    """Draw one tensor in fp64, before bf16 rounding."""
+    k = TENSOR_ORDER.index(name)
+    T, d, f, r = s.T, s.d, s.f, s.r
+    if name == "X":
+        return _normal(k, seed, (T, d), 0.0, 1.0)
+    if name == "w":
+        return _normal(k, seed, (d,), 1.0, 0.1)
+    if name in ("Wg", "Wu"):
+        return _normal(k, seed, (f, d), 0.0, 0.02)
+    if name == "Wd":
+        return _normal(k, seed, (d, f), 0.0, 0.02)
+    if name in ("Ag", "Au"):
+        return _uniform(k, seed, (r, d), 1.0 / np.sqrt(d))
+    if name == "Ad":
+        return _uniform(k, seed, (r, f), 1.0 / np.sqrt(f))
+    if name in ("Bg", "Bu"):
+        return _normal(k, seed, (f, r), 0.0, 0.01)
+    if name == "Bd":
+        return _normal(k, seed, (d, r), 0.0, 0.01)
+    if name == "dY":
+        return _normal(k, seed, (T, d), 0.0, 1.0)
+    raise KeyError(name)
+
+
+def make_inputs_bits(s: Shape, seed: int = BASE_SEED, names=TENSOR_ORDER) -> dict:
+    """All inputs as bf16 bit arrays (uint16), keyed by name."""
+    return {n: f32_to_bf16_bits(tensor_f64(n, s, seed).astype(np.float32)) for n in names}
+
+
+def bits_to_f64(bits: dict) -> dict:
+    return {k: bf16_bits_to_f64(v) for k, v in bits.items()}
+
+
+def row_slice_bits(bits: dict, rows) -> dict:
+    """Restrict the per-token tensors (X, dY) to a subset of rows."""
+    out = dict(bits)
+    for k in ("X", "dY"):
+        if k in out:
+            out[k] = np.ascontiguousarray(out[k][rows])
+    return out

@@ -1,0 +1,144 @@
+"""fp64 CPU oracle for the LoRA-augmented Llama MLP sub-block, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
+CPU-baseline / reference arm may import or call anything under oracle/.  The CUDA
+product path never does, and shares no code with it.
+
+What it computes (plain definitions, float64, no rounding anywhere; bf16 inputs
+are taken exactly):
+
+  RMSNorm with cached rstd ("Unsloth提速秘诀：Triton内核如何加速反向传播", §3.2,
+  the _rms_norm_forward_kernel description): mean of squares over the true column
+  count, eps inside the square root, rstd kept for the backward, y = x * rstd * w.
+  No bias (Llama), norm weight frozen.
+
+  LoRA linear ("Unsloth 深度实战", §1.3, LoRALayer / LinearWithLoRA):
+  y = x W^T + s (x A^T) B^T with A [r x in], B [out x r], s = alpha / r, base W frozen,
+  no dropout (the fast path needs lora_dropout == 0: "Unsloth — 用手写 Triton kernel
+  给 HF 微调换心脏", §5).
+
+  SwiGLU MLP ("Unsloth — 用手写 Triton kernel 给 HF 微调换心脏", §2.3 and §7,
+  swiglu_fg_kernel / LoRA_MLP): act = silu(gate) * up, silu(z) = z * sigmoid(z),
+  then the LoRA-augmented down projection.  No residual connection: Y = MLP(RMSNorm(X)).
+
+  Backward: the closed-form chain rule of the same expressions (the pages name a
+  hand-derived LoRA_MLP backward that writes gradients directly, §4 of the same
+  page, and the SiLU derivative, "Unsloth提速秘诀…", §2.2); gradients for X and for
+  the six adapter matrices only (W and the norm weight are frozen).
+
+Rows are independent in every step except the adapter-gradient reductions over T,
+so long inputs are processed in row chunks with fp64 accumulation across chunks.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def sigmoid(z):
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z):
+    return z * sigmoid(z)
+
+
+def silu_grad(z):
+    """d/dz [z * sigmoid(z)] = sigmoid(z) * (1 + z * (1 - sigmoid(z)))."""
+    sg = sigmoid(z)
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def rmsnorm_fwd(X, w, eps):
+    """rstd_t = 1/sqrt(mean_j x_tj^2 + eps);  H = X * rstd[:, None] * w."""
+    ms = np.mean(X * X, axis=1)
+    rstd = 1.0 / np.sqrt(ms + eps)
+    H = X * rstd[:, None] * w[None, :]
+    return H, rstd
+
+
+def rmsnorm_bwd(dH, X, w, rstd):
+    """dX for H = X * rstd * w (rstd depending on X), using the cached rstd.
+
+    With g = dH * w and xhat = X * rstd:  dX = rstd * (g - xhat * mean_j(g * xhat)).
+    """
+    g = dH * w[None, :]
+    xhat = X * rstd[:, None]
+    c = np.mean(g * xhat, axis=1)
+    return rstd[:, None] * (g - xhat * c[:, None])
+
+
+def lora_linear(x, W, A, B, s):
+    """x W^T + s * (x A^T) B^T, in the pages' order (x @ A.T @ B.T * scaling)."""
+    return x @ W.T + s * ((x @ A.T) @ B.T)
+
+
+def forward(X, w, eps, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
+    """Full forward; returns every intermediate the backward needs."""
+    H, rstd = rmsnorm_fwd(X, w, eps)
+    Pg = H @ Ag.T
+    Pu = H @ Au.T
+    G = H @ Wg.T + s * (Pg @ Bg.T)
+    U = H @ Wu.T + s * (Pu @ Bu.T)
+    Act = silu(G) * U
+    Pd = Act @ Ad.T
+    Y = Act @ Wd.T + s * (Pd @ Bd.T)
+    return dict(rstd=rstd, H=H, G=G, U=U, Act=Act, Pg=Pg, Pu=Pu, Pd=Pd, Y=Y)
+
+
+def backward(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
+    """Gradients of <dY, Y> w.r.t. X and the six adapter matrices."""
+    H, G, U, Act = fw["H"], fw["G"], fw["U"], fw["Act"]
+    Pg, Pu, Pd = fw["Pg"], fw["Pu"], fw["Pd"]
+    # down projection  Y = Act Wd^T + s (Act Ad^T) Bd^T
+    Qd = dY @ Bd                      # [T x r]
+    dBd = s * (dY.T @ Pd)             # [d x r]
+    dAd = s * (Qd.T @ Act)            # [r x f]
+    dAct = dY @ Wd + s * (Qd @ Ad)    # [T x f]
+    # SwiGLU  Act = silu(G) * U
+    dG = dAct * U * silu_grad(G)
+    dU = dAct * silu(G)
+    # gate / up projections  G = H Wg^T + s (H Ag^T) Bg^T  (same for U)
+    Qg = dG @ Bg
+    Qu = dU @ Bu
+    dBg = s * (dG.T @ Pg)
+    dBu = s * (dU.T @ Pu)
+    dAg = s * (Qg.T @ H)
+    dAu = s * (Qu.T @ H)
+    dH = dG @ Wg + dU @ Wu + s * (Qg @ Ag + Qu @ Au)
+    dX = rmsnorm_bwd(dH, X, w, fw["rstd"])
+    return dict(dX=dX, dAg=dAg, dBg=dBg, dAu=dAu, dBu=dBu, dAd=dAd, dBd=dBd,
+                dAct=dAct, dG=dG, dU=dU, dH=dH, Qd=Qd, Qg=Qg, Qu=Qu)
+
+
+_GRADS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
+
+
+def fwd_bwd(inp: dict, s: float, eps: float, chunk: int = 2048, keep=("Y", "dX")):
+    """Forward + backward over all rows in chunks of `chunk` tokens.
+
+    `inp` holds fp64 arrays X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, dY.
+    Returns the per-row tensors named in `keep` (concatenated over chunks) and the
+    six adapter gradients summed over all rows.
+    """
+    X, dY = inp["X"], inp["dY"]
+    W = {k: inp[k] for k in ("w", "Wg", "Wu", "Wd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    T = X.shape[0]
+    grads = None
+    rows = {k: [] for k in keep}
+    for t0 in range(0, T, chunk):
+        xs, dys = X[t0:t0 + chunk], dY[t0:t0 + chunk]
+        fw = forward(xs, W["w"], eps, W["Wg"], W["Wu"], W["Wd"], W["Ag"], W["Bg"],
+                     W["Au"], W["Bu"], W["Ad"], W["Bd"], s)
+        bw = backward(fw, dys, xs, W["w"], W["Wg"], W["Wu"], W["Wd"], W["Ag"], W["Bg"],
+                      W["Au"], W["Bu"], W["Ad"], W["Bd"], s)
+        both = {**fw, **bw}
+        for k in keep:
+            rows[k].append(both[k])
+        if grads is None:
+            grads = {k: bw[k].copy() for k in _GRADS}
+        else:
+            for k in _GRADS:
+                grads[k] += bw[k]
+    out = {k: np.concatenate(v, axis=0) for k, v in rows.items()}
+    out.update(grads)
+    return out
