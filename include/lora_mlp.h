@@ -1,0 +1,197 @@
+/*
+ * lora_mlp.h — C ABI of the B200 (sm_100a) LoRA-augmented Llama MLP sub-block.
+ *
+ *   H   = RMSNorm(X; w, eps)                (cached rstd per row)
+ *   G   = H Wg^T + s (H Ag^T) Bg^T           U = H Wu^T + s (H Au^T) Bu^T
+ *   Act = silu(G) * U                        silu(z) = z * sigmoid(z)
+ *   Y   = Act Wd^T + s (Act Ad^T) Bd^T
+ * and the hand-derived backward giving dX and the six adapter gradients
+ * (W, the norm weight and eps are frozen; no autograd).
+ *
+ * Sources of the definitions (web pages on Unsloth-style LoRA fine-tuning):
+ *   RMSNorm with cached rstd, mean over the true column count, eps inside the sqrt:
+ *     "Unsloth提速秘诀：Triton内核如何加速反向传播", §3.2 (FastRMSNorm).
+ *   LoRA linear x W^T + (x A^T) B^T * (alpha / r), A [r x in], B [out x r], frozen W:
+ *     "Unsloth 深度实战：Triton 内核 + 手写反向传播引擎…", §1.3 (LoRALayer, LinearWithLoRA).
+ *   SwiGLU MLP with a hand-written LoRA_MLP autograd that saves only X, e, g, and the
+ *   4-bit dequantise-then-matmul path (matmul_lora / fast_dequantize):
+ *     "Unsloth — 用手写 Triton kernel 给 HF 微调换心脏", §2.3, §4, §7.
+ *   4-bit NormalFloat storage with normal-quantile codes, dequantisation fused with the
+ *   matmul: "Unsloth 深度实战…", §1.4; "Unsloth加速原理揭秘：为何训练快5-8倍？", §5.2.
+ *
+ * Conventions (all entry points):
+ *   - Matrices are row-major.  bf16 tensors are passed as `const void*` to 16-bit
+ *     elements (IEEE bfloat16 bit patterns); fp32 tensors as float*.
+ *   - All pointers are DEVICE pointers (cudaMalloc'd or equivalent) unless stated,
+ *     and must be 16-byte aligned.  The caller owns every buffer; the library
+ *     allocates no device memory.  Inputs are never written.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call only enqueues work on that stream and returns; it does not
+ *     synchronise (except with LORA_MLP_DEBUG=1 in the environment, where each call
+ *     synchronises the stream and reports device-side errors).
+ *   - Return value 0 (LORA_OK) on success or a negative LORA_ERR_* code; no C++
+ *     exception or abort crosses the ABI.  lora_mlp_last_error() then gives a
+ *     thread-local message.
+ *   - Calls on different streams may run concurrently if their output, ctx and
+ *     workspace buffers differ.
+ */
+#ifndef LORA_MLP_H
+#define LORA_MLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum lora_status {
+  LORA_OK = 0,
+  LORA_ERR_INVALID_ARG = -1, /* null pointer, non-positive or inconsistent size      */
+  LORA_ERR_ALIGNMENT = -2,   /* pointer not 16-B aligned; d, f, r not multiples of 8 */
+  LORA_ERR_UNSUPPORTED = -3, /* size outside the supported range (see each call)     */
+  LORA_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (message has text)  */
+  LORA_ERR_TIMEOUT = -5      /* a bounded device-side wait gave up (debug mode only) */
+};
+
+enum lora_wfmt {
+  LORA_WFMT_BF16 = 0, /* frozen Wg, Wu, Wd given as bf16                              */
+  LORA_WFMT_4BIT = 1  /* frozen weights given as 4-bit blockwise codes (qblock = 64)  */
+};
+
+/* Problem sizes.  T tokens, hidden d, intermediate f, LoRA rank r.
+ * Limits: 1 <= T < 2^31; d, f multiples of 8 with 8 <= d <= 65536, 8 <= f;
+ * r a multiple of 8 with 8 <= r <= 256.  scale = alpha / r (any finite value).
+ * wfmt = LORA_WFMT_BF16 or LORA_WFMT_4BIT (then qblock must be 64 and d, f
+ * multiples of 64). */
+typedef struct lora_mlp_dims {
+  int64_t T;
+  int32_t d, f, r;
+  float eps;
+  float scale;
+  int32_t wfmt;
+  int32_t qblock;
+} lora_mlp_dims;
+
+/* Frozen base weights, nn.Linear layout (out x in):
+ *   Wg, Wu [f x d], Wd [d x f]              bf16       (wfmt = LORA_WFMT_BF16)
+ *   Qg, Qu [f*d/2], Qd [d*f/2] bytes        two 4-bit codes per byte, the even element of
+ *                                           the row-major matrix in the low nibble
+ *   absmax_g, absmax_u [f*d/64], absmax_d [d*f/64]  fp32 per-block absmax
+ *   codebook [16] fp32                      code values (wfmt = LORA_WFMT_4BIT)
+ * Unused members may be NULL. */
+typedef struct lora_mlp_weights {
+  const void* Wg;
+  const void* Wu;
+  const void* Wd;
+  const uint8_t* Qg;
+  const uint8_t* Qu;
+  const uint8_t* Qd;
+  const float* absmax_g;
+  const float* absmax_u;
+  const float* absmax_d;
+  const float* codebook;
+} lora_mlp_weights;
+
+/* LoRA adapters, bf16: Ag, Au [r x d]; Bg, Bu [f x r]; Ad [r x f]; Bd [d x r]. */
+typedef struct lora_mlp_adapters {
+  const void* Ag;
+  const void* Bg;
+  const void* Au;
+  const void* Bu;
+  const void* Ad;
+  const void* Bd;
+} lora_mlp_adapters;
+
+/* Adapter gradients, fp32, same shapes as the adapters.  OVERWRITTEN by the
+ * backward (not accumulated).  Sums over T are formed with fp32 atomics, so the
+ * last bits may differ between runs. */
+typedef struct lora_mlp_grads {
+  float* dAg;
+  float* dBg;
+  float* dAu;
+  float* dBu;
+  float* dAd;
+  float* dBd;
+} lora_mlp_grads;
+
+/* Byte offsets of the saved-activation context (one caller-owned device buffer,
+ * written by lora_mlp_fwd, read by lora_mlp_bwd).  rp = r rounded up to 16.
+ *   rstd [T] fp32;  H [T x d] bf16 (normalised input);  G, U, Act [T x f] bf16;
+ *   P [T x 2rp] bf16 = s*(H Ag^T | 0 | H Au^T | 0), columns [0,r) and [rp, rp+r);
+ *   Pd [T x rp] bf16 = s*(Act Ad^T | 0).
+ * Offsets are multiples of 256. */
+typedef struct lora_mlp_ctx_layout {
+  size_t rstd, H, G, U, Act, P, Pd;
+  size_t total;
+  int32_t rp;
+} lora_mlp_ctx_layout;
+
+/* Saved-context size and layout for `dims`.  Returns LORA_ERR_* on bad dims. */
+int lora_mlp_ctx_layout_get(const lora_mlp_dims* dims, lora_mlp_ctx_layout* out);
+
+/* Workspace bytes needed by lora_mlp_fwd / lora_mlp_bwd (one buffer serves both;
+ * it holds the backward's dH fp32 [T x d], dG, dU bf16 [T x f], the rank-r
+ * projections and a device status word).  Contents need not be initialised. */
+int lora_mlp_workspace_bytes(const lora_mlp_dims* dims, size_t* bytes);
+
+/* Forward.  X [T x d] bf16, rms_w [d] bf16 -> Y [T x d] bf16, and the saved context
+ * `ctx` (lora_mlp_ctx_layout_get().total bytes).  `workspace` as above.
+ * Errors: INVALID_ARG (null/inconsistent), ALIGNMENT, UNSUPPORTED, CUDA. */
+int lora_mlp_fwd(const lora_mlp_dims* dims, const void* X, const void* rms_w,
+                 const lora_mlp_weights* W, const lora_mlp_adapters* A, void* Y, void* ctx,
+                 void* workspace, void* stream);
+
+/* Backward.  dY [T x d] bf16 plus the forward's X, rms_w, weights, adapters and ctx
+ * -> dX [T x d] bf16 and the six fp32 adapter gradients (overwritten).
+ * The gradient of <dY, Y>:
+ *   dAct = dY Wd + s (dY Bd) Ad;  dG = dAct * U * silu'(G);  dU = dAct * silu(G);
+ *   dH = dG Wg + dU Wu + s ((dG Bg) Ag + (dU Bu) Au);  dX = RMSNorm'(dH);
+ *   dBg = s dG^T (H Ag^T), dAg = s (dG Bg)^T H, and likewise for u and d. */
+int lora_mlp_bwd(const lora_mlp_dims* dims, const void* dY, const void* X, const void* rms_w,
+                 const lora_mlp_weights* W, const lora_mlp_adapters* A, const void* ctx,
+                 void* dX, const lora_mlp_grads* grads, void* workspace, void* stream);
+
+/* RMSNorm forward alone: H = X * rstd * w, rstd = 1/sqrt(mean(X^2) + eps) in fp32.
+ * X, H [T x d] bf16, w [d] bf16, rstd [T] fp32.  d a multiple of 8, <= 65536. */
+int lora_rmsnorm_fwd(int64_t T, int32_t d, float eps, const void* X, const void* w, void* H,
+                     float* rstd, void* stream);
+
+/* RMSNorm backward alone (weight frozen): dX = rstd * (g - xhat * mean(g * xhat)),
+ * g = dH * w, xhat = X * rstd.  dH [T x d] fp32, X [T x d] bf16, w [d] bf16,
+ * rstd [T] fp32 (from the forward) -> dX [T x d] bf16. */
+int lora_rmsnorm_bwd(int64_t T, int32_t d, const float* dH, const void* X, const void* w,
+                     const float* rstd, void* dX, void* stream);
+
+/* 4-bit blockwise quantisation of a bf16 matrix (flattened row-major, numel a
+ * multiple of block = 64): per block absmax = max|w| (fp32); code index
+ * idx = #{ i in 0..14 : w > absmax * m_i }, m_i = fl32((c_i + c_{i+1}) / 2), decided
+ * exactly (nearest code, ties to the lower index; all-zero block -> 0).  codebook16
+ * [16] fp32 ascending.  codes [numel/2] bytes (even element in the low nibble),
+ * absmax [numel/64] fp32. */
+int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float* codebook16,
+                       uint8_t* codes, float* absmax, void* stream);
+
+/* Plain tensor-core GEMM (the core the fused path is built on), fp32 out:
+ *   C[M x N] = A' B'^T,  A' [M x K] = A (a_mn = 0, A row-major [M x K]) or A^T
+ *   (a_mn = 1, A row-major [K x M]);  B' [N x K] = B (b_mn = 0, B [N x K]) or B^T
+ *   (b_mn = 1, B [K x N]).  The contiguous dimension must be a multiple of 8. */
+int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B,
+                   int32_t b_mn, float* C, void* stream);
+
+/* Per-phase timing.  With timing enabled, every kernel launch of the calls above
+ * is bracketed by CUDA events on the caller's stream.  lora_mlp_timing_collect()
+ * synchronises those events and returns, per phase id, the summed milliseconds and
+ * the number of launches since the previous collect (arrays of LORA_NUM_PHASES). */
+#define LORA_NUM_PHASES 16
+int lora_mlp_timing_enable(int32_t on);
+int lora_mlp_timing_collect(double* ms, int64_t* launches);
+const char* lora_mlp_phase_name(int32_t phase);
+
+/* Thread-local description of the last error (never NULL). */
+const char* lora_mlp_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LORA_MLP_H */

@@ -1,0 +1,473 @@
+// Warp-specialised, persistent tcgen05 GEMM for sm_100a with TMA-fed operands,
+// TMEM accumulators and fused epilogues.  One kernel template serves every
+// contraction of the LoRA-MLP forward/backward:
+//
+//   D_a[m, n] = sum over segments s feeding accumulator a of
+//               sum_k  A_s[m, a_k0 + k] * B_{s,a}[n, b_k0 + k],   k in [0, k_len_s)
+//
+// A "segment" is a K range with its own A and B tensor maps, so the LoRA rank-r
+// term is folded into the same accumulator as one short extra K range
+// ([H | s P] x [W | B]^T), and gate/up share one A tile with two accumulators
+// (NACC = 2).  Operands are bf16, 128-byte swizzled in shared memory, either
+// K-major (x = K innermost) or MN-major (x = M/N innermost); out-of-range boxes
+// are zero-filled by TMA, which also pads ragged K tails and rank r to 16.
+//
+// CTA = 6 warps: warp 0 issues TMA loads into a `stages`-deep ring, warp 1 owns
+// TMEM and issues tcgen05.mma from one thread, warps 2..5 drain the double-
+// buffered TMEM accumulators (tcgen05.ld) through the epilogue while the next
+// tile's main loop runs.  Tile order is M-fastest over a persistent grid.
+#pragma once
+#include "ptx.cuh"
+
+namespace lm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kMaxStages = 8;
+constexpr int kMaxSegs = 4;
+constexpr int kMaxMaps = 8;
+constexpr int kGemmThreads = 192;
+
+enum Epi : int {
+  EPI_F32 = 0,         // out[0] fp32 = acc * alpha
+  EPI_BF16 = 1,        // out[0] bf16 = acc_a * alpha, accumulator a at column a * out_acc_col
+  EPI_SWIGLU_FWD = 2,  // acc0 = G, acc1 = U -> out[0] G, out[1] U, out[2] silu(G) * U (bf16)
+  EPI_SWIGLU_BWD = 3,  // acc0 = dAct; in[0] G, in[1] U -> out[0] dG, out[1] dU (bf16)
+  EPI_ATOMIC = 4       // rows [lo, hi) of an accumulator atomically added into fp32 outputs
+};
+
+struct Seg {
+  int a_map;
+  int a_k0;
+  int b_map[2];  // -1: this segment does not feed that accumulator
+  int b_k0[2];
+  int k_len;
+};
+
+struct OutRange {
+  float* out;
+  int acc;
+  int lo, hi;     // accumulator rows (global M index) routed to `out`
+  int trans;      // 0: out[(m - lo) * ld + n]; 1: out[n * ld + (m - lo)]
+  long long ld;
+};
+
+struct GemmArgs {
+  CUtensorMap maps[kMaxMaps];
+  Seg seg[kMaxSegs];
+  int nseg;
+  int M, N;  // valid rows / valid columns per accumulator
+  int bn;    // N tile per accumulator (multiple of 16; multiple of 64 when B is MN-major)
+  int tiles_m, tiles_n, splits;
+  int k_chunk;  // split-K chunk in elements (multiple of BK) when splits > 1
+  int stages;
+  uint32_t stage_bytes;
+  uint32_t tmem_cols;
+  void* out[3];
+  long long ld_out;
+  int out_acc_col;
+  float alpha;
+  const void* in[2];
+  long long ld_in;
+  OutRange rng[2];
+  int nrng;
+  int* status;
+  unsigned long long limit_ns;
+};
+
+__device__ __forceinline__ void decode_tile(const GemmArgs& p, int t, int& mt, int& nt, int& ks) {
+  mt = t % p.tiles_m;
+  t /= p.tiles_m;
+  nt = t % p.tiles_n;
+  ks = t / p.tiles_n;
+}
+
+__device__ __forceinline__ void seg_kb_range(const GemmArgs& p, int s, int ks, int& lo, int& hi) {
+  const int nkb = (p.seg[s].k_len + BK - 1) / BK;
+  if (p.splits > 1) {
+    const int per = p.k_chunk / BK;
+    lo = ks * per;
+    hi = min(nkb, lo + per);
+  } else {
+    lo = 0;
+    hi = nkb;
+  }
+}
+
+// Drain wait used after an abort: ignores the abort flag, bounded by the limit.
+__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const WaitCtl& c) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_test(bar, parity)) {
+    if (global_ns() - t0 > c.limit_ns) {
+      if (c.status) atomicCAS(c.status, 0, kDevTimeoutDrain);
+      return;
+    }
+  }
+}
+
+template <int A_MN, int B_MN, int NACC>
+__device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
+                                              uint32_t empty0, const WaitCtl& wc) {
+  const int total = p.tiles_m * p.tiles_n * p.splits;
+  int stage = 0;
+  uint32_t phase = 0;
+  uint32_t issued_mask = 0, issued_par = 0;
+  const uint32_t a_bytes = BM * BK * 2;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
+  bool ok = true;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    int mt, nt, ks;
+    decode_tile(p, t, mt, nt, ks);
+    const int m0 = mt * BM, n0 = nt * p.bn;
+    for (int s = 0; s < p.nseg && ok; ++s) {
+      const Seg& sg = p.seg[s];
+      int kb0, kb1;
+      seg_kb_range(p, s, ks, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t full = full0 + 8 * stage, empty = empty0 + 8 * stage;
+        if (!mbar_wait(empty, phase ^ 1, wc, kDevTimeoutProducer)) {
+          ok = false;
+          break;
+        }
+        // Boxes that would lie entirely outside the matrix are skipped: the rows /
+        // columns they would feed are never stored by the epilogue.
+        const int nA = A_MN ? ((m0 + 64 < p.M) ? 2 : 1) : 1;
+        int nBc = B_MN ? 0 : 1;
+        if (B_MN) {
+          for (int c = 0; c < p.bn / 64; ++c)
+            if (n0 + 64 * c < p.N) ++nBc;
+        }
+        uint32_t bytes = static_cast<uint32_t>(nA) * (A_MN ? 8192u : a_bytes);
+#pragma unroll
+        for (int a = 0; a < NACC; ++a)
+          if (sg.b_map[a] >= 0) bytes += B_MN ? static_cast<uint32_t>(nBc) * 8192u : b_bytes;
+        mbar_expect_tx(full, bytes);
+        const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
+        const int k = kb * BK;
+        const CUtensorMap* am = &p.maps[sg.a_map];
+        if (A_MN) {
+          tma_load_2d(sA, am, full, m0, sg.a_k0 + k);
+          if (nA == 2) tma_load_2d(sA + 8192, am, full, m0 + 64, sg.a_k0 + k);
+        } else {
+          tma_load_2d(sA, am, full, sg.a_k0 + k, m0);
+        }
+#pragma unroll
+        for (int a = 0; a < NACC; ++a) {
+          if (sg.b_map[a] < 0) continue;
+          const uint32_t sB = sA + a_bytes + a * b_bytes;
+          const CUtensorMap* bm = &p.maps[sg.b_map[a]];
+          if (B_MN) {
+            for (int c = 0; c < nBc; ++c)
+              tma_load_2d(sB + c * 8192, bm, full, n0 + 64 * c, sg.b_k0[a] + k);
+          } else {
+            tma_load_2d(sB, bm, full, sg.b_k0[a] + k, n0);
+          }
+        }
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  }
+  if (!ok) {
+    // Aborting: make sure no TMA write into shared memory is still in flight.
+    for (int s = 0; s < p.stages; ++s)
+      if (issued_mask & (1u << s)) drain_wait(full0 + 8 * s, (issued_par >> s) & 1, wc);
+  }
+}
+
+template <int A_MN, int B_MN, int NACC>
+__device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
+                                         uint32_t empty0, uint32_t tfull0, uint32_t tempty0,
+                                         uint32_t drain_bar, uint32_t tmem_base,
+                                         const WaitCtl& wc) {
+  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const uint32_t idesc = idesc_bf16(BM, p.bn, A_MN, B_MN);
+  const uint32_t a_bytes = BM * BK * 2;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
+  int stage = 0;
+  uint32_t phase = 0;
+  uint32_t it = 0;
+  bool ok = true, issued_any = false;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+    int mt, nt, ks;
+    decode_tile(p, t, mt, nt, ks);
+    const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
+    if (!mbar_wait(tempty0 + 8 * buf, aphase ^ 1, wc, kDevTimeoutMma)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    uint32_t started = 0;
+    for (int s = 0; s < p.nseg && ok; ++s) {
+      const Seg& sg = p.seg[s];
+      int kb0, kb1;
+      seg_kb_range(p, s, ks, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int rem = sg.k_len - kb * BK;
+        const int nsteps = rem >= BK ? BK / 16 : (rem + 15) / 16;
+        const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
+#pragma unroll
+        for (int a = 0; a < NACC; ++a) {
+          if (sg.b_map[a] < 0) continue;
+          const uint32_t sB = sA + a_bytes + a * b_bytes;
+          const uint32_t d = tmem_base + buf * (NACC * p.bn) + a * p.bn;
+          for (int j = 0; j < nsteps; ++j) {
+            const uint64_t ad = A_MN ? sdesc_sw128(sA + j * 2048, 8192, 1024)
+                                     : sdesc_sw128(sA + j * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(sB + j * 2048, 8192, 1024)
+                                     : sdesc_sw128(sB + j * 32, 16, 1024);
+            mma_bf16(d, ad, bd, idesc, (started >> a) & 1);
+            started |= 1u << a;
+            issued_any = true;
+          }
+        }
+        mma_commit(empty0 + 8 * stage);  // frees the smem stage once these MMAs finish
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (ok) mma_commit(tfull0 + 8 * buf);  // accumulator ready for the epilogue
+  }
+  if (!ok && issued_any) {
+    // Aborting: wait for the MMAs already issued before TMEM is released.
+    mma_commit(drain_bar);
+    drain_wait(drain_bar, 0, wc);
+  }
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <int NACC, int EPI>
+__device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0, uint32_t tempty0,
+                                              uint32_t tmem_base, const WaitCtl& wc) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int q = warp & 3;  // TMEM lane quarter this warp may access
+  const int total = p.tiles_m * p.tiles_n * p.splits;
+  uint32_t it = 0;
+  for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+    int mt, nt, ks;
+    decode_tile(p, t, mt, nt, ks);
+    const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(tfull0 + 8 * buf, aphase, wc, kDevTimeoutEpilogue) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    tc_fence_after();
+    const int m0 = mt * BM, n0 = nt * p.bn;
+    const long long row = static_cast<long long>(m0) + 32 * q + lane;
+    const bool row_ok = row < p.M;
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (NACC * p.bn);
+
+    if (EPI == EPI_F32 || EPI == EPI_BF16) {
+#pragma unroll 1
+      for (int a = 0; a < NACC; ++a) {
+#pragma unroll 1
+        for (int c = 0; c < p.bn; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + a * p.bn + c, r);
+          tmem_wait16(r);
+          const int n = n0 + c;
+          if (!row_ok) continue;
+          if (EPI == EPI_F32) {
+            float* o = static_cast<float*>(p.out[0]) + row * p.ld_out + n;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              if (n + 4 * h < p.N) {
+                float4 v = make_float4(__uint_as_float(r[4 * h]) * p.alpha,
+                                       __uint_as_float(r[4 * h + 1]) * p.alpha,
+                                       __uint_as_float(r[4 * h + 2]) * p.alpha,
+                                       __uint_as_float(r[4 * h + 3]) * p.alpha);
+                *reinterpret_cast<float4*>(o + 4 * h) = v;
+              }
+            }
+          } else {
+            uint16_t* o = static_cast<uint16_t*>(p.out[0]) + row * p.ld_out + a * p.out_acc_col + n;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (n + 8 * h < p.N) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(r[8 * h + 0]) * p.alpha, __uint_as_float(r[8 * h + 1]) * p.alpha);
+                v.y = pack_bf16x2(__uint_as_float(r[8 * h + 2]) * p.alpha, __uint_as_float(r[8 * h + 3]) * p.alpha);
+                v.z = pack_bf16x2(__uint_as_float(r[8 * h + 4]) * p.alpha, __uint_as_float(r[8 * h + 5]) * p.alpha);
+                v.w = pack_bf16x2(__uint_as_float(r[8 * h + 6]) * p.alpha, __uint_as_float(r[8 * h + 7]) * p.alpha);
+                *reinterpret_cast<uint4*>(o + 8 * h) = v;
+              }
+            }
+          }
+        }
+      }
+    } else if (EPI == EPI_SWIGLU_FWD) {
+#pragma unroll 1
+      for (int c = 0; c < p.bn; c += 16) {
+        uint32_t rg[16], ru[16];
+        tmem_ld16(tbase + c, rg);
+        tmem_ld16(tbase + p.bn + c, ru);
+        tmem_wait32(rg, ru);
+        const int n = n0 + c;
+        if (!row_ok) continue;
+        const long long off = row * p.ld_out + n;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (n + 8 * h >= p.N) continue;
+          uint32_t pg[4], pu[4], pa[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float g0 = __uint_as_float(rg[8 * h + 2 * j]), g1 = __uint_as_float(rg[8 * h + 2 * j + 1]);
+            const float u0 = __uint_as_float(ru[8 * h + 2 * j]), u1 = __uint_as_float(ru[8 * h + 2 * j + 1]);
+            pg[j] = pack_bf16x2(g0, g1);
+            pu[j] = pack_bf16x2(u0, u1);
+            pa[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+          }
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[2]) + off + 8 * h) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+        }
+      }
+    } else if (EPI == EPI_SWIGLU_BWD) {
+#pragma unroll 1
+      for (int c = 0; c < p.bn; c += 16) {
+        const int n = n0 + c;
+        uint4 gv[2], uv[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (row_ok && n + 8 * h < p.N) {
+            const long long off = row * p.ld_in + n + 8 * h;
+            gv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.in[0]) + off));
+            uv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.in[1]) + off));
+          } else {
+            gv[h] = make_uint4(0, 0, 0, 0);
+            uv[h] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        uint32_t r[16];
+        tmem_ld16(tbase + c, r);
+        tmem_wait16(r);
+        if (!row_ok) continue;
+        const long long off = row * p.ld_out + n;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (n + 8 * h >= p.N) continue;
+          const uint32_t gw[4] = {gv[h].x, gv[h].y, gv[h].z, gv[h].w};
+          const uint32_t uw[4] = {uv[h].x, uv[h].y, uv[h].z, uv[h].w};
+          uint32_t pdg[4], pdu[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float dg[2], du[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float g = e ? bf16hi(gw[j]) : bf16lo(gw[j]);
+              const float u = e ? bf16hi(uw[j]) : bf16lo(uw[j]);
+              const float da = __uint_as_float(r[8 * h + 2 * j + e]);
+              const float sg = 1.0f / (1.0f + __expf(-g));
+              du[e] = da * g * sg;
+              dg[e] = da * u * sg * (1.0f + g * (1.0f - sg));
+            }
+            pdg[j] = pack_bf16x2(dg[0], dg[1]);
+            pdu[j] = pack_bf16x2(du[0], du[1]);
+          }
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h) = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h) = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
+        }
+      }
+    } else if (EPI == EPI_ATOMIC) {
+#pragma unroll 1
+      for (int ri = 0; ri < p.nrng; ++ri) {
+        const OutRange& R = p.rng[ri];
+        const long long wlo = static_cast<long long>(m0) + 32 * q;
+        if (wlo + 31 < R.lo || wlo >= R.hi) continue;  // warp-uniform skip
+        const bool mine = row >= R.lo && row < R.hi;
+        const long long k = row - R.lo;
+#pragma unroll 1
+        for (int c = 0; c < p.bn; c += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + R.acc * p.bn + c, r);
+          tmem_wait16(r);
+          if (!mine) continue;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const long long n = n0 + c + j;
+            if (n < p.N) {
+              float* dst = R.trans ? R.out + n * R.ld + k : R.out + k * R.ld + n;
+              atomicAdd(dst, __uint_as_float(r[j]) * p.alpha);
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+  }
+}
+
+template <int A_MN, int B_MN, int NACC, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + static_cast<size_t>(p.stages) * p.stage_bytes);
+  const int S = p.stages;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * S;
+  const uint32_t tfull0 = empty0 + 8 * S;
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t drain_bar = tempty0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(tfull0, 1);
+    mbar_init(tfull0 + 8, 1);
+    mbar_init(tempty0, 4);
+    mbar_init(tempty0 + 8, 4);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kMaxMaps; ++i) tma_prefetch_desc(&p.maps[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.status, p.limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC>(p, tiles, full0, empty0, wc);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0)
+      gemm_mma<A_MN, B_MN, NACC>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc);
+    __syncwarp();
+  } else {
+    gemm_epilogue<NACC, EPI>(p, tfull0, tempty0, tmem_base, wc);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace lm

@@ -1,0 +1,722 @@
+// Host side of liblora_mlp.so: argument validation, TMA tensor-map construction,
+// the launch sequence of the LoRA-MLP forward/backward, per-phase timing and the
+// extern "C" entry points declared in include/lora_mlp.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lora_mlp.h"
+#include "gemm_sm100.cuh"
+#include "rowops.cuh"
+
+using namespace lm;
+
+namespace {
+
+thread_local char g_err[512] = "no error";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                   \
+  do {                                                                                   \
+    cudaError_t e_ = (expr);                                                             \
+    if (e_ != cudaSuccess)                                                               \
+      return fail(LORA_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));        \
+  } while (0)
+
+#define TRY(expr)            \
+  do {                       \
+    int rc_ = (expr);        \
+    if (rc_ != LORA_OK) return rc_; \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+bool debug_mode() {
+  static int v = [] {
+    const char* e = getenv("LORA_MLP_DEBUG");
+    return (e && e[0] && e[0] != '0') ? 1 : 0;
+  }();
+  return v != 0;
+}
+
+unsigned long long wait_limit_ns() {
+  const char* e = getenv("LORA_MLP_WAIT_LIMIT_MS");
+  long long ms = e ? atoll(e) : 5000;
+  if (ms < 1) ms = 1;
+  return static_cast<unsigned long long>(ms) * 1000000ull;
+}
+
+// ------------------------------------------------------------------ driver API
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder() {
+  if (g_encode) return LORA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return fail(LORA_ERR_CUDA, "cannot resolve cuTensorMapEncodeTiled");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return LORA_OK;
+}
+
+// 2-D bf16 tensor map, 128-byte swizzle: `inner` contiguous elements per row,
+// `outer` rows `ld` elements apart, box of box_inner x box_outer elements.
+int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+             uint32_t box_inner, uint32_t box_outer) {
+  TRY(get_encoder());
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): inner=%llu outer=%llu ld=%llu box=%ux%u",
+                static_cast<int>(r), (unsigned long long)inner, (unsigned long long)outer,
+                (unsigned long long)ld, box_inner, box_outer);
+  return LORA_OK;
+}
+// Operand with K contiguous: [rows x K], box 64 (K) x box_rows.
+int map_k(CUtensorMap* m, const void* p, uint64_t rows, uint64_t K, uint64_t ld, uint32_t box_rows) {
+  return make_map(m, p, K, rows, ld, 64, box_rows);
+}
+// Operand with M/N contiguous: [K x MN], box 64 (MN) x 64 (K).
+int map_mn(CUtensorMap* m, const void* p, uint64_t K, uint64_t MN, uint64_t ld) {
+  return make_map(m, p, MN, K, ld, 64, 64);
+}
+
+// --------------------------------------------------------------------- timing
+const char* kPhaseNames[LORA_NUM_PHASES] = {
+    "rmsnorm_fwd", "proj_P_gate_up", "gemm_gate_up_swiglu", "proj_P_down", "gemm_down",
+    "proj_Q_down", "gemm_dact_swiglu_bwd", "proj_Q_gate_up", "gemm_dH", "rmsnorm_bwd",
+    "zero_grads", "reduce_dA_gate_up", "reduce_dB_gate_up", "reduce_dB_down", "reduce_dA_down",
+    "other"};
+enum Phase {
+  PH_RMS_FWD = 0, PH_P_GU, PH_GATEUP, PH_P_D, PH_DOWN, PH_Q_D, PH_DACT, PH_Q_GU, PH_DH,
+  PH_RMS_BWD, PH_ZERO, PH_RED_DA_GU, PH_RED_DB_GU, PH_RED_DB_D, PH_RED_DA_D, PH_OTHER
+};
+
+struct Timing {
+  std::mutex mu;
+  bool on = false;
+  struct Rec { cudaEvent_t a, b; int phase; };
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+} g_timing;
+
+struct PhaseScope {
+  cudaStream_t st;
+  int phase;
+  cudaEvent_t a = nullptr, b = nullptr;
+  PhaseScope(cudaStream_t s, int ph) : st(s), phase(ph) {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    if (!g_timing.on) return;
+    a = g_timing.get();
+    b = g_timing.get();
+    cudaEventRecord(a, st);
+  }
+  ~PhaseScope() {
+    if (!a) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    g_timing.pending.push_back({a, b, phase});
+  }
+};
+
+// ------------------------------------------------------------------ launches
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
+
+template <int A_MN, int B_MN, int NACC, int EPI>
+int launch_gemm(GemmArgs& a, cudaStream_t st, int phase, int max_ctas = 0) {
+  if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % 64))
+    return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
+  a.stage_bytes = BM * BK * 2 + NACC * a.bn * BK * 2;
+  const int avail = kSmemLimit - 1024 - 256;
+  a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
+  if (a.stages < 2) return fail(LORA_ERR_UNSUPPORTED, "internal: stage does not fit");
+  int cols = 2 * NACC * a.bn;
+  uint32_t tc = 32;
+  while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
+  if (tc > 512) return fail(LORA_ERR_UNSUPPORTED, "internal: TMEM columns %d > 512", cols);
+  a.tmem_cols = tc;
+  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + 256;
+  // more than half of TMEM per CTA: keep one CTA per SM so allocation never waits
+  if (tc > 256) smem = std::max(smem, kSmemLimit / 2 + 4096);
+  a.limit_ns = wait_limit_ns();
+  const long long tiles = static_cast<long long>(a.tiles_m) * a.tiles_n * a.splits;
+  if (tiles <= 0) return LORA_OK;
+  if (tiles > 0x7fffffffLL) return fail(LORA_ERR_UNSUPPORTED, "too many tiles");
+  int grid = static_cast<int>(std::min<long long>(tiles, max_ctas > 0 ? max_ctas : sm_count()));
+  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI>;
+  CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  PhaseScope ps(st, phase);
+  kern<<<grid, kGemmThreads, smem, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
+
+int launch_rms_fwd(cudaStream_t st, const void* X, const void* w, void* H, float* rstd, long long T, int d,
+                   float eps) {
+  const int nvec = d / 8;
+  int threads = kRowThreads, vpt = (nvec + threads - 1) / threads;
+  if (vpt > 8) {
+    vpt = 8;
+    threads = round_up((nvec + 7) / 8, 32);
+  }
+  if (threads > 1024) return fail(LORA_ERR_UNSUPPORTED, "d = %d too large for the row kernel", d);
+  int v = vpt <= 1 ? 1 : vpt <= 2 ? 2 : vpt <= 4 ? 4 : 8;
+  auto X16 = static_cast<const uint16_t*>(X);
+  auto w16 = static_cast<const uint16_t*>(w);
+  auto H16 = static_cast<uint16_t*>(H);
+  PhaseScope ps(st, PH_RMS_FWD);
+  for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
+    unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
+    switch (v) {
+      case 1: rmsnorm_fwd_kernel<1><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
+      case 2: rmsnorm_fwd_kernel<2><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
+      case 4: rmsnorm_fwd_kernel<4><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
+      default: rmsnorm_fwd_kernel<8><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
+    }
+  }
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
+
+int launch_rms_bwd(cudaStream_t st, const float* dH, const void* X, const void* w, const float* rstd, void* dX,
+                   long long T, int d) {
+  const int nvec = d / 8;
+  int threads = kRowThreads, vpt = (nvec + threads - 1) / threads;
+  if (vpt > 4) {
+    vpt = 4;
+    threads = round_up((nvec + 3) / 4, 32);
+  }
+  if (threads > 1024) return fail(LORA_ERR_UNSUPPORTED, "d = %d too large for the row kernel", d);
+  int v = vpt <= 1 ? 1 : vpt <= 2 ? 2 : 4;
+  auto X16 = static_cast<const uint16_t*>(X);
+  auto w16 = static_cast<const uint16_t*>(w);
+  auto dX16 = static_cast<uint16_t*>(dX);
+  PhaseScope ps(st, PH_RMS_BWD);
+  for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
+    unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
+    switch (v) {
+      case 1: rmsnorm_bwd_kernel<1><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dX16 + r0 * d, d); break;
+      case 2: rmsnorm_bwd_kernel<2><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dX16 + r0 * d, d); break;
+      default: rmsnorm_bwd_kernel<4><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dX16 + r0 * d, d); break;
+    }
+  }
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
+
+// --------------------------------------------------------------- layouts
+struct WsLayout {
+  size_t status, Q, Qd, dG, dU, dH, total;
+};
+
+int check_dims(const lora_mlp_dims* D) {
+  if (!D) return fail(LORA_ERR_INVALID_ARG, "dims is NULL");
+  if (D->T < 1 || D->T >= (1LL << 31)) return fail(LORA_ERR_INVALID_ARG, "T = %lld out of range", (long long)D->T);
+  if (D->d < 8 || D->f < 8 || D->r < 1) return fail(LORA_ERR_INVALID_ARG, "d, f, r must be positive (d, f >= 8)");
+  if (D->d % 8 || D->f % 8 || D->r % 8)
+    return fail(LORA_ERR_ALIGNMENT, "d, f, r must be multiples of 8 (16-byte rows); got %d %d %d", D->d, D->f, D->r);
+  if (D->d > 65536) return fail(LORA_ERR_UNSUPPORTED, "d = %d > 65536", D->d);
+  if (D->r > 128) return fail(LORA_ERR_UNSUPPORTED, "r = %d > 128", D->r);
+  if (D->wfmt != LORA_WFMT_BF16 && D->wfmt != LORA_WFMT_4BIT) return fail(LORA_ERR_INVALID_ARG, "bad wfmt");
+  if (D->wfmt == LORA_WFMT_4BIT) {
+    if (D->qblock != 64) return fail(LORA_ERR_UNSUPPORTED, "qblock must be 64");
+    if (D->d % 64 || D->f % 64) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights need d, f multiples of 64");
+  }
+  return LORA_OK;
+}
+
+int rp_of(const lora_mlp_dims* D) { return round_up(D->r, 16); }
+
+lora_mlp_ctx_layout ctx_layout(const lora_mlp_dims* D) {
+  const size_t T = D->T, d = D->d, f = D->f, rp = rp_of(D);
+  lora_mlp_ctx_layout L{};
+  size_t o = 0;
+  L.rstd = o; o = up256(o + T * 4);
+  L.H = o;    o = up256(o + T * d * 2);
+  L.G = o;    o = up256(o + T * f * 2);
+  L.U = o;    o = up256(o + T * f * 2);
+  L.Act = o;  o = up256(o + T * f * 2);
+  L.P = o;    o = up256(o + T * 2 * rp * 2);
+  L.Pd = o;   o = up256(o + T * rp * 2);
+  L.total = o;
+  L.rp = static_cast<int32_t>(rp);
+  return L;
+}
+
+WsLayout ws_layout(const lora_mlp_dims* D) {
+  const size_t T = D->T, d = D->d, f = D->f, rp = rp_of(D);
+  WsLayout L{};
+  size_t o = 0;
+  L.status = o; o = 256;
+  L.Q = o;  o = up256(o + T * 2 * rp * 2);
+  L.Qd = o; o = up256(o + T * rp * 2);
+  L.dG = o; o = up256(o + T * f * 2);
+  L.dU = o; o = up256(o + T * f * 2);
+  L.dH = o; o = up256(o + T * d * 4);
+  L.total = o;
+  return L;
+}
+
+template <class P>
+P* at(void* base, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(base) + off); }
+template <class P>
+const P* at(const void* base, size_t off) { return reinterpret_cast<const P*>(static_cast<const char*>(base) + off); }
+
+int check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return fail(LORA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned16(p)) return fail(LORA_ERR_ALIGNMENT, "pointer %p is not 16-byte aligned", p);
+  }
+  return LORA_OK;
+}
+
+int begin_call(int* status, cudaStream_t st) {
+  if (debug_mode() && status) CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  return LORA_OK;
+}
+
+int end_call(int* status, cudaStream_t st) {
+  if (!debug_mode()) return LORA_OK;
+  CUDA_TRY(cudaStreamSynchronize(st));
+  if (status) {
+    int v = 0;
+    CUDA_TRY(cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost));
+    if (v) return fail(LORA_ERR_TIMEOUT, "device-side bounded wait gave up (code 0x%x)", v);
+  }
+  return LORA_OK;
+}
+
+GemmArgs new_args(int* status) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.splits = 1;
+  a.alpha = 1.0f;
+  a.status = status;
+  for (int s = 0; s < kMaxSegs; ++s) a.seg[s].b_map[0] = a.seg[s].b_map[1] = -1;
+  return a;
+}
+
+void set_seg(GemmArgs& a, int s, int amap, int ak0, int b0, int bk0, int b1, int bk1, int klen) {
+  a.seg[s].a_map = amap;
+  a.seg[s].a_k0 = ak0;
+  a.seg[s].b_map[0] = b0;
+  a.seg[s].b_k0[0] = bk0;
+  a.seg[s].b_map[1] = b1;
+  a.seg[s].b_k0[1] = bk1;
+  a.seg[s].k_len = klen;
+  a.nseg = std::max(a.nseg, s + 1);
+}
+
+// Split the T reduction so that roughly two CTAs per SM are busy.
+void choose_splits(GemmArgs& a, long long K) {
+  const long long tiles = static_cast<long long>(a.tiles_m) * a.tiles_n;
+  const long long nkb = (K + BK - 1) / BK;
+  long long want = std::max<long long>(1, (2LL * sm_count() + tiles - 1) / tiles);
+  want = std::min(want, nkb);
+  long long per = (nkb + want - 1) / want;
+  a.k_chunk = static_cast<int>(per * BK);
+  a.splits = static_cast<int>((nkb + per - 1) / per);
+}
+
+}  // namespace
+
+// ======================================================================= ABI
+extern "C" {
+
+const char* lora_mlp_last_error(void) { return g_err; }
+
+const char* lora_mlp_phase_name(int32_t phase) {
+  if (phase < 0 || phase >= LORA_NUM_PHASES) return "invalid";
+  return kPhaseNames[phase];
+}
+
+int lora_mlp_timing_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  g_timing.on = on != 0;
+  return LORA_OK;
+}
+
+int lora_mlp_timing_collect(double* ms, int64_t* launches) {
+  std::vector<Timing::Rec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_timing.mu);
+    recs.swap(g_timing.pending);
+  }
+  if (ms)
+    for (int i = 0; i < LORA_NUM_PHASES; ++i) ms[i] = 0.0;
+  if (launches)
+    for (int i = 0; i < LORA_NUM_PHASES; ++i) launches[i] = 0;
+  int rc = LORA_OK;
+  for (auto& r : recs) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) rc = fail(LORA_ERR_CUDA, "timing event: %s", cudaGetErrorString(e));
+    if (ms) ms[r.phase] += t;
+    if (launches) launches[r.phase] += 1;
+  }
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  for (auto& r : recs) {
+    g_timing.pool.push_back(r.a);
+    g_timing.pool.push_back(r.b);
+  }
+  return rc;
+}
+
+int lora_mlp_ctx_layout_get(const lora_mlp_dims* dims, lora_mlp_ctx_layout* out) {
+  TRY(check_dims(dims));
+  if (!out) return fail(LORA_ERR_INVALID_ARG, "out is NULL");
+  *out = ctx_layout(dims);
+  return LORA_OK;
+}
+
+int lora_mlp_workspace_bytes(const lora_mlp_dims* dims, size_t* bytes) {
+  TRY(check_dims(dims));
+  if (!bytes) return fail(LORA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = ws_layout(dims).total;
+  return LORA_OK;
+}
+
+int lora_rmsnorm_fwd(int64_t T, int32_t d, float eps, const void* X, const void* w, void* H, float* rstd,
+                     void* stream) {
+  if (T < 1 || d < 8 || d % 8 || d > 65536) return fail(LORA_ERR_INVALID_ARG, "bad T/d (%lld, %d)", (long long)T, d);
+  TRY(check_ptrs({X, w, H, rstd}));
+  return launch_rms_fwd(static_cast<cudaStream_t>(stream), X, w, H, rstd, T, d, eps);
+}
+
+int lora_rmsnorm_bwd(int64_t T, int32_t d, const float* dH, const void* X, const void* w, const float* rstd,
+                     void* dX, void* stream) {
+  if (T < 1 || d < 8 || d % 8 || d > 65536) return fail(LORA_ERR_INVALID_ARG, "bad T/d (%lld, %d)", (long long)T, d);
+  TRY(check_ptrs({dH, X, w, rstd, dX}));
+  return launch_rms_bwd(static_cast<cudaStream_t>(stream), dH, X, w, rstd, dX, T, d);
+}
+
+int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float* codebook16, uint8_t* codes,
+                       float* absmax, void* stream) {
+  if (block != 64) return fail(LORA_ERR_UNSUPPORTED, "block must be 64");
+  if (numel < 64 || numel % 64) return fail(LORA_ERR_INVALID_ARG, "numel must be a positive multiple of 64");
+  TRY(check_ptrs({W, codebook16, codes, absmax}));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long nb = numel / 64;
+  const int threads = 256;
+  const long long blocks = std::min<long long>((nb + 7) / 8, 148LL * 16);
+  PhaseScope ps(st, PH_OTHER);
+  quantize4_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(static_cast<const uint16_t*>(W), nb,
+                                                                       codebook16, codes, absmax);
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
+
+int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B, int32_t b_mn,
+                   float* C, void* stream) {
+  if (M < 1 || N < 1 || K < 1 || M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31))
+    return fail(LORA_ERR_INVALID_ARG, "bad M/N/K");
+  if (M % 8 || N % 8 || K % 8) return fail(LORA_ERR_ALIGNMENT, "M, N, K must be multiples of 8");
+  TRY(check_ptrs({A, B, C}));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GemmArgs a = new_args(nullptr);
+  const int bn = b_mn ? (N >= 256 ? 256 : round_up(static_cast<int>(N), 64))
+                      : (N >= 256 ? 256 : round_up(static_cast<int>(N), 16));
+  if (a_mn) TRY(map_mn(&a.maps[0], A, K, M, M)); else TRY(map_k(&a.maps[0], A, M, K, K, 128));
+  if (b_mn) TRY(map_mn(&a.maps[1], B, K, N, N)); else TRY(map_k(&a.maps[1], B, N, K, K, bn));
+  set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(K));
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.bn = bn;
+  a.tiles_m = static_cast<int>((M + BM - 1) / BM);
+  a.tiles_n = static_cast<int>((N + bn - 1) / bn);
+  a.out[0] = C;
+  a.ld_out = N;
+  if (!a_mn && !b_mn) return launch_gemm<0, 0, 1, EPI_F32>(a, st, PH_OTHER);
+  if (!a_mn && b_mn) return launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_OTHER);
+  if (a_mn && !b_mn) return launch_gemm<1, 0, 1, EPI_F32>(a, st, PH_OTHER);
+  return launch_gemm<1, 1, 1, EPI_F32>(a, st, PH_OTHER);
+}
+
+int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const lora_mlp_weights* W,
+                 const lora_mlp_adapters* A, void* Y, void* ctx, void* workspace, void* stream) {
+  TRY(check_dims(D));
+  if (!W || !A) return fail(LORA_ERR_INVALID_ARG, "weights/adapters is NULL");
+  if (D->wfmt != LORA_WFMT_BF16) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights are not built into this entry point yet");
+  TRY(check_ptrs({X, rms_w, Y, ctx, workspace, W->Wg, W->Wu, W->Wd, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd}));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long T = D->T;
+  const int d = D->d, f = D->f, r = D->r, rp = rp_of(D);
+  const float s = D->scale;
+  const lora_mlp_ctx_layout L = ctx_layout(D);
+  const WsLayout WL = ws_layout(D);
+  int* status = at<int>(workspace, WL.status);
+  void* H = at<char>(ctx, L.H);
+  float* rstd = at<float>(ctx, L.rstd);
+  void* G = at<char>(ctx, L.G);
+  void* U = at<char>(ctx, L.U);
+  void* Act = at<char>(ctx, L.Act);
+  void* P = at<char>(ctx, L.P);
+  void* Pd = at<char>(ctx, L.Pd);
+  TRY(begin_call(status, st));
+
+  // S1: RMSNorm (cached rstd)
+  TRY(launch_rms_fwd(st, X, rms_w, H, rstd, T, d, D->eps));
+
+  // S2: P = s * [H Ag^T | H Au^T]  (rank-r projections, padded to rp columns each)
+  {
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], H, T, d, d, 128));
+    TRY(map_k(&a.maps[1], A->Ag, r, d, d, rp));
+    TRY(map_k(&a.maps[2], A->Au, r, d, d, rp));
+    set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
+    a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
+    a.out[0] = P; a.ld_out = 2 * rp; a.out_acc_col = rp; a.alpha = s;
+    TRY((launch_gemm<0, 0, 2, EPI_BF16>(a, st, PH_P_GU)));
+  }
+  // S3: G = H Wg^T + P_g Bg^T, U = H Wu^T + P_u Bu^T, Act = silu(G) * U
+  {
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], H, T, d, d, 128));
+    TRY(map_k(&a.maps[1], W->Wg, f, d, d, 128));
+    TRY(map_k(&a.maps[2], W->Wu, f, d, d, 128));
+    TRY(map_k(&a.maps[3], P, T, 2 * rp, 2 * rp, 128));
+    TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128));
+    TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
+    set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
+    set_seg(a, 1, 3, 0, 4, 0, -1, 0, rp);
+    set_seg(a, 2, 3, rp, -1, 0, 5, 0, rp);
+    a.M = static_cast<int>(T); a.N = f; a.bn = 128;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (f + 127) / 128;
+    a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
+    TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD>(a, st, PH_GATEUP)));
+  }
+  // S4a: Pd = s * Act Ad^T
+  {
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], Act, T, f, f, 128));
+    TRY(map_k(&a.maps[1], A->Ad, r, f, f, rp));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
+    a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
+    a.out[0] = Pd; a.ld_out = rp; a.alpha = s;
+    TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_P_D)));
+  }
+  // S4b: Y = Act Wd^T + Pd Bd^T
+  {
+    GemmArgs a = new_args(status);
+    const int bn = d >= 256 ? 256 : round_up(d, 16);
+    TRY(map_k(&a.maps[0], Act, T, f, f, 128));
+    TRY(map_k(&a.maps[1], W->Wd, d, f, f, bn));
+    TRY(map_k(&a.maps[2], Pd, T, rp, rp, 128));
+    TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
+    set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    a.M = static_cast<int>(T); a.N = d; a.bn = bn;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
+    a.out[0] = Y; a.ld_out = d;
+    TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_DOWN)));
+  }
+  return end_call(status, st);
+}
+
+int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const void* rms_w, const lora_mlp_weights* W,
+                 const lora_mlp_adapters* A, const void* ctx, void* dX, const lora_mlp_grads* gr, void* workspace,
+                 void* stream) {
+  TRY(check_dims(D));
+  if (!W || !A || !gr) return fail(LORA_ERR_INVALID_ARG, "weights/adapters/grads is NULL");
+  if (D->wfmt != LORA_WFMT_BF16) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights are not built into this entry point yet");
+  TRY(check_ptrs({dY, X, rms_w, ctx, dX, workspace, W->Wg, W->Wu, W->Wd, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd,
+                  gr->dAg, gr->dBg, gr->dAu, gr->dBu, gr->dAd, gr->dBd}));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long T = D->T;
+  const int d = D->d, f = D->f, r = D->r, rp = rp_of(D);
+  const float s = D->scale;
+  const lora_mlp_ctx_layout L = ctx_layout(D);
+  const WsLayout WL = ws_layout(D);
+  int* status = at<int>(workspace, WL.status);
+  const void* H = at<char>(ctx, L.H);
+  const float* rstd = at<float>(ctx, L.rstd);
+  const void* G = at<char>(ctx, L.G);
+  const void* U = at<char>(ctx, L.U);
+  const void* Act = at<char>(ctx, L.Act);
+  const void* P = at<char>(ctx, L.P);
+  const void* Pd = at<char>(ctx, L.Pd);
+  void* Q = at<char>(workspace, WL.Q);
+  void* Qd = at<char>(workspace, WL.Qd);
+  void* dG = at<char>(workspace, WL.dG);
+  void* dU = at<char>(workspace, WL.dU);
+  float* dH = at<float>(workspace, WL.dH);
+  const int tm = static_cast<int>((T + BM - 1) / BM);
+  const int qbn = rp <= 64 ? 64 : 128;
+  TRY(begin_call(status, st));
+
+  // S5a: Qd = s * dY Bd
+  {
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], dY, T, d, d, 128));
+    TRY(map_mn(&a.maps[1], A->Bd, d, r, r));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
+    a.M = static_cast<int>(T); a.N = rp; a.bn = qbn; a.tiles_m = tm; a.tiles_n = 1;
+    a.out[0] = Qd; a.ld_out = rp; a.alpha = s;
+    TRY((launch_gemm<0, 1, 1, EPI_BF16>(a, st, PH_Q_D)));
+  }
+  // S5b + S6: dAct = dY Wd + Qd Ad  ->  dG = dAct U silu'(G), dU = dAct silu(G)
+  {
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], dY, T, d, d, 128));
+    TRY(map_mn(&a.maps[1], W->Wd, d, f, f));
+    TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
+    TRY(map_mn(&a.maps[3], A->Ad, r, f, f));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
+    set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    const int bn = f >= 256 ? 256 : round_up(f, 64);
+    a.M = static_cast<int>(T); a.N = f; a.bn = bn; a.tiles_m = tm; a.tiles_n = (f + bn - 1) / bn;
+    a.in[0] = G; a.in[1] = U; a.ld_in = f;
+    a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
+    TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
+  }
+  // S7a: Q = s * [dG Bg | dU Bu]
+  {
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], dG, T, f, f, 128));
+    TRY(map_k(&a.maps[1], dU, T, f, f, 128));
+    TRY(map_mn(&a.maps[2], A->Bg, f, r, r));
+    TRY(map_mn(&a.maps[3], A->Bu, f, r, r));
+    set_seg(a, 0, 0, 0, 2, 0, -1, 0, f);
+    set_seg(a, 1, 1, 0, -1, 0, 3, 0, f);
+    a.M = static_cast<int>(T); a.N = rp; a.bn = qbn; a.tiles_m = tm; a.tiles_n = 1;
+    a.out[0] = Q; a.ld_out = 2 * rp; a.out_acc_col = rp; a.alpha = s;
+    TRY((launch_gemm<0, 1, 2, EPI_BF16>(a, st, PH_Q_GU)));
+  }
+  // S8: dH = dG Wg + dU Wu + Q_g Ag + Q_u Au   (fp32)
+  {
+    GemmArgs a = new_args(status);
+    const int bn = d >= 256 ? 256 : round_up(d, 64);
+    TRY(map_k(&a.maps[0], dG, T, f, f, 128));
+    TRY(map_mn(&a.maps[1], W->Wg, f, d, d));
+    TRY(map_k(&a.maps[2], dU, T, f, f, 128));
+    TRY(map_mn(&a.maps[3], W->Wu, f, d, d));
+    TRY(map_k(&a.maps[4], Q, T, 2 * rp, 2 * rp, 128));
+    TRY(map_mn(&a.maps[5], A->Ag, r, d, d));
+    TRY(map_mn(&a.maps[6], A->Au, r, d, d));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
+    set_seg(a, 1, 2, 0, 3, 0, -1, 0, f);
+    set_seg(a, 2, 4, 0, 5, 0, -1, 0, rp);
+    set_seg(a, 3, 4, rp, 6, 0, -1, 0, rp);
+    a.M = static_cast<int>(T); a.N = d; a.bn = bn; a.tiles_m = tm; a.tiles_n = (d + bn - 1) / bn;
+    a.out[0] = dH; a.ld_out = d;
+    TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
+  }
+  // S10: dX = RMSNorm backward (cached rstd)
+  TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));
+
+  // adapter gradients: overwrite semantics -> zero, then split-T atomic reductions
+  {
+    ZeroList z;
+    z.p[0] = gr->dAg; z.n[0] = static_cast<long long>(r) * d;
+    z.p[1] = gr->dAu; z.n[1] = static_cast<long long>(r) * d;
+    z.p[2] = gr->dBg; z.n[2] = static_cast<long long>(f) * r;
+    z.p[3] = gr->dBu; z.n[3] = static_cast<long long>(f) * r;
+    z.p[4] = gr->dAd; z.n[4] = static_cast<long long>(r) * f;
+    z.p[5] = gr->dBd; z.n[5] = static_cast<long long>(d) * r;
+    PhaseScope ps(st, PH_ZERO);
+    zero6_kernel<<<296, 256, 0, st>>>(z);
+    CUDA_TRY(cudaGetLastError());
+  }
+  // S9: dAg = Q_g^T H, dAu = Q_u^T H  ([r x d]; rows of Q^T H)
+  {
+    GemmArgs a = new_args(status);
+    const int bn = d >= 256 ? 256 : round_up(d, 64);
+    TRY(map_mn(&a.maps[0], Q, T, 2 * rp, 2 * rp));
+    TRY(map_mn(&a.maps[1], H, T, d, d));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
+    a.M = 2 * rp; a.N = d; a.bn = bn; a.tiles_m = (2 * rp + BM - 1) / BM; a.tiles_n = (d + bn - 1) / bn;
+    a.rng[0] = OutRange{gr->dAg, 0, 0, r, 0, d};
+    a.rng[1] = OutRange{gr->dAu, 0, rp, rp + r, 0, d};
+    a.nrng = 2;
+    choose_splits(a, T);
+    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DA_GU)));
+  }
+  // S7b: dBg = dG^T P_g, dBu = dU^T P_u  ([f x r]; transposed rows of P^T dG)
+  {
+    GemmArgs a = new_args(status);
+    const int bn = f >= 128 ? 128 : round_up(f, 64);
+    TRY(map_mn(&a.maps[0], P, T, 2 * rp, 2 * rp));
+    TRY(map_mn(&a.maps[1], dG, T, f, f));
+    TRY(map_mn(&a.maps[2], dU, T, f, f));
+    set_seg(a, 0, 0, 0, 1, 0, 2, 0, static_cast<int>(T));
+    a.M = 2 * rp; a.N = f; a.bn = bn; a.tiles_m = (2 * rp + BM - 1) / BM; a.tiles_n = (f + bn - 1) / bn;
+    a.rng[0] = OutRange{gr->dBg, 0, 0, r, 1, r};
+    a.rng[1] = OutRange{gr->dBu, 1, rp, rp + r, 1, r};
+    a.nrng = 2;
+    choose_splits(a, T);
+    TRY((launch_gemm<1, 1, 2, EPI_ATOMIC>(a, st, PH_RED_DB_GU)));
+  }
+  // S5c: dBd = dY^T Pd  ([d x r])
+  {
+    GemmArgs a = new_args(status);
+    const int bn = d >= 256 ? 256 : round_up(d, 64);
+    TRY(map_mn(&a.maps[0], Pd, T, rp, rp));
+    TRY(map_mn(&a.maps[1], dY, T, d, d));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
+    a.M = rp; a.N = d; a.bn = bn; a.tiles_m = 1; a.tiles_n = (d + bn - 1) / bn;
+    a.rng[0] = OutRange{gr->dBd, 0, 0, r, 1, r};
+    a.nrng = 1;
+    choose_splits(a, T);
+    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DB_D)));
+  }
+  // S6b: dAd = Qd^T Act  ([r x f])
+  {
+    GemmArgs a = new_args(status);
+    const int bn = f >= 256 ? 256 : round_up(f, 64);
+    TRY(map_mn(&a.maps[0], Qd, T, rp, rp));
+    TRY(map_mn(&a.maps[1], Act, T, f, f));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
+    a.M = rp; a.N = f; a.bn = bn; a.tiles_m = 1; a.tiles_n = (f + bn - 1) / bn;
+    a.rng[0] = OutRange{gr->dAd, 0, 0, r, 0, f};
+    a.nrng = 1;
+    choose_splits(a, T);
+    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DA_D)));
+  }
+  return end_call(status, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,170 @@
+// Row kernels bounded by HBM bandwidth: RMSNorm forward/backward, the 4-bit
+// blockwise quantiser, and zero-fill of the fp32 gradient outputs.
+//
+// RMSNorm ("Unsloth提速秘诀：Triton内核如何加速反向传播", §3.2): one CTA per row,
+// 16-byte vector loads held in registers (the row is read once), fp32 sums,
+// rstd cached for the backward, the normalised row rounded once to bf16.
+#pragma once
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace lm {
+
+constexpr int kRowThreads = 128;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
+  __syncthreads();  // protect `red` from a previous use
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < nw; ++i) s += red[i];
+  return s;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+  f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+// VPT = 16-byte vectors (8 bf16) per thread; blockDim.x * VPT * 8 >= d.
+template <int VPT>
+__global__ void __launch_bounds__(1024) rmsnorm_fwd_kernel(const uint16_t* __restrict__ X,
+                                                           const uint16_t* __restrict__ w,
+                                                           uint16_t* __restrict__ H,
+                                                           float* __restrict__ rstd, int d,
+                                                           float eps) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const int nvec = d / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(X + row * d);
+  uint4 xv[VPT];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int v = threadIdx.x + i * blockDim.x;
+    xv[i] = v < nvec ? __ldcs(xr + v) : make_uint4(0, 0, 0, 0);
+    float f[8];
+    unpack8(xv[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+  }
+  ss = block_sum(ss, red);
+  const float rs = rsqrtf(ss / static_cast<float>(d) + eps);
+  if (threadIdx.x == 0) rstd[row] = rs;
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  uint4* hr = reinterpret_cast<uint4*>(H + row * d);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int v = threadIdx.x + i * blockDim.x;
+    if (v >= nvec) continue;
+    float f[8], g[8];
+    unpack8(xv[i], f);
+    unpack8(__ldg(wr + v), g);
+    uint4 o;
+    o.x = pack_bf16x2(f[0] * rs * g[0], f[1] * rs * g[1]);
+    o.y = pack_bf16x2(f[2] * rs * g[2], f[3] * rs * g[3]);
+    o.z = pack_bf16x2(f[4] * rs * g[4], f[5] * rs * g[5]);
+    o.w = pack_bf16x2(f[6] * rs * g[6], f[7] * rs * g[7]);
+    hr[v] = o;
+  }
+}
+
+// dX = rstd * (g - xhat * mean(g * xhat)), g = dH * w, xhat = x * rstd.
+template <int VPT>
+__global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restrict__ dH,
+                                                           const uint16_t* __restrict__ X,
+                                                           const uint16_t* __restrict__ w,
+                                                           const float* __restrict__ rstd,
+                                                           uint16_t* __restrict__ dX, int d) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const int nvec = d / 8;
+  const float rs = rstd[row];
+  const float4* hr = reinterpret_cast<const float4*>(dH + row * d);
+  const uint4* xr = reinterpret_cast<const uint4*>(X + row * d);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  float g[VPT][8], xh[VPT][8];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int v = threadIdx.x + i * blockDim.x;
+    if (v < nvec) {
+      const float4 h0 = __ldcs(hr + 2 * v), h1 = __ldcs(hr + 2 * v + 1);
+      float xf[8], wf[8];
+      unpack8(__ldcs(xr + v), xf);
+      unpack8(__ldg(wr + v), wf);
+      const float hh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        g[i][j] = hh[j] * wf[j];
+        xh[i][j] = xf[j] * rs;
+        dot = fmaf(g[i][j], xh[i][j], dot);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) g[i][j] = xh[i][j] = 0.f;
+    }
+  }
+  dot = block_sum(dot, red);
+  const float c = dot / static_cast<float>(d);
+  uint4* dr = reinterpret_cast<uint4*>(dX + row * d);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int v = threadIdx.x + i * blockDim.x;
+    if (v >= nvec) continue;
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = rs * (g[i][j] - xh[i][j] * c);
+    uint4 ov;
+    ov.x = pack_bf16x2(o[0], o[1]);
+    ov.y = pack_bf16x2(o[2], o[3]);
+    ov.z = pack_bf16x2(o[4], o[5]);
+    ov.w = pack_bf16x2(o[6], o[7]);
+    dr[v] = ov;
+  }
+}
+
+// One warp per 64-element block: two elements per lane, absmax by warp max,
+// code index = number of midpoints the value exceeds (decided exactly: the sign of
+// a fused multiply-add w - absmax * m_i is the sign of the exact difference).
+__global__ void quantize4_kernel(const uint16_t* __restrict__ W, long long nblocks,
+                                 const float* __restrict__ code, uint8_t* __restrict__ codes,
+                                 float* __restrict__ absmax) {
+  __shared__ float mid[15];
+  if (threadIdx.x < 15) mid[threadIdx.x] = (code[threadIdx.x] + code[threadIdx.x + 1]) * 0.5f;
+  __syncthreads();
+  const int lane = threadIdx.x % 32;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+       b < nblocks; b += warps) {
+    const uint32_t pair = reinterpret_cast<const uint32_t*>(W + b * 64)[lane];
+    const float w0 = bf16lo(pair), w1 = bf16hi(pair);
+    float am = fmaxf(fabsf(w0), fabsf(w1));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    int i0 = 0, i1 = 0;
+#pragma unroll
+    for (int i = 0; i < 15; ++i) {
+      i0 += fmaf(-am, mid[i], w0) > 0.f;
+      i1 += fmaf(-am, mid[i], w1) > 0.f;
+    }
+    codes[b * 32 + lane] = static_cast<uint8_t>(i0 | (i1 << 4));
+    if (lane == 0) absmax[b] = am;
+  }
+}
+
+struct ZeroList {
+  float* p[6];
+  long long n[6];
+};
+__global__ void zero6_kernel(ZeroList z) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (int k = 0; k < 6; ++k)
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < z.n[k]; i += stride)
+      z.p[k][i] = 0.f;
+}
+
+}  // namespace lm

@@ -1,0 +1,214 @@
+"""ctypes binding of liblora_mlp.so (include/lora_mlp.h): argument marshalling only.
+
+Every step of the LoRA-MLP path runs in the library's CUDA kernels; torch is used
+here only to allocate device memory and to name the current stream.  If the
+library is missing the import fails loudly: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblora_mlp.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "lora_mlp.h")
+
+LORA_OK = 0
+ERRORS = {-1: "INVALID_ARG", -2: "ALIGNMENT", -3: "UNSUPPORTED", -4: "CUDA", -5: "TIMEOUT"}
+WFMT_BF16, WFMT_4BIT = 0, 1
+NUM_PHASES = 16
+
+
+class LoraError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("f", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("eps", ctypes.c_float), ("scale", ctypes.c_float), ("wfmt", ctypes.c_int32),
+                ("qblock", ctypes.c_int32)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("Wg", "Wu", "Wd", "Qg", "Qu", "Qd", "absmax_g", "absmax_u", "absmax_d", "codebook")]
+
+
+class Adapters(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")]
+
+
+class CtxLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("rstd", "H", "G", "U", "Act", "P", "Pd", "total")] + \
+               [("rp", ctypes.c_int32)]
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/lora_mlp.h declares."""
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(lora_\w+)\s*\(", txt, flags=re.M)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m lora_fine_tuning_rmsnorm_b200.build` "
+                          "(the LoRA-MLP path has no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    sig = {
+        "lora_mlp_ctx_layout_get": [ctypes.POINTER(Dims), ctypes.POINTER(CtxLayout)],
+        "lora_mlp_workspace_bytes": [ctypes.POINTER(Dims), ctypes.POINTER(ctypes.c_size_t)],
+        "lora_mlp_fwd": [ctypes.POINTER(Dims), vp, vp, ctypes.POINTER(Weights), ctypes.POINTER(Adapters), vp, vp,
+                         vp, vp],
+        "lora_mlp_bwd": [ctypes.POINTER(Dims), vp, vp, vp, ctypes.POINTER(Weights), ctypes.POINTER(Adapters), vp,
+                         vp, ctypes.POINTER(Grads), vp, vp],
+        "lora_rmsnorm_fwd": [i64, i32, f32, vp, vp, vp, vp, vp],
+        "lora_rmsnorm_bwd": [i64, i32, vp, vp, vp, vp, vp, vp],
+        "lora_quantize_4bit": [vp, i64, i32, vp, vp, vp, vp],
+        "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, vp],
+        "lora_mlp_timing_enable": [i32],
+        "lora_mlp_timing_collect": [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.lora_mlp_last_error.restype = ctypes.c_char_p
+    L.lora_mlp_last_error.argtypes = []
+    L.lora_mlp_phase_name.restype = ctypes.c_char_p
+    L.lora_mlp_phase_name.argtypes = [i32]
+    _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != LORA_OK:
+        raise LoraError(rc, lib().lora_mlp_last_error().decode())
+
+
+def _p(t):
+    """Device (or host) address of a tensor, or None."""
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_dims(T, d, f, r, eps=1e-6, scale=1.0, wfmt=WFMT_BF16, qblock=64) -> Dims:
+    return Dims(T, d, f, r, eps, scale, wfmt, qblock)
+
+
+def ctx_layout(dims: Dims) -> CtxLayout:
+    out = CtxLayout()
+    _check(lib().lora_mlp_ctx_layout_get(ctypes.byref(dims), ctypes.byref(out)))
+    return out
+
+
+def workspace_bytes(dims: Dims) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)))
+    return out.value
+
+
+def alloc_ctx(dims: Dims, device="cuda"):
+    import torch
+    return torch.empty(ctx_layout(dims).total, dtype=torch.uint8, device=device)
+
+
+def alloc_workspace(dims: Dims, device="cuda"):
+    import torch
+    return torch.empty(workspace_bytes(dims), dtype=torch.uint8, device=device)
+
+
+def ctx_views(dims: Dims, ctx):
+    """Typed views of the saved context (rstd, H, G, U, Act, P, Pd) for inspection."""
+    import torch
+    L = ctx_layout(dims)
+    T, d, f, rp = dims.T, dims.d, dims.f, L.rp
+
+    def v(off, n, dt, shape):
+        nbytes = n * (4 if dt == torch.float32 else 2)
+        return ctx[off:off + nbytes].view(dt).view(*shape)
+    return dict(rstd=v(L.rstd, T, torch.float32, (T,)), H=v(L.H, T * d, torch.bfloat16, (T, d)),
+                G=v(L.G, T * f, torch.bfloat16, (T, f)), U=v(L.U, T * f, torch.bfloat16, (T, f)),
+                Act=v(L.Act, T * f, torch.bfloat16, (T, f)), P=v(L.P, T * 2 * rp, torch.bfloat16, (T, 2 * rp)),
+                Pd=v(L.Pd, T * rp, torch.bfloat16, (T, rp)))
+
+
+def make_weights(Wg=None, Wu=None, Wd=None, Qg=None, Qu=None, Qd=None, absmax_g=None, absmax_u=None,
+                 absmax_d=None, codebook=None) -> Weights:
+    return Weights(*[_p(t) for t in (Wg, Wu, Wd, Qg, Qu, Qd, absmax_g, absmax_u, absmax_d, codebook)])
+
+
+def make_adapters(Ag, Bg, Au, Bu, Ad, Bd) -> Adapters:
+    return Adapters(*[_p(t) for t in (Ag, Bg, Au, Bu, Ad, Bd)])
+
+
+def make_grads(dAg, dBg, dAu, dBu, dAd, dBd) -> Grads:
+    return Grads(*[_p(t) for t in (dAg, dBg, dAu, dBu, dAd, dBd)])
+
+
+def lora_mlp_fwd(dims: Dims, X, rms_w, weights: Weights, adapters: Adapters, Y, ctx, workspace, stream=None):
+    _check(lib().lora_mlp_fwd(ctypes.byref(dims), _p(X), _p(rms_w), ctypes.byref(weights),
+                              ctypes.byref(adapters), _p(Y), _p(ctx), _p(workspace), _stream(stream)))
+
+
+def lora_mlp_bwd(dims: Dims, dY, X, rms_w, weights: Weights, adapters: Adapters, ctx, dX, grads: Grads,
+                 workspace, stream=None):
+    _check(lib().lora_mlp_bwd(ctypes.byref(dims), _p(dY), _p(X), _p(rms_w), ctypes.byref(weights),
+                              ctypes.byref(adapters), _p(ctx), _p(dX), ctypes.byref(grads), _p(workspace),
+                              _stream(stream)))
+
+
+def lora_rmsnorm_fwd(X, w, H, rstd, eps, stream=None):
+    T, d = X.shape
+    _check(lib().lora_rmsnorm_fwd(T, d, eps, _p(X), _p(w), _p(H), _p(rstd), _stream(stream)))
+
+
+def lora_rmsnorm_bwd(dH, X, w, rstd, dX, stream=None):
+    T, d = X.shape
+    _check(lib().lora_rmsnorm_bwd(T, d, _p(dH), _p(X), _p(w), _p(rstd), _p(dX), _stream(stream)))
+
+
+def lora_quantize_4bit(W, codebook, codes, absmax, block=64, stream=None):
+    _check(lib().lora_quantize_4bit(_p(W), W.numel(), block, _p(codebook), _p(codes), _p(absmax),
+                                    _stream(stream)))
+
+
+def lora_gemm_bf16(A, a_mn, B, b_mn, C, stream=None):
+    M, N = C.shape
+    K = A.shape[0] if a_mn else A.shape[1]
+    _check(lib().lora_gemm_bf16(M, N, K, _p(A), int(a_mn), _p(B), int(b_mn), _p(C), _stream(stream)))
+
+
+def timing_enable(on: bool = True):
+    _check(lib().lora_mlp_timing_enable(1 if on else 0))
+
+
+def timing_collect() -> dict:
+    ms = (ctypes.c_double * NUM_PHASES)()
+    n = (ctypes.c_int64 * NUM_PHASES)()
+    _check(lib().lora_mlp_timing_collect(ms, n))
+    out = {}
+    for i in range(NUM_PHASES):
+        if n[i]:
+            out[lib().lora_mlp_phase_name(i).decode()] = (ms[i], n[i])
+    return out

@@ -19,3 +19,9 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+# GPU tests run the library in debug mode: every call synchronises and reports
+# device-side bounded-wait failures as LORA_ERR_TIMEOUT instead of silent garbage.
+os.environ.setdefault("LORA_MLP_DEBUG", "1")
+os.environ.setdefault("LORA_MLP_WAIT_LIMIT_MS", "3000")

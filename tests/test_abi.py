@@ -1,0 +1,95 @@
+"""The C-ABI library: it loads, exports every function include/lora_mlp.h declares,
+and rejects bad arguments on the host with the documented codes (no GPU needed:
+validation happens before any CUDA call)."""
+import ctypes
+
+import pytest
+
+from lora_fine_tuning_rmsnorm_b200 import build, ops
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = ops.header_functions()
+    assert {"lora_mlp_fwd", "lora_mlp_bwd", "lora_rmsnorm_fwd", "lora_rmsnorm_bwd", "lora_quantize_4bit",
+            "lora_gemm_bf16", "lora_mlp_ctx_layout_get", "lora_mlp_workspace_bytes",
+            "lora_mlp_last_error"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_layout_and_workspace_sizes(L):
+    dims = ops.make_dims(8192, 4096, 14336, 16)
+    lay = ops.ctx_layout(dims)
+    assert lay.rp == 16
+    T, d, f = 8192, 4096, 14336
+    assert lay.H - lay.rstd >= T * 4 and lay.G - lay.H >= T * d * 2
+    assert lay.total >= T * 4 + T * d * 2 + 3 * T * f * 2 + 3 * T * 16 * 2
+    for off in (lay.rstd, lay.H, lay.G, lay.U, lay.Act, lay.P, lay.Pd):
+        assert off % 256 == 0
+    ws = ops.workspace_bytes(dims)
+    assert ws >= T * d * 4 + 2 * T * f * 2
+    assert ops.ctx_layout(ops.make_dims(64, 128, 344, 8)).rp == 16
+
+
+@pytest.mark.parametrize("T,d,f,r,code", [
+    (0, 128, 344, 8, ops.ERRORS and -1),
+    (64, 0, 344, 8, -1),
+    (64, 130, 344, 8, -2),
+    (64, 128, 340, 8, -2),
+    (64, 128, 344, 12, -2),
+    (64, 128, 344, 136, -3),
+    (64, 70000, 344, 8, -3),
+])
+def test_bad_dims_rejected(L, T, d, f, r, code):
+    dims = ops.make_dims(T, d, f, r)
+    out = ctypes.c_size_t()
+    rc = L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out))
+    assert rc == code
+    assert len(L.lora_mlp_last_error()) > 0
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    dims = ops.make_dims(64, 128, 344, 8)
+    w = ops.Weights()
+    a = ops.Adapters()
+    rc = L.lora_mlp_fwd(ctypes.byref(dims), None, None, ctypes.byref(w), ctypes.byref(a), None, None, None, None)
+    assert rc == -1
+    assert b"NULL" in L.lora_mlp_last_error()
+    bad = ctypes.c_void_p(0x1001)
+    good = ctypes.c_void_p(0x1000)
+    rc = L.lora_rmsnorm_fwd(64, 128, 1e-6, bad, good, good, good, None)
+    assert rc == -2
+    rc = L.lora_rmsnorm_fwd(64, 129, 1e-6, good, good, good, good, None)
+    assert rc == -1
+    rc = L.lora_quantize_4bit(good, 100, 64, good, good, good, None)
+    assert rc == -1
+    rc = L.lora_quantize_4bit(good, 128, 32, good, good, good, None)
+    assert rc == -3
+    rc = L.lora_gemm_bf16(64, 60, 64, good, 0, good, 0, good, None)
+    assert rc == -2
+    g = ops.Grads()
+    rc = L.lora_mlp_bwd(ctypes.byref(dims), good, good, good, ctypes.byref(w), ctypes.byref(a), good, good,
+                        ctypes.byref(g), good, None)
+    assert rc == -1
+
+
+def test_4bit_dims_rules(L):
+    dims = ops.make_dims(64, 128, 344, 8, wfmt=ops.WFMT_4BIT)
+    out = ctypes.c_size_t()
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3   # f % 64 != 0
+    dims = ops.make_dims(64, 128, 384, 8, wfmt=ops.WFMT_4BIT, qblock=32)
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3
+    dims = ops.make_dims(64, 128, 384, 8, wfmt=ops.WFMT_4BIT)
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == 0
+
+
+def test_phase_names(L):
+    names = [L.lora_mlp_phase_name(i).decode() for i in range(ops.NUM_PHASES)]
+    assert "gemm_gate_up_swiglu" in names and "rmsnorm_fwd" in names
+    assert L.lora_mlp_phase_name(99) == b"invalid"
