@@ -1,0 +1,345 @@
+"""LoRA-MLP fwd+bwd throughput on B200 (tokens/s at the Llama-3-8B MLP shape).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 8b|1b|tiny]
+
+One step = RMSNorm -> gate/up(+LoRA) -> SwiGLU -> down(+LoRA) forward and the
+hand-derived backward (dX and the six adapter gradients) over one batch of
+T = 8192 tokens (batch 4 x seq 2048), d = 4096, f = 14336, r = 16, alpha = 16,
+on seeded synthetic bf16 inputs.  With N > 1 (one process per GPU under torchrun)
+every rank runs its own batch (weak scaling) and the adapter gradients are summed
+across ranks with one NCCL all-reduce per step, as data-parallel LoRA training
+does.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on this host's cores instead (a bounded
+sample of rows per step), on the same metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LoRA-MLP fwd+bwd tokens/s at Llama-3-8B shape; % of bf16 tensor-core peak"
+UNIT = "tokens/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return j.get("hbm_gbs", 6650.0), j.get("bf16_tflops", 1590.0), j.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def shape_for(name, T=None):
+    import dataclasses
+    from lora_fine_tuning_rmsnorm_b200 import configs
+    s = {"8b": configs.LLAMA3_8B, "1b": configs.LLAMA32_1B, "tiny": configs.TINY}[name]
+    return dataclasses.replace(s, T=T) if T else s
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        return len(os.sched_getaffinity(0))
+
+
+class OracleTimer:
+    """Times the fp64 oracle (as it stands) fwd+bwd on a bounded sample of rows."""
+
+    def __init__(self, shape, bits=None, max_rows=2048):
+        from lora_fine_tuning_rmsnorm_b200 import synth
+        self.shape = shape
+        if bits is None:
+            bits = synth.make_inputs_bits(synth.Shape(T=min(shape.T, max_rows), d=shape.d, f=shape.f, r=shape.r,
+                                                      alpha=shape.alpha, eps=shape.eps))
+        self.inp = synth.bits_to_f64({k: (v[:max_rows] if k in ("X", "dY") else v) for k, v in bits.items()})
+        self.cores = _blas_threads()
+
+    def run(self, n):
+        from oracle import lora_mlp_ref as ref
+        sub = dict(self.inp)
+        sub["X"], sub["dY"] = self.inp["X"][:n], self.inp["dY"][:n]
+        t0 = time.perf_counter()
+        ref.fwd_bwd(sub, self.shape.scale, self.shape.eps, chunk=1024, keep=("Y", "dX"))
+        return time.perf_counter() - t0
+
+    def size_for(self, target_s):
+        n = 64
+        t = self.run(n)
+        n = int(n * target_s / max(t, 1e-3))
+        return max(16, min(n, len(self.inp["X"])))
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    shape = shape_for(args.config)
+    ot = OracleTimer(shape)
+    n = ot.size_for(max(1.0, 90.0 / (args.steps + args.warmup)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = ot.run(n)
+        if i >= args.warmup:
+            times.append(t)
+    t_med = statistics.median(times)
+    value = n / t_med
+    sample = f"{n} of {shape.T} rows per step (fp64 NumPy oracle fwd+bwd over all weights)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_med,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, bf16-rounded)",
+        "config": {"workload": f"LoRA-MLP {args.config} T={shape.T} d={shape.d} f={shape.f} r={shape.r}",
+                   "global_batch": shape.T, "seq_len": 2048, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": ot.cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for ln in open(self.path):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+def ours_arm(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from lora_fine_tuning_rmsnorm_b200 import configs, ops, synth
+    from lora_fine_tuning_rmsnorm_b200.runner import GRADS, Problem, bf16_tensor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    shape = shape_for(args.config, args.T)
+    bits = synth.make_inputs_bits(shape)
+    pb = Problem(shape, bits, device=dev)
+    # one flat fp32 buffer for the six adapter gradients -> one all-reduce per step
+    sizes = {"dAg": (shape.r, shape.d), "dBg": (shape.f, shape.r), "dAu": (shape.r, shape.d),
+             "dBu": (shape.f, shape.r), "dAd": (shape.r, shape.f), "dBd": (shape.d, shape.r)}
+    total = sum(a * b for a, b in sizes.values())
+    flat = torch.zeros(total, dtype=torch.float32, device=dev)
+    off = 0
+    for k in GRADS:
+        n = sizes[k][0] * sizes[k][1]
+        pb.g[k] = flat[off:off + n].view(*sizes[k])
+        off += n
+    pb.grads = ops.make_grads(*(pb.g[k] for k in GRADS))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pb.forward(stream=stream)
+        pb.backward(stream=stream)
+        if world > 1:
+            dist.all_reduce(flat)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    clk = ClockSampler(local_rank) if (rank == 0 and not args.no_clocks) else None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # ---- device-resident timed region
+    ops.timing_enable(True)
+    ops.timing_collect()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1)
+    phases = ops.timing_collect()
+    ops.timing_enable(False)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms = max_over_ranks(ms)
+    tokens = world * shape.T * args.steps
+    value = tokens / (ms / 1e3)
+
+    # ---- end-to-end through the C ABI with host buffers (pinned), copies inside the timed region
+    hX = bf16_tensor(bits["X"], "cpu", pin=True)
+    hdY = bf16_tensor(bits["dY"], "cpu", pin=True)
+    dX_in = torch.empty_like(pb.t["X"])
+    dY_in = torch.empty_like(pb.t["dY"])
+    hY = torch.empty(pb.Y.shape, dtype=torch.bfloat16, pin_memory=True)
+    hdX = torch.empty(pb.dX.shape, dtype=torch.bfloat16, pin_memory=True)
+    hflat = torch.empty(flat.shape, dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        dX_in.copy_(hX, non_blocking=True)
+        dY_in.copy_(hdY, non_blocking=True)
+        pb.forward(X=dX_in, stream=stream)
+        pb.backward(dY=dY_in, X=dX_in, stream=stream)
+        if world > 1:
+            dist.all_reduce(flat)
+        hY.copy_(pb.Y, non_blocking=True)
+        hdX.copy_(pb.dX, non_blocking=True)
+        hflat.copy_(flat, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1))
+    e2e_value = world * shape.T * args.steps / (ms_e2e / 1e3)
+    clocks = clk.stop() if clk else None
+    h2d = hX.numel() * 2 + hdY.numel() * 2
+    d2h = hY.numel() * 2 + hdX.numel() * 2 + hflat.numel() * 4
+
+    if rank != 0:
+        return
+    hbm, bf16_burst, bf16_sust, src = peaks()
+    T, d, f, r = shape.T, shape.d, shape.f, shape.r
+    # dominant kernel: the gate/up GEMM with the LoRA B-term and the SwiGLU epilogue
+    dom = "gemm_gate_up_swiglu"
+    dom_ms, dom_n = phases.get(dom, (0.0, 0))
+    dom_flops = 4.0 * T * d * f + 4.0 * T * r * f
+    dom_tflops = dom_flops / (dom_ms / dom_n / 1e3) / 1e12 if dom_n else None
+    flops = configs.algorithmic_flops(shape)
+    step_ms = ms / args.steps
+    gemm_names = ("gemm_gate_up_swiglu", "gemm_down", "gemm_dact_swiglu_bwd", "gemm_dH")
+    gemm_ms = sum(phases.get(k, (0.0, 0))[0] for k in gemm_names) / args.steps
+    gemm_flops = 12.0 * T * d * f + 4.0 * T * r * f + 2.0 * T * r * d + 2.0 * T * r * f + 4.0 * T * r * d
+    rms_fwd_ms = phases.get("rmsnorm_fwd", (0.0, 1))[0] / args.steps
+    rms_bwd_ms = phases.get("rmsnorm_bwd", (0.0, 1))[0] / args.steps
+    rms_fwd_bytes = T * (4 * d + 4)
+    rms_bwd_bytes = T * (8 * d + 4)
+    launches = sum(n for _, n in phases.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; bf16 weights/activations, fp32 accumulate)",
+        "config": {"workload": f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape: T={T} (batch 4 x seq 2048) d={d} f={f} "
+                               f"r={r} alpha={shape.alpha:g}" if args.config == "8b" else
+                               f"LoRA-MLP fwd+bwd {args.config}: T={T} d={d} f={f} r={r}",
+                   "global_batch": T * world, "seq_len": 2048, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (weights 336 MB + activations), no flush"},
+        "tflops": flops / (step_ms / 1e3) / 1e12,
+        "pct_bf16_peak": flops / (step_ms / 1e3) / 1e12 / bf16_sust,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tflops, "peak": bf16_sust,
+                     "unit": "TFLOP/s", "frac": (dom_tflops / bf16_sust) if dom_tflops else None,
+                     "traffic": None, "peak_source": f"bf16_tflops_sustained ({src})",
+                     "flops_per_launch": dom_flops},
+        "phase_rooflines": {
+            "gemm_phases_frac_of_bf16_sustained": gemm_flops / (gemm_ms / 1e3) / 1e12 / bf16_sust if gemm_ms else None,
+            "rmsnorm_fwd_frac_of_hbm": rms_fwd_bytes / (rms_fwd_ms / 1e3) / 1e9 / hbm if rms_fwd_ms else None,
+            "rmsnorm_bwd_frac_of_hbm": rms_bwd_bytes / (rms_bwd_ms / 1e3) / 1e9 / hbm if rms_bwd_ms else None,
+        },
+        "phases_ms_per_step": {k: v[0] / args.steps for k, v in sorted(phases.items())},
+        "gpu_launches": launches,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        ot = OracleTimer(shape, bits, max_rows=shape.T)
+        n = ot.size_for(12.0)
+        t = ot.run(n)
+        line["cpu_baseline"] = {"value": n / t, "unit": UNIT, "cores": ot.cores, "kind": "oracle",
+                                "sample": f"{n} of {T} rows, fp64 NumPy oracle fwd+bwd over all weights ({t:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="8b", choices=["8b", "1b", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
+    ap.add_argument("--T", type=int, default=None, help="override the token count (profiling on small cases)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        ours_arm(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
