@@ -61,7 +61,7 @@ enum lora_wfmt {
 
 /* Problem sizes.  T tokens, hidden d, intermediate f, LoRA rank r.
  * Limits: 1 <= T < 2^31; d, f multiples of 8 with 8 <= d <= 65536, 8 <= f;
- * r a multiple of 8 with 8 <= r <= 256.  scale = alpha / r (any finite value).
+ * r a multiple of 8 with 8 <= r <= 128.  scale = alpha / r (any finite value).
  * wfmt = LORA_WFMT_BF16 or LORA_WFMT_4BIT (then qblock must be 64 and d, f
  * multiples of 64). */
 typedef struct lora_mlp_dims {
@@ -175,9 +175,12 @@ int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float*
 /* Plain tensor-core GEMM (the core the fused path is built on), fp32 out:
  *   C[M x N] = A' B'^T,  A' [M x K] = A (a_mn = 0, A row-major [M x K]) or A^T
  *   (a_mn = 1, A row-major [K x M]);  B' [N x K] = B (b_mn = 0, B [N x K]) or B^T
- *   (b_mn = 1, B [K x N]).  The contiguous dimension must be a multiple of 8. */
+ *   (b_mn = 1, B [K x N]).  M, N, K must be multiples of 8.
+ * flags: LORA_GEMM_CTA_PAIR runs 256-row tiles on pairs of SMs (tcgen05
+ * cta_group::2; needs a_mn = 0), otherwise one 128-row tile per SM. */
+#define LORA_GEMM_CTA_PAIR 1
 int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B,
-                   int32_t b_mn, float* C, void* stream);
+                   int32_t b_mn, float* C, int32_t flags, void* stream);
 
 /* Per-phase timing.  With timing enabled, every kernel launch of the calls above
  * is bracketed by CUDA events on the caller's stream.  lora_mlp_timing_collect()

@@ -12,10 +12,17 @@
 // K-major (x = K innermost) or MN-major (x = M/N innermost); out-of-range boxes
 // are zero-filled by TMA, which also pads ragged K tails and rank r to 16.
 //
-// CTA = 6 warps: warp 0 issues TMA loads into a `stages`-deep ring, warp 1 owns
-// TMEM and issues tcgen05.mma from one thread, warps 2..5 drain the double-
+// PAIR = 2 runs the same roles on a cluster of two CTAs that share one 256-row
+// tile through tcgen05 cta_group::2: each CTA loads its own 128 rows of A and its
+// half of the N columns of B (TMA completions counted on the even CTA's barrier,
+// no multicast loads), the even CTA issues the pair MMA, and commits arrive on both
+// CTAs' barriers.  This halves the B bytes each SM pulls from L2 per MMA.
+//
+// CTA = 10 warps: warp 0 issues TMA loads into a `stages`-deep ring, warp 1 owns
+// TMEM and issues tcgen05.mma from one thread, warps 2..9 drain the double-
 // buffered TMEM accumulators (tcgen05.ld) through the epilogue while the next
-// tile's main loop runs.  Tile order is M-fastest over a persistent grid.
+// tile's main loop runs (two warps per TMEM lane quarter, alternating 16-column
+// chunks).  Tile order is M-fastest over a persistent grid.
 #pragma once
 #include "ptx.cuh"
 
@@ -26,14 +33,15 @@ constexpr int BK = 64;
 constexpr int kMaxStages = 8;
 constexpr int kMaxSegs = 4;
 constexpr int kMaxMaps = 8;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16-column chunks
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 enum Epi : int {
-  EPI_F32 = 0,         // out[0] fp32 = acc * alpha
+  EPI_F32 = 0,         // out[0] fp32 = acc_a * alpha at column a * out_acc_col (+ split * split_stride)
   EPI_BF16 = 1,        // out[0] bf16 = acc_a * alpha, accumulator a at column a * out_acc_col
   EPI_SWIGLU_FWD = 2,  // acc0 = G, acc1 = U -> out[0] G, out[1] U, out[2] silu(G) * U (bf16)
   EPI_SWIGLU_BWD = 3,  // acc0 = dAct; in[0] G, in[1] U -> out[0] dG, out[1] dU (bf16)
-  EPI_ATOMIC = 4       // rows [lo, hi) of an accumulator atomically added into fp32 outputs
+  EPI_ATOMIC = 4       // accumulator a atomically added into fp32 output rng[a] (split-K reductions)
 };
 
 struct Seg {
@@ -45,10 +53,9 @@ struct Seg {
 };
 
 struct OutRange {
-  float* out;
+  float* out;     // destination of accumulator `acc` (rows m < M, columns n < N)
   int acc;
-  int lo, hi;     // accumulator rows (global M index) routed to `out`
-  int trans;      // 0: out[(m - lo) * ld + n]; 1: out[n * ld + (m - lo)]
+  int trans;      // 0: out[m * ld + n]; 1: out[n * ld + m]
   long long ld;
 };
 
@@ -65,6 +72,7 @@ struct GemmArgs {
   uint32_t tmem_cols;
   void* out[3];
   long long ld_out;
+  long long split_stride;  // EPI_F32: element offset between the partial sums of K splits
   int out_acc_col;
   float alpha;
   const void* in[2];
@@ -75,6 +83,7 @@ struct GemmArgs {
   unsigned long long limit_ns;
 };
 
+// Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
 __device__ __forceinline__ void decode_tile(const GemmArgs& p, int t, int& mt, int& nt, int& ks) {
   mt = t % p.tiles_m;
   t /= p.tiles_m;
@@ -105,20 +114,22 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const Wai
   }
 }
 
-template <int A_MN, int B_MN, int NACC>
+template <int A_MN, int B_MN, int NACC, int PAIR>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
-                                              uint32_t empty0, const WaitCtl& wc) {
+                                              uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
+  const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
+  const int bnl = p.bn / PAIR;  // B rows (N) held by this CTA
   int stage = 0;
   uint32_t phase = 0;
   uint32_t issued_mask = 0, issued_par = 0;
   const uint32_t a_bytes = BM * BK * 2;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
+  const uint32_t b_bytes = static_cast<uint32_t>(bnl) * BK * 2;
   bool ok = true;
-  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+  for (int t = unit0; t < total && ok; t += nunits) {
     int mt, nt, ks;
     decode_tile(p, t, mt, nt, ks);
-    const int m0 = mt * BM, n0 = nt * p.bn;
+    const int mbase = mt * BM * PAIR, n0 = nt * p.bn;
     for (int s = 0; s < p.nseg && ok; ++s) {
       const Seg& sg = p.seg[s];
       int kb0, kb1;
@@ -129,27 +140,46 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           ok = false;
           break;
         }
-        // Boxes that would lie entirely outside the matrix are skipped: the rows /
-        // columns they would feed are never stored by the epilogue.
-        const int nA = A_MN ? ((m0 + 64 < p.M) ? 2 : 1) : 1;
-        int nBc = B_MN ? 0 : 1;
-        if (B_MN) {
-          for (int c = 0; c < p.bn / 64; ++c)
-            if (n0 + 64 * c < p.N) ++nBc;
-        }
-        uint32_t bytes = static_cast<uint32_t>(nA) * (A_MN ? 8192u : a_bytes);
+        // Bytes landing for CTA rank rr.  Boxes that would lie entirely outside the
+        // matrix are skipped: the rows / columns they feed are never stored.
+        auto bytes_of = [&](uint32_t rr) -> uint32_t {
+          const int m0r = mbase + static_cast<int>(rr) * BM;
+          uint32_t by = 0;
+          if (A_MN) by += (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
+          else by += (m0r < p.M ? a_bytes : 0u);
+          const int nb0 = n0 + static_cast<int>(rr) * bnl;
+          uint32_t bb = 0;
+          if (B_MN) {
+            for (int c = 0; c < bnl / 64; ++c)
+              if (nb0 + 64 * c < p.N) bb += 8192u;
+          } else {
+            bb = nb0 < p.N ? b_bytes : 0u;
+          }
 #pragma unroll
-        for (int a = 0; a < NACC; ++a)
-          if (sg.b_map[a] >= 0) bytes += B_MN ? static_cast<uint32_t>(nBc) * 8192u : b_bytes;
-        mbar_expect_tx(full, bytes);
+          for (int a = 0; a < NACC; ++a)
+            if (sg.b_map[a] >= 0) by += bb;
+          return by;
+        };
+        if (PAIR == 1) {
+          mbar_expect_tx(full, bytes_of(0));
+        } else if (rank == 0) {
+          mbar_expect_tx(full, bytes_of(0) + bytes_of(1));
+        }
+        const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);
+        const int m0 = mbase + static_cast<int>(rank) * BM;
+        const int nb0 = n0 + static_cast<int>(rank) * bnl;
         const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
         const int k = kb * BK;
         const CUtensorMap* am = &p.maps[sg.a_map];
+        auto load = [&](uint32_t dst, const CUtensorMap* m, int x, int y) {
+          if (PAIR == 1) tma_load_2d(dst, m, bar, x, y);
+          else tma_load_2d_pair(dst, m, bar, x, y);
+        };
         if (A_MN) {
-          tma_load_2d(sA, am, full, m0, sg.a_k0 + k);
-          if (nA == 2) tma_load_2d(sA + 8192, am, full, m0 + 64, sg.a_k0 + k);
-        } else {
-          tma_load_2d(sA, am, full, sg.a_k0 + k, m0);
+          if (m0 < p.M) load(sA, am, m0, sg.a_k0 + k);
+          if (m0 + 64 < p.M) load(sA + 8192, am, m0 + 64, sg.a_k0 + k);
+        } else if (m0 < p.M) {
+          load(sA, am, sg.a_k0 + k, m0);
         }
 #pragma unroll
         for (int a = 0; a < NACC; ++a) {
@@ -157,10 +187,10 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           const uint32_t sB = sA + a_bytes + a * b_bytes;
           const CUtensorMap* bm = &p.maps[sg.b_map[a]];
           if (B_MN) {
-            for (int c = 0; c < nBc; ++c)
-              tma_load_2d(sB + c * 8192, bm, full, n0 + 64 * c, sg.b_k0[a] + k);
-          } else {
-            tma_load_2d(sB, bm, full, sg.b_k0[a] + k, n0);
+            for (int c = 0; c < bnl / 64; ++c)
+              if (nb0 + 64 * c < p.N) load(sB + c * 8192, bm, nb0 + 64 * c, sg.b_k0[a] + k);
+          } else if (nb0 < p.N) {
+            load(sB, bm, sg.b_k0[a] + k, nb0);
           }
         }
         issued_mask |= 1u << stage;
@@ -172,27 +202,29 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
       }
     }
   }
-  if (!ok) {
-    // Aborting: make sure no TMA write into shared memory is still in flight.
+  if (!ok && rank == 0) {
+    // Aborting: make sure no TMA write into shared memory is still in flight (the
+    // even CTA's full barriers also count the odd CTA's bytes).
     for (int s = 0; s < p.stages; ++s)
       if (issued_mask & (1u << s)) drain_wait(full0 + 8 * s, (issued_par >> s) & 1, wc);
   }
 }
 
-template <int A_MN, int B_MN, int NACC>
+template <int A_MN, int B_MN, int NACC, int PAIR>
 __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                          uint32_t empty0, uint32_t tfull0, uint32_t tempty0,
                                          uint32_t drain_bar, uint32_t tmem_base,
                                          const WaitCtl& wc) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
-  const uint32_t idesc = idesc_bf16(BM, p.bn, A_MN, B_MN);
+  const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
+  const uint32_t idesc = idesc_bf16(BM * PAIR, p.bn, A_MN, B_MN);
   const uint32_t a_bytes = BM * BK * 2;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.bn / PAIR) * BK * 2;
   int stage = 0;
   uint32_t phase = 0;
   uint32_t it = 0;
   bool ok = true, issued_any = false;
-  for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+  for (int t = unit0; t < total && ok; t += nunits, ++it) {
     int mt, nt, ks;
     decode_tile(p, t, mt, nt, ks);
     const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
@@ -225,37 +257,53 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
                                      : sdesc_sw128(sA + j * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(sB + j * 2048, 8192, 1024)
                                      : sdesc_sw128(sB + j * 32, 16, 1024);
-            mma_bf16(d, ad, bd, idesc, (started >> a) & 1);
+            if (PAIR == 1) mma_bf16(d, ad, bd, idesc, (started >> a) & 1);
+            else mma_bf16_pair(d, ad, bd, idesc, (started >> a) & 1);
             started |= 1u << a;
             issued_any = true;
           }
         }
-        mma_commit(empty0 + 8 * stage);  // frees the smem stage once these MMAs finish
+        // frees the smem stage (in both CTAs of a pair) once these MMAs finish
+        if (PAIR == 1) mma_commit(empty0 + 8 * stage);
+        else mma_commit_pair(empty0 + 8 * stage, 0x3);
         if (++stage == p.stages) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
-    if (ok) mma_commit(tfull0 + 8 * buf);  // accumulator ready for the epilogue
+    if (ok) {  // accumulator ready for the epilogue(s)
+      if (PAIR == 1) mma_commit(tfull0 + 8 * buf);
+      else mma_commit_pair(tfull0 + 8 * buf, 0x3);
+    }
   }
   if (!ok && issued_any) {
     // Aborting: wait for the MMAs already issued before TMEM is released.
-    mma_commit(drain_bar);
+    if (PAIR == 1) mma_commit(drain_bar);
+    else mma_commit_pair(drain_bar, 0x1);
     drain_wait(drain_bar, 0, wc);
   }
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+// sigmoid(g) = 1 / (1 + e^-g); for g << 0 the reciprocal of +inf is 0.
+__device__ __forceinline__ float sigmoid_f(float g) { return rcp_approx(1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
-template <int NACC, int EPI>
+template <int NACC, int EPI, int PAIR>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0, uint32_t tempty0,
-                                              uint32_t tmem_base, const WaitCtl& wc) {
+                                              uint32_t tmem_base, const WaitCtl& wc, uint32_t rank) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int q = warp & 3;  // TMEM lane quarter this warp may access
+  const int q = warp & 3;             // TMEM lane quarter this warp may access
+  const int c0 = ((warp - 2) >> 2) * 16;  // first 16-column chunk of this warp; stride 32
   const int total = p.tiles_m * p.tiles_n * p.splits;
+  const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   uint32_t it = 0;
-  for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+  for (int t = unit0; t < total; t += nunits, ++it) {
     int mt, nt, ks;
     decode_tile(p, t, mt, nt, ks);
     const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
@@ -264,7 +312,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) break;
     tc_fence_after();
-    const int m0 = mt * BM, n0 = nt * p.bn;
+    const int m0 = mt * BM * PAIR + static_cast<int>(rank) * BM, n0 = nt * p.bn;
     const long long row = static_cast<long long>(m0) + 32 * q + lane;
     const bool row_ok = row < p.M;
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (NACC * p.bn);
@@ -273,14 +321,15 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 #pragma unroll 1
       for (int a = 0; a < NACC; ++a) {
 #pragma unroll 1
-        for (int c = 0; c < p.bn; c += 16) {
+        for (int c = c0; c < p.bn; c += 32) {
           uint32_t r[16];
           tmem_ld16(tbase + a * p.bn + c, r);
           tmem_wait16(r);
           const int n = n0 + c;
           if (!row_ok) continue;
           if (EPI == EPI_F32) {
-            float* o = static_cast<float*>(p.out[0]) + row * p.ld_out + n;
+            float* o = static_cast<float*>(p.out[0]) + ks * p.split_stride + row * p.ld_out +
+                       a * p.out_acc_col + n;
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               if (n + 4 * h < p.N) {
@@ -309,7 +358,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       }
     } else if (EPI == EPI_SWIGLU_FWD) {
 #pragma unroll 1
-      for (int c = 0; c < p.bn; c += 16) {
+      for (int c = c0; c < p.bn; c += 32) {
         uint32_t rg[16], ru[16];
         tmem_ld16(tbase + c, rg);
         tmem_ld16(tbase + p.bn + c, ru);
@@ -336,7 +385,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       }
     } else if (EPI == EPI_SWIGLU_BWD) {
 #pragma unroll 1
-      for (int c = 0; c < p.bn; c += 16) {
+      for (int c = c0; c < p.bn; c += 32) {
         const int n = n0 + c;
         uint4 gv[2], uv[2];
 #pragma unroll
@@ -369,7 +418,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
               const float g = e ? bf16hi(gw[j]) : bf16lo(gw[j]);
               const float u = e ? bf16hi(uw[j]) : bf16lo(uw[j]);
               const float da = __uint_as_float(r[8 * h + 2 * j + e]);
-              const float sg = 1.0f / (1.0f + __expf(-g));
+              const float sg = sigmoid_f(g);
               du[e] = da * g * sg;
               dg[e] = da * u * sg * (1.0f + g * (1.0f - sg));
             }
@@ -384,34 +433,42 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 #pragma unroll 1
       for (int ri = 0; ri < p.nrng; ++ri) {
         const OutRange& R = p.rng[ri];
-        const long long wlo = static_cast<long long>(m0) + 32 * q;
-        if (wlo + 31 < R.lo || wlo >= R.hi) continue;  // warp-uniform skip
-        const bool mine = row >= R.lo && row < R.hi;
-        const long long k = row - R.lo;
 #pragma unroll 1
-        for (int c = 0; c < p.bn; c += 16) {
+        for (int c = c0; c < p.bn; c += 32) {
+          const int n = n0 + c;
+          if (n >= p.N) break;  // warp-uniform: remaining chunks are padding columns
           uint32_t r[16];
           tmem_ld16(tbase + R.acc * p.bn + c, r);
           tmem_wait16(r);
-          if (!mine) continue;
+          if (!row_ok) continue;
+          if (R.trans) {
+            // out[n * ld + m]: lanes hold consecutive m -> coalesced across the warp
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const long long n = n0 + c + j;
-            if (n < p.N) {
-              float* dst = R.trans ? R.out + n * R.ld + k : R.out + k * R.ld + n;
-              atomicAdd(dst, __uint_as_float(r[j]) * p.alpha);
-            }
+            for (int j = 0; j < 16; ++j)
+              if (n + j < p.N) atomicAdd(R.out + static_cast<long long>(n + j) * R.ld + row, __uint_as_float(r[j]) * p.alpha);
+          } else {
+            // out[m * ld + n]: 16 consecutive columns of one row -> four 16-byte vector atomics
+            float* o = R.out + row * R.ld + n;
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              if (n + 4 * h < p.N)
+                atomicAdd(reinterpret_cast<float4*>(o + 4 * h),
+                          make_float4(__uint_as_float(r[4 * h]) * p.alpha, __uint_as_float(r[4 * h + 1]) * p.alpha,
+                                      __uint_as_float(r[4 * h + 2]) * p.alpha, __uint_as_float(r[4 * h + 3]) * p.alpha));
           }
         }
       }
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+    if (lane == 0) {
+      if (PAIR == 1) mbar_arrive(tempty0 + 8 * buf);
+      else mbar_arrive_cluster(mapa_shared(tempty0 + 8 * buf, 0));  // the MMA issuer's barrier
+    }
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int EPI>
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -425,6 +482,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = PAIR == 1 ? 0u : cluster_ctarank();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -433,8 +491,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     mbar_init(tfull0, 1);
     mbar_init(tfull0 + 8, 1);
-    mbar_init(tempty0, 4);
-    mbar_init(tempty0 + 8, 4);
+    mbar_init(tempty0, kEpiWarps * PAIR);
+    mbar_init(tempty0 + 8, kEpiWarps * PAIR);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -443,30 +501,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     for (int i = 0; i < kMaxMaps; ++i) tma_prefetch_desc(&p.maps[i]);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
-    tmem_relinquish();
+    if (PAIR == 1) {
+      tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+      tmem_relinquish();
+    } else {
+      tmem_alloc_pair(smem_u32(tmem_slot), p.tmem_cols);
+      tmem_relinquish_pair();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync_all();  // peer barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl wc{abort_flag, p.status, p.limit_ns};
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer<A_MN, B_MN, NACC>(p, tiles, full0, empty0, wc);
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR>(p, tiles, full0, empty0, wc, rank);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0)
-      gemm_mma<A_MN, B_MN, NACC>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc);
+    if (lane == 0 && rank == 0)
+      gemm_mma<A_MN, B_MN, NACC, PAIR>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc);
     __syncwarp();
   } else {
-    gemm_epilogue<NACC, EPI>(p, tfull0, tempty0, tmem_base, wc);
+    gemm_epilogue<NACC, EPI, PAIR>(p, tfull0, tempty0, tmem_base, wc, rank);
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync_all();  // no CTA leaves while its pair may still touch its memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if (PAIR == 1) tmem_dealloc(tmem_base, p.tmem_cols);
+    else tmem_dealloc_pair(tmem_base, p.tmem_cols);
   }
 }
 

@@ -163,13 +163,21 @@ int sm_count() {
 
 constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
 
-template <int A_MN, int B_MN, int NACC, int EPI>
-int launch_gemm(GemmArgs& a, cudaStream_t st, int phase, int max_ctas = 0) {
-  if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % 64))
+// Launch one GEMM.  PAIR = 2 runs clusters of two CTAs sharing 256-row tiles
+// (tcgen05 cta_group::2); the caller sets tiles_m = ceil(M / (128 * PAIR)).
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1>
+int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
+  static_assert(PAIR == 1 || (PAIR == 2 && !A_MN), "CTA pairs take a K-major A operand");
+  if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
     return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
-  a.stage_bytes = BM * BK * 2 + NACC * a.bn * BK * 2;
+  a.stage_bytes = BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
   const int avail = kSmemLimit - 1024 - 256;
   a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
+  static const int stage_cap = [] {
+    const char* e = getenv("LORA_MLP_MAX_STAGES");  // tuning knob: cap the TMA ring depth
+    return e ? atoi(e) : 0;
+  }();
+  if (stage_cap >= 2) a.stages = std::min(a.stages, stage_cap);
   if (a.stages < 2) return fail(LORA_ERR_UNSUPPORTED, "internal: stage does not fit");
   int cols = 2 * NACC * a.bn;
   uint32_t tc = 32;
@@ -183,11 +191,27 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase, int max_ctas = 0) {
   const long long tiles = static_cast<long long>(a.tiles_m) * a.tiles_n * a.splits;
   if (tiles <= 0) return LORA_OK;
   if (tiles > 0x7fffffffLL) return fail(LORA_ERR_UNSUPPORTED, "too many tiles");
-  int grid = static_cast<int>(std::min<long long>(tiles, max_ctas > 0 ? max_ctas : sm_count()));
-  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI>;
+  const int units = static_cast<int>(std::min<long long>(tiles, sm_count() / PAIR));
+  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR>;
   CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   PhaseScope ps(st, phase);
-  kern<<<grid, kGemmThreads, smem, st>>>(a);
+  if (PAIR == 1) {
+    kern<<<units, kGemmThreads, smem, st>>>(a);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * PAIR, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = PAIR;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
+  }
   CUDA_TRY(cudaGetLastError());
   return LORA_OK;
 }
@@ -247,8 +271,21 @@ int launch_rms_bwd(cudaStream_t st, const float* dH, const void* X, const void* 
 
 // --------------------------------------------------------------- layouts
 struct WsLayout {
-  size_t status, Q, Qd, dG, dU, dH, total;
+  size_t status, Q, Qd, dG, dU, dH, part, total;
 };
+
+// K-split count of a rank-r projection: about two waves of CTAs on a 148-SM part,
+// at most 8 splits (fixed, so workspace sizes do not depend on the device).
+constexpr int kProjTargetCtas = 296;
+constexpr int kProjMaxSplits = 8;
+int proj_splits(long long T, long long K) {
+  const long long tiles = (T + 127) / 128;
+  const long long nkb = (K + 63) / 64;
+  long long s = std::max<long long>(1, (kProjTargetCtas + tiles - 1) / tiles);
+  s = std::min<long long>(std::min<long long>(s, kProjMaxSplits), nkb);
+  const long long per = (nkb + s - 1) / s;
+  return static_cast<int>((nkb + per - 1) / per);
+}
 
 int check_dims(const lora_mlp_dims* D) {
   if (!D) return fail(LORA_ERR_INVALID_ARG, "dims is NULL");
@@ -294,6 +331,12 @@ WsLayout ws_layout(const lora_mlp_dims* D) {
   L.dG = o; o = up256(o + T * f * 2);
   L.dU = o; o = up256(o + T * f * 2);
   L.dH = o; o = up256(o + T * d * 4);
+  size_t part = 0;
+  part = std::max(part, size_t(proj_splits(T, d)) * T * 2 * rp);   // P  = s H [Ag|Au]^T
+  part = std::max(part, size_t(proj_splits(T, f)) * T * rp);       // Pd = s Act Ad^T
+  part = std::max(part, size_t(proj_splits(T, d)) * T * rp);       // Qd = s dY Bd
+  part = std::max(part, size_t(proj_splits(T, f)) * T * 2 * rp);   // Q  = s [dG Bg | dU Bu]
+  L.part = o; o = up256(o + part * 4);
   L.total = o;
   return L;
 }
@@ -346,6 +389,30 @@ void set_seg(GemmArgs& a, int s, int amap, int ak0, int b0, int bk0, int b1, int
   a.seg[s].b_k0[1] = bk1;
   a.seg[s].k_len = klen;
   a.nseg = std::max(a.nseg, s + 1);
+}
+
+// Rank-r projection out[T x cols] (bf16) = scale * sum of K-split fp32 partials.
+// The GEMM args must already hold maps/segments/M/N/bn/tiles and NACC columns.
+template <int B_MN, int NACC>
+int launch_proj(GemmArgs& a, long long T, long long K, int cols, float* part, void* out, float scale,
+                cudaStream_t st, int phase) {
+  const int s = proj_splits(T, K);
+  const long long nkb = (K + BK - 1) / BK;
+  const long long per = (nkb + s - 1) / s;
+  a.splits = s;
+  a.k_chunk = static_cast<int>(per * BK);
+  a.out[0] = part;
+  a.ld_out = cols;
+  a.split_stride = T * cols;
+  a.alpha = 1.0f;
+  TRY((launch_gemm<0, B_MN, NACC, EPI_F32>(a, st, phase)));
+  const long long n = T * cols;
+  const long long blocks = (n / 4 + 255) / 256;
+  PhaseScope ps(st, phase);
+  splitk_finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, s, T * cols, n, scale,
+                                                                        static_cast<uint16_t*>(out));
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
 }
 
 // Split the T reduction so that roughly two CTAs per SM are busy.
@@ -449,25 +516,31 @@ int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float*
 }
 
 int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B, int32_t b_mn,
-                   float* C, void* stream) {
+                   float* C, int32_t flags, void* stream) {
   if (M < 1 || N < 1 || K < 1 || M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31))
     return fail(LORA_ERR_INVALID_ARG, "bad M/N/K");
   if (M % 8 || N % 8 || K % 8) return fail(LORA_ERR_ALIGNMENT, "M, N, K must be multiples of 8");
   TRY(check_ptrs({A, B, C}));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   GemmArgs a = new_args(nullptr);
-  const int bn = b_mn ? (N >= 256 ? 256 : round_up(static_cast<int>(N), 64))
-                      : (N >= 256 ? 256 : round_up(static_cast<int>(N), 16));
+  const int pair = (flags & LORA_GEMM_CTA_PAIR) && !a_mn ? 2 : 1;
+  int bn = b_mn ? (N >= 256 ? 256 : round_up(static_cast<int>(N), 64))
+                : (N >= 256 ? 256 : round_up(static_cast<int>(N), 16));
+  if (pair == 2) bn = b_mn ? std::min(256, round_up(static_cast<int>(N), 128)) : std::max(bn, 32);
   if (a_mn) TRY(map_mn(&a.maps[0], A, K, M, M)); else TRY(map_k(&a.maps[0], A, M, K, K, 128));
-  if (b_mn) TRY(map_mn(&a.maps[1], B, K, N, N)); else TRY(map_k(&a.maps[1], B, N, K, K, bn));
+  if (b_mn) TRY(map_mn(&a.maps[1], B, K, N, N)); else TRY(map_k(&a.maps[1], B, N, K, K, bn / pair));
   set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(K));
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.bn = bn;
-  a.tiles_m = static_cast<int>((M + BM - 1) / BM);
+  a.tiles_m = static_cast<int>((M + BM * pair - 1) / (BM * pair));
   a.tiles_n = static_cast<int>((N + bn - 1) / bn);
   a.out[0] = C;
   a.ld_out = N;
+  if (pair == 2) {
+    if (b_mn) return launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_OTHER);
+    return launch_gemm<0, 0, 1, EPI_F32, 2>(a, st, PH_OTHER);
+  }
   if (!a_mn && !b_mn) return launch_gemm<0, 0, 1, EPI_F32>(a, st, PH_OTHER);
   if (!a_mn && b_mn) return launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_OTHER);
   if (a_mn && !b_mn) return launch_gemm<1, 0, 1, EPI_F32>(a, st, PH_OTHER);
@@ -500,6 +573,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
   TRY(launch_rms_fwd(st, X, rms_w, H, rstd, T, d, D->eps));
 
   // S2: P = s * [H Ag^T | H Au^T]  (rank-r projections, padded to rp columns each)
+  float* part = at<float>(workspace, WL.part);
   {
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
@@ -507,26 +581,27 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     TRY(map_k(&a.maps[2], A->Au, r, d, d, rp));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
     a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
-    a.out[0] = P; a.ld_out = 2 * rp; a.out_acc_col = rp; a.alpha = s;
-    TRY((launch_gemm<0, 0, 2, EPI_BF16>(a, st, PH_P_GU)));
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1; a.out_acc_col = rp;
+    TRY((launch_proj<0, 2>(a, T, d, 2 * rp, part, P, s, st, PH_P_GU)));
   }
   // S3: G = H Wg^T + P_g Bg^T, U = H Wu^T + P_u Bu^T, Act = silu(G) * U
   {
     GemmArgs a = new_args(status);
+    const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
-    TRY(map_k(&a.maps[1], W->Wg, f, d, d, 128));
-    TRY(map_k(&a.maps[2], W->Wu, f, d, d, 128));
+    TRY(map_k(&a.maps[1], W->Wg, f, d, d, 128 / pair));
+    TRY(map_k(&a.maps[2], W->Wu, f, d, d, 128 / pair));
     TRY(map_k(&a.maps[3], P, T, 2 * rp, 2 * rp, 128));
-    TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128));
-    TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
+    TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128 / pair));
+    TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128 / pair));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
     set_seg(a, 1, 3, 0, 4, 0, -1, 0, rp);
     set_seg(a, 2, 3, rp, -1, 0, 5, 0, rp);
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (f + 127) / 128;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
-    TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD>(a, st, PH_GATEUP)));
+    if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2>(a, st, PH_GATEUP)));
+    else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD>(a, st, PH_GATEUP)));
   }
   // S4a: Pd = s * Act Ad^T
   {
@@ -536,23 +611,24 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
     a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
     a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
-    a.out[0] = Pd; a.ld_out = rp; a.alpha = s;
-    TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_P_D)));
+    TRY((launch_proj<0, 1>(a, T, f, rp, part, Pd, s, st, PH_P_D)));
   }
   // S4b: Y = Act Wd^T + Pd Bd^T
   {
     GemmArgs a = new_args(status);
     const int bn = d >= 256 ? 256 : round_up(d, 16);
+    const int pair = (T > 128 && bn >= 32) ? 2 : 1;
     TRY(map_k(&a.maps[0], Act, T, f, f, 128));
-    TRY(map_k(&a.maps[1], W->Wd, d, f, f, bn));
+    TRY(map_k(&a.maps[1], W->Wd, d, f, f, bn / pair));
     TRY(map_k(&a.maps[2], Pd, T, rp, rp, 128));
-    TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn));
+    TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn / pair));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
-    TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_DOWN)));
+    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_DOWN)));
+    else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_DOWN)));
   }
   return end_call(status, st);
 }
@@ -588,6 +664,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   const int qbn = rp <= 64 ? 64 : 128;
   TRY(begin_call(status, st));
 
+  float* part = at<float>(workspace, WL.part);
   // S5a: Qd = s * dY Bd
   {
     GemmArgs a = new_args(status);
@@ -595,23 +672,25 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY(map_mn(&a.maps[1], A->Bd, d, r, r));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     a.M = static_cast<int>(T); a.N = rp; a.bn = qbn; a.tiles_m = tm; a.tiles_n = 1;
-    a.out[0] = Qd; a.ld_out = rp; a.alpha = s;
-    TRY((launch_gemm<0, 1, 1, EPI_BF16>(a, st, PH_Q_D)));
+    TRY((launch_proj<1, 1>(a, T, d, rp, part, Qd, s, st, PH_Q_D)));
   }
   // S5b + S6: dAct = dY Wd + Qd Ad  ->  dG = dAct U silu'(G), dU = dAct silu(G)
   {
     GemmArgs a = new_args(status);
+    const int bn = f >= 256 ? 256 : round_up(f, 64);
+    const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
     TRY(map_k(&a.maps[0], dY, T, d, d, 128));
     TRY(map_mn(&a.maps[1], W->Wd, d, f, f));
     TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
     TRY(map_mn(&a.maps[3], A->Ad, r, f, f));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
-    const int bn = f >= 256 ? 256 : round_up(f, 64);
-    a.M = static_cast<int>(T); a.N = f; a.bn = bn; a.tiles_m = tm; a.tiles_n = (f + bn - 1) / bn;
+    a.M = static_cast<int>(T); a.N = f; a.bn = bn;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
-    TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
+    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
+    else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
   }
   // S7a: Q = s * [dG Bg | dU Bu]
   {
@@ -622,14 +701,14 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY(map_mn(&a.maps[3], A->Bu, f, r, r));
     set_seg(a, 0, 0, 0, 2, 0, -1, 0, f);
     set_seg(a, 1, 1, 0, -1, 0, 3, 0, f);
-    a.M = static_cast<int>(T); a.N = rp; a.bn = qbn; a.tiles_m = tm; a.tiles_n = 1;
-    a.out[0] = Q; a.ld_out = 2 * rp; a.out_acc_col = rp; a.alpha = s;
-    TRY((launch_gemm<0, 1, 2, EPI_BF16>(a, st, PH_Q_GU)));
+    a.M = static_cast<int>(T); a.N = rp; a.bn = qbn; a.tiles_m = tm; a.tiles_n = 1; a.out_acc_col = rp;
+    TRY((launch_proj<1, 2>(a, T, f, 2 * rp, part, Q, s, st, PH_Q_GU)));
   }
   // S8: dH = dG Wg + dU Wu + Q_g Ag + Q_u Au   (fp32)
   {
     GemmArgs a = new_args(status);
     const int bn = d >= 256 ? 256 : round_up(d, 64);
+    const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
     TRY(map_k(&a.maps[0], dG, T, f, f, 128));
     TRY(map_mn(&a.maps[1], W->Wg, f, d, d));
     TRY(map_k(&a.maps[2], dU, T, f, f, 128));
@@ -641,9 +720,11 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, f);
     set_seg(a, 2, 4, 0, 5, 0, -1, 0, rp);
     set_seg(a, 3, 4, rp, 6, 0, -1, 0, rp);
-    a.M = static_cast<int>(T); a.N = d; a.bn = bn; a.tiles_m = tm; a.tiles_n = (d + bn - 1) / bn;
+    a.M = static_cast<int>(T); a.N = d; a.bn = bn;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
-    TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
+    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_DH)));
+    else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
   }
   // S10: dX = RMSNorm backward (cached rstd)
   TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));
@@ -661,31 +742,35 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     zero6_kernel<<<296, 256, 0, st>>>(z);
     CUDA_TRY(cudaGetLastError());
   }
-  // S9: dAg = Q_g^T H, dAu = Q_u^T H  ([r x d]; rows of Q^T H)
+  // Adapter-gradient reductions over T: accumulator rows are the big dimension
+  // (M = d or f, MN-major A), columns the rank (N = r, MN-major narrow B).
+  const int rbn = r <= 64 ? 64 : 128;
+  // S9: dAg = Q_g^T H, dAu = Q_u^T H   ([r x d], written transposed from [d x r] tiles)
   {
     GemmArgs a = new_args(status);
-    const int bn = d >= 256 ? 256 : round_up(d, 64);
-    TRY(map_mn(&a.maps[0], Q, T, 2 * rp, 2 * rp));
-    TRY(map_mn(&a.maps[1], H, T, d, d));
-    set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
-    a.M = 2 * rp; a.N = d; a.bn = bn; a.tiles_m = (2 * rp + BM - 1) / BM; a.tiles_n = (d + bn - 1) / bn;
-    a.rng[0] = OutRange{gr->dAg, 0, 0, r, 0, d};
-    a.rng[1] = OutRange{gr->dAu, 0, rp, rp + r, 0, d};
+    TRY(map_mn(&a.maps[0], H, T, d, d));
+    TRY(map_mn(&a.maps[1], Q, T, r, 2 * rp));
+    TRY(map_mn(&a.maps[2], static_cast<const char*>(Q) + rp * 2, T, r, 2 * rp));
+    set_seg(a, 0, 0, 0, 1, 0, 2, 0, static_cast<int>(T));
+    a.M = d; a.N = r; a.bn = rbn; a.tiles_m = (d + BM - 1) / BM; a.tiles_n = 1;
+    a.rng[0] = OutRange{gr->dAg, 0, 1, d};
+    a.rng[1] = OutRange{gr->dAu, 1, 1, d};
     a.nrng = 2;
     choose_splits(a, T);
-    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DA_GU)));
+    TRY((launch_gemm<1, 1, 2, EPI_ATOMIC>(a, st, PH_RED_DA_GU)));
   }
-  // S7b: dBg = dG^T P_g, dBu = dU^T P_u  ([f x r]; transposed rows of P^T dG)
+  // S7b: dBg = dG^T P_g, dBu = dU^T P_u  ([f x r])
   {
     GemmArgs a = new_args(status);
-    const int bn = f >= 128 ? 128 : round_up(f, 64);
-    TRY(map_mn(&a.maps[0], P, T, 2 * rp, 2 * rp));
-    TRY(map_mn(&a.maps[1], dG, T, f, f));
-    TRY(map_mn(&a.maps[2], dU, T, f, f));
-    set_seg(a, 0, 0, 0, 1, 0, 2, 0, static_cast<int>(T));
-    a.M = 2 * rp; a.N = f; a.bn = bn; a.tiles_m = (2 * rp + BM - 1) / BM; a.tiles_n = (f + bn - 1) / bn;
-    a.rng[0] = OutRange{gr->dBg, 0, 0, r, 1, r};
-    a.rng[1] = OutRange{gr->dBu, 1, rp, rp + r, 1, r};
+    TRY(map_mn(&a.maps[0], dG, T, f, f));
+    TRY(map_mn(&a.maps[1], dU, T, f, f));
+    TRY(map_mn(&a.maps[2], P, T, r, 2 * rp));
+    TRY(map_mn(&a.maps[3], static_cast<const char*>(P) + rp * 2, T, r, 2 * rp));
+    set_seg(a, 0, 0, 0, 2, 0, -1, 0, static_cast<int>(T));
+    set_seg(a, 1, 1, 0, -1, 0, 3, 0, static_cast<int>(T));
+    a.M = f; a.N = r; a.bn = rbn; a.tiles_m = (f + BM - 1) / BM; a.tiles_n = 1;
+    a.rng[0] = OutRange{gr->dBg, 0, 0, r};
+    a.rng[1] = OutRange{gr->dBu, 1, 0, r};
     a.nrng = 2;
     choose_splits(a, T);
     TRY((launch_gemm<1, 1, 2, EPI_ATOMIC>(a, st, PH_RED_DB_GU)));
@@ -693,25 +778,23 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // S5c: dBd = dY^T Pd  ([d x r])
   {
     GemmArgs a = new_args(status);
-    const int bn = d >= 256 ? 256 : round_up(d, 64);
-    TRY(map_mn(&a.maps[0], Pd, T, rp, rp));
-    TRY(map_mn(&a.maps[1], dY, T, d, d));
+    TRY(map_mn(&a.maps[0], dY, T, d, d));
+    TRY(map_mn(&a.maps[1], Pd, T, r, rp));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
-    a.M = rp; a.N = d; a.bn = bn; a.tiles_m = 1; a.tiles_n = (d + bn - 1) / bn;
-    a.rng[0] = OutRange{gr->dBd, 0, 0, r, 1, r};
+    a.M = d; a.N = r; a.bn = rbn; a.tiles_m = (d + BM - 1) / BM; a.tiles_n = 1;
+    a.rng[0] = OutRange{gr->dBd, 0, 0, r};
     a.nrng = 1;
     choose_splits(a, T);
     TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DB_D)));
   }
-  // S6b: dAd = Qd^T Act  ([r x f])
+  // S6b: dAd = Qd^T Act  ([r x f], written transposed from [f x r] tiles)
   {
     GemmArgs a = new_args(status);
-    const int bn = f >= 256 ? 256 : round_up(f, 64);
-    TRY(map_mn(&a.maps[0], Qd, T, rp, rp));
-    TRY(map_mn(&a.maps[1], Act, T, f, f));
+    TRY(map_mn(&a.maps[0], Act, T, f, f));
+    TRY(map_mn(&a.maps[1], Qd, T, r, rp));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
-    a.M = rp; a.N = f; a.bn = bn; a.tiles_m = 1; a.tiles_n = (f + bn - 1) / bn;
-    a.rng[0] = OutRange{gr->dAd, 0, 0, r, 0, f};
+    a.M = f; a.N = r; a.bn = rbn; a.tiles_m = (f + BM - 1) / BM; a.tiles_n = 1;
+    a.rng[0] = OutRange{gr->dAd, 0, 1, f};
     a.nrng = 1;
     choose_splits(a, T);
     TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DA_D)));

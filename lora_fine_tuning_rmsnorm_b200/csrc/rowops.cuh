@@ -156,6 +156,23 @@ __global__ void quantize4_kernel(const uint16_t* __restrict__ W, long long nbloc
   }
 }
 
+// out[i] = bf16(scale * sum_s part[s * stride + i]) for the K-split partial sums
+// of a rank-r projection (deterministic: fixed summation order).
+__global__ void splitk_finalize_kernel(const float* __restrict__ part, int splits, long long stride,
+                                       long long n, float scale, uint16_t* __restrict__ out) {
+  const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i4 >= n) return;
+  float4 acc = *reinterpret_cast<const float4*>(part + i4);
+  for (int s = 1; s < splits; ++s) {
+    const float4 v = *reinterpret_cast<const float4*>(part + s * stride + i4);
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  uint2 o;
+  o.x = pack_bf16x2(acc.x * scale, acc.y * scale);
+  o.y = pack_bf16x2(acc.z * scale, acc.w * scale);
+  *reinterpret_cast<uint2*>(out + i4) = o;
+}
+
 struct ZeroList {
   float* p[6];
   long long n[6];

@@ -79,7 +79,7 @@ def lib() -> ctypes.CDLL:
         "lora_rmsnorm_fwd": [i64, i32, f32, vp, vp, vp, vp, vp],
         "lora_rmsnorm_bwd": [i64, i32, vp, vp, vp, vp, vp, vp],
         "lora_quantize_4bit": [vp, i64, i32, vp, vp, vp, vp],
-        "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, vp],
+        "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, i32, vp],
         "lora_mlp_timing_enable": [i32],
         "lora_mlp_timing_collect": [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
     }
@@ -193,10 +193,14 @@ def lora_quantize_4bit(W, codebook, codes, absmax, block=64, stream=None):
                                     _stream(stream)))
 
 
-def lora_gemm_bf16(A, a_mn, B, b_mn, C, stream=None):
+GEMM_CTA_PAIR = 1
+
+
+def lora_gemm_bf16(A, a_mn, B, b_mn, C, pair=False, stream=None):
     M, N = C.shape
     K = A.shape[0] if a_mn else A.shape[1]
-    _check(lib().lora_gemm_bf16(M, N, K, _p(A), int(a_mn), _p(B), int(b_mn), _p(C), _stream(stream)))
+    _check(lib().lora_gemm_bf16(M, N, K, _p(A), int(a_mn), _p(B), int(b_mn), _p(C),
+                                GEMM_CTA_PAIR if pair else 0, _stream(stream)))
 
 
 def timing_enable(on: bool = True):

@@ -71,7 +71,7 @@ def test_null_and_misaligned_pointers_rejected(L):
     assert rc == -1
     rc = L.lora_quantize_4bit(good, 128, 32, good, good, good, None)
     assert rc == -3
-    rc = L.lora_gemm_bf16(64, 60, 64, good, 0, good, 0, good, None)
+    rc = L.lora_gemm_bf16(64, 60, 64, good, 0, good, 0, good, 0, None)
     assert rc == -2
     g = ops.Grads()
     rc = L.lora_mlp_bwd(ctypes.byref(dims), good, good, good, ctypes.byref(w), ctypes.byref(a), good, good,

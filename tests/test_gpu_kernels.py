@@ -19,19 +19,22 @@ def rand_bf16(shape, seed, scale=1.0):
     return bits, synth.bf16_bits_to_f64(bits)
 
 
-GEMM_SIZES = [(128, 256, 64), (200, 136, 344), (64, 64, 8), (384, 512, 1024), (136, 72, 200)]
+GEMM_SIZES = [(128, 256, 64), (200, 136, 344), (64, 64, 8), (384, 512, 1024), (136, 72, 200), (520, 264, 128)]
 
 
+@pytest.mark.parametrize("pair", [False, True], ids=["1cta", "pair"])
 @pytest.mark.parametrize("a_mn", [0, 1])
 @pytest.mark.parametrize("b_mn", [0, 1])
 @pytest.mark.parametrize("M,N,K", GEMM_SIZES)
-def test_gemm_core(cuda_ok, M, N, K, a_mn, b_mn):
+def test_gemm_core(cuda_ok, M, N, K, a_mn, b_mn, pair):
+    if pair and a_mn:
+        pytest.skip("CTA pairs take a K-major A operand")
     Ab, Af = rand_bf16((K, M) if a_mn else (M, K), 1 + M + K)
     Bb, Bf = rand_bf16((K, N) if b_mn else (N, K), 2 + N + K)
     A = bf16_tensor(Ab)
     B = bf16_tensor(Bb)
     C = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
-    ops.lora_gemm_bf16(A, a_mn, B, b_mn, C)
+    ops.lora_gemm_bf16(A, a_mn, B, b_mn, C, pair=pair)
     torch.cuda.synchronize()
     Am = Af.T if a_mn else Af
     Bm = Bf.T if b_mn else Bf
