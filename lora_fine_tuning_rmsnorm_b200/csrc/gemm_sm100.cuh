@@ -134,37 +134,34 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
       const Seg& sg = p.seg[s];
       int kb0, kb1;
       seg_kb_range(p, s, ks, kb0, kb1);
+      // Bytes landing per stage for CTA rank rr.  Boxes that would lie entirely
+      // outside the matrix are skipped: the rows / columns they feed are never stored.
+      auto bytes_of = [&](uint32_t rr) -> uint32_t {
+        const int m0r = mbase + static_cast<int>(rr) * BM;
+        uint32_t by = 0;
+        if (A_MN) by += (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
+        else by += (m0r < p.M ? a_bytes : 0u);
+        const int nb0 = n0 + static_cast<int>(rr) * bnl;
+        uint32_t bb = 0;
+        if (B_MN) {
+          for (int c = 0; c < bnl / 64; ++c)
+            if (nb0 + 64 * c < p.N) bb += 8192u;
+        } else {
+          bb = nb0 < p.N ? b_bytes : 0u;
+        }
+#pragma unroll
+        for (int a = 0; a < NACC; ++a)
+          if (sg.b_map[a] >= 0) by += bb;
+        return by;
+      };
+      const uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
       for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t full = full0 + 8 * stage, empty = empty0 + 8 * stage;
         if (!mbar_wait(empty, phase ^ 1, wc, kDevTimeoutProducer)) {
           ok = false;
           break;
         }
-        // Bytes landing for CTA rank rr.  Boxes that would lie entirely outside the
-        // matrix are skipped: the rows / columns they feed are never stored.
-        auto bytes_of = [&](uint32_t rr) -> uint32_t {
-          const int m0r = mbase + static_cast<int>(rr) * BM;
-          uint32_t by = 0;
-          if (A_MN) by += (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
-          else by += (m0r < p.M ? a_bytes : 0u);
-          const int nb0 = n0 + static_cast<int>(rr) * bnl;
-          uint32_t bb = 0;
-          if (B_MN) {
-            for (int c = 0; c < bnl / 64; ++c)
-              if (nb0 + 64 * c < p.N) bb += 8192u;
-          } else {
-            bb = nb0 < p.N ? b_bytes : 0u;
-          }
-#pragma unroll
-          for (int a = 0; a < NACC; ++a)
-            if (sg.b_map[a] >= 0) by += bb;
-          return by;
-        };
-        if (PAIR == 1) {
-          mbar_expect_tx(full, bytes_of(0));
-        } else if (rank == 0) {
-          mbar_expect_tx(full, bytes_of(0) + bytes_of(1));
-        }
+        if (stage_tx) mbar_expect_tx(full, stage_tx);
         const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);
         const int m0 = mbase + static_cast<int>(rank) * BM;
         const int nb0 = n0 + static_cast<int>(rank) * bnl;
@@ -245,23 +242,34 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
         }
         tc_fence_after();
         const int rem = sg.k_len - kb * BK;
-        const int nsteps = rem >= BK ? BK / 16 : (rem + 15) / 16;
         const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
+        // descriptors of k-step 0; later k-steps only move the start address
+        // (+32 B in a K-major 128-byte row, +2048 B = 16 rows for MN-major)
+        const uint64_t ad0 = A_MN ? sdesc_sw128(sA, 8192, 1024) : sdesc_sw128(sA, 16, 1024);
+        constexpr uint32_t a_step = A_MN ? (2048 >> 4) : (32 >> 4);
+        constexpr uint32_t b_step = B_MN ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
         for (int a = 0; a < NACC; ++a) {
           if (sg.b_map[a] < 0) continue;
           const uint32_t sB = sA + a_bytes + a * b_bytes;
+          const uint64_t bd0 = B_MN ? sdesc_sw128(sB, 8192, 1024) : sdesc_sw128(sB, 16, 1024);
           const uint32_t d = tmem_base + buf * (NACC * p.bn) + a * p.bn;
-          for (int j = 0; j < nsteps; ++j) {
-            const uint64_t ad = A_MN ? sdesc_sw128(sA + j * 2048, 8192, 1024)
-                                     : sdesc_sw128(sA + j * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc_sw128(sB + j * 2048, 8192, 1024)
-                                     : sdesc_sw128(sB + j * 32, 16, 1024);
-            if (PAIR == 1) mma_bf16(d, ad, bd, idesc, (started >> a) & 1);
-            else mma_bf16_pair(d, ad, bd, idesc, (started >> a) & 1);
-            started |= 1u << a;
-            issued_any = true;
+          const uint32_t acc0 = (started >> a) & 1;
+          if (rem >= BK) {
+#pragma unroll
+            for (int j = 0; j < BK / 16; ++j) {
+              if (PAIR == 1) mma_bf16(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+              else mma_bf16_pair(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+            }
+          } else {
+            const int nsteps = (rem + 15) / 16;
+            for (int j = 0; j < nsteps; ++j) {
+              if (PAIR == 1) mma_bf16(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+              else mma_bf16_pair(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+            }
           }
+          started |= 1u << a;
+          issued_any = true;
         }
         // frees the smem stage (in both CTAs of a pair) once these MMAs finish
         if (PAIR == 1) mma_commit(empty0 + 8 * stage);

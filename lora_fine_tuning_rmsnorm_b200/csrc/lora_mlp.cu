@@ -13,7 +13,7 @@
 #include <mutex>
 #include <vector>
 
-#include "../../include/lora_mlp.h"
+#include "lora_mlp.h"
 #include "gemm_sm100.cuh"
 #include "rowops.cuh"
 

@@ -50,6 +50,19 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread sleeps (no issue slots) until the
+// phase completes or about `ns` nanoseconds pass, instead of spinning.
+__device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
 
 // Shared state for bounded waits inside one CTA.
 struct WaitCtl {
@@ -58,15 +71,12 @@ struct WaitCtl {
   uint64_t limit_ns;
 };
 
-// Wait until the phase with the given parity has completed.  Returns false when
-// the CTA is aborting (another role gave up) or the limit was reached.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
-  if (mbar_test(bar, parity)) return true;
+// Slow path of mbar_wait: sleep in suspend-hinted try_waits, checking the abort
+// flag and the time limit between them.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
   const uint64_t t0 = global_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_test(bar, parity)) return true;
+    if (mbar_test_sleep(bar, parity, 200000u)) return true;
     if (*c.abort_flag) return false;
     if (global_ns() - t0 > c.limit_ns) {
       if (c.status) atomicCAS(c.status, 0, code);
@@ -75,6 +85,12 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Wait
       return false;
     }
   }
+}
+// Wait until the phase with the given parity has completed.  Returns false when
+// the CTA is aborting (another role gave up) or the limit was reached.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, c, code);
 }
 
 // ----------------------------------------------------------------------- TMA
