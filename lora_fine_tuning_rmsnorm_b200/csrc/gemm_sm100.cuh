@@ -114,7 +114,10 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const Wai
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int PAIR>
+// FUSE = 1 (gate/up): the two B operands of a segment are two halves of ONE
+// N = 2 * bn MMA (branch 0 -> columns [0, bn), branch 1 -> [bn, 2 bn)), so a k-step
+// issues one wide MMA instead of two; with PAIR = 2, CTA rank r loads branch r.
+template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                               uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
@@ -141,7 +144,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         uint32_t by = 0;
         if (A_MN) by += (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
         else by += (m0r < p.M ? a_bytes : 0u);
-        const int nb0 = n0 + static_cast<int>(rr) * bnl;
+        const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rr) * bnl;
         uint32_t bb = 0;
         if (B_MN) {
           for (int c = 0; c < bnl / 64; ++c)
@@ -164,7 +167,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         if (stage_tx) mbar_expect_tx(full, stage_tx);
         const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);
         const int m0 = mbase + static_cast<int>(rank) * BM;
-        const int nb0 = n0 + static_cast<int>(rank) * bnl;
+        const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rank) * bnl;
         const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
         const int k = kb * BK;
         const CUtensorMap* am = &p.maps[sg.a_map];
@@ -178,16 +181,28 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         } else if (m0 < p.M) {
           load(sA, am, sg.a_k0 + k, m0);
         }
+        if (FUSE) {
+          // branch r fills B rows [r * bn, (r + 1) * bn) of the wide tile; a CTA of a
+          // pair holds only its own branch
+          const uint32_t sB = sA + a_bytes;
 #pragma unroll
-        for (int a = 0; a < NACC; ++a) {
-          if (sg.b_map[a] < 0) continue;
-          const uint32_t sB = sA + a_bytes + a * b_bytes;
-          const CUtensorMap* bm = &p.maps[sg.b_map[a]];
-          if (B_MN) {
-            for (int c = 0; c < bnl / 64; ++c)
-              if (nb0 + 64 * c < p.N) load(sB + c * 8192, bm, nb0 + 64 * c, sg.b_k0[a] + k);
-          } else if (nb0 < p.N) {
-            load(sB, bm, sg.b_k0[a] + k, nb0);
+          for (int r = 0; r < 2; ++r) {
+            if (PAIR == 2 && static_cast<uint32_t>(r) != rank) continue;
+            const uint32_t dst = PAIR == 2 ? sB : sB + r * p.bn * BK * 2;
+            load(dst, &p.maps[sg.b_map[r]], sg.b_k0[r] + k, n0);
+          }
+        } else {
+#pragma unroll
+          for (int a = 0; a < NACC; ++a) {
+            if (sg.b_map[a] < 0) continue;
+            const uint32_t sB = sA + a_bytes + a * b_bytes;
+            const CUtensorMap* bm = &p.maps[sg.b_map[a]];
+            if (B_MN) {
+              for (int c = 0; c < bnl / 64; ++c)
+                if (nb0 + 64 * c < p.N) load(sB + c * 8192, bm, nb0 + 64 * c, sg.b_k0[a] + k);
+            } else if (nb0 < p.N) {
+              load(sB, bm, sg.b_k0[a] + k, nb0);
+            }
           }
         }
         issued_mask |= 1u << stage;
@@ -207,14 +222,14 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int PAIR>
+template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE>
 __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                          uint32_t empty0, uint32_t tfull0, uint32_t tempty0,
                                          uint32_t drain_bar, uint32_t tmem_base,
                                          const WaitCtl& wc) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
-  const uint32_t idesc = idesc_bf16(BM * PAIR, p.bn, A_MN, B_MN);
+  const uint32_t idesc = idesc_bf16(BM * PAIR, FUSE ? 2 * p.bn : p.bn, A_MN, B_MN);
   const uint32_t a_bytes = BM * BK * 2;
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn / PAIR) * BK * 2;
   int stage = 0;
@@ -249,7 +264,7 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
         constexpr uint32_t a_step = A_MN ? (2048 >> 4) : (32 >> 4);
         constexpr uint32_t b_step = B_MN ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
-        for (int a = 0; a < NACC; ++a) {
+        for (int a = 0; a < (FUSE ? 1 : NACC); ++a) {
           if (sg.b_map[a] < 0) continue;
           const uint32_t sB = sA + a_bytes + a * b_bytes;
           const uint64_t bd0 = B_MN ? sdesc_sw128(sB, 8192, 1024) : sdesc_sw128(sB, 16, 1024);
@@ -476,8 +491,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR>
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
+  static_assert(!FUSE || (NACC == 2 && !B_MN), "fused wide MMA: two K-major B halves");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + static_cast<size_t>(p.stages) * p.stage_bytes);
@@ -525,11 +541,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const WaitCtl wc{abort_flag, p.status, p.limit_ns};
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR>(p, tiles, full0, empty0, wc, rank);
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE>(p, tiles, full0, empty0, wc, rank);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
-      gemm_mma<A_MN, B_MN, NACC, PAIR>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc);
+      gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc);
     __syncwarp();
   } else {
     gemm_epilogue<NACC, EPI, PAIR>(p, tfull0, tempty0, tmem_base, wc, rank);

@@ -165,7 +165,7 @@ constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
 
 // Launch one GEMM.  PAIR = 2 runs clusters of two CTAs sharing 256-row tiles
 // (tcgen05 cta_group::2); the caller sets tiles_m = ceil(M / (128 * PAIR)).
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1>
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1, int FUSE = 0>
 int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   static_assert(PAIR == 1 || (PAIR == 2 && !A_MN), "CTA pairs take a K-major A operand");
   if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
@@ -192,7 +192,7 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   if (tiles <= 0) return LORA_OK;
   if (tiles > 0x7fffffffLL) return fail(LORA_ERR_UNSUPPORTED, "too many tiles");
   const int units = static_cast<int>(std::min<long long>(tiles, sm_count() / PAIR));
-  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR>;
+  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR, FUSE>;
   CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   PhaseScope ps(st, phase);
   if (PAIR == 1) {
@@ -584,24 +584,26 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1; a.out_acc_col = rp;
     TRY((launch_proj<0, 2>(a, T, d, 2 * rp, part, P, s, st, PH_P_GU)));
   }
-  // S3: G = H Wg^T + P_g Bg^T, U = H Wu^T + P_u Bu^T, Act = silu(G) * U
+  // S3: G = H Wg^T + P_g Bg^T, U = H Wu^T + P_u Bu^T, Act = silu(G) * U.
+  // One N = 256 MMA per k-step covers 128 gate and 128 up columns; the LoRA term is
+  // one K = 2rp extension [P_g | P_u] x [[Bg | 0]; [0 | Bu]]^T, the zero blocks
+  // coming from TMA out-of-range fill (Bu is read from column -rp).
   {
     GemmArgs a = new_args(status);
     const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
-    TRY(map_k(&a.maps[1], W->Wg, f, d, d, 128 / pair));
-    TRY(map_k(&a.maps[2], W->Wu, f, d, d, 128 / pair));
+    TRY(map_k(&a.maps[1], W->Wg, f, d, d, 128));
+    TRY(map_k(&a.maps[2], W->Wu, f, d, d, 128));
     TRY(map_k(&a.maps[3], P, T, 2 * rp, 2 * rp, 128));
-    TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128 / pair));
-    TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128 / pair));
+    TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128));
+    TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
-    set_seg(a, 1, 3, 0, 4, 0, -1, 0, rp);
-    set_seg(a, 2, 3, rp, -1, 0, 5, 0, rp);
+    set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
-    if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2>(a, st, PH_GATEUP)));
-    else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD>(a, st, PH_GATEUP)));
+    if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1>(a, st, PH_GATEUP)));
+    else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1>(a, st, PH_GATEUP)));
   }
   // S4a: Pd = s * Act Ad^T
   {
