@@ -182,6 +182,26 @@ int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float*
 int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B,
                    int32_t b_mn, float* C, int32_t flags, void* stream);
 
+/* Allocation-free rank-r projection.  The pages have no counterpart to this entry
+ * point; it exists for callers that cannot allocate device memory themselves, such
+ * as a plugin inside a host framework that owns the device memory and hands it only
+ * its input and output buffers, so it has nowhere to put a workspace.
+ *   P[T x rp] bf16 = scale * X A^T,  X [T x K] bf16, A [r x K] bf16, rp = r rounded up
+ *   to 16 (columns [r, rp) are written as 0).  Same result as the projection the
+ *   forward stores in the saved context (P there holds scale * H Ag^T at columns
+ *   [0, rp)).  K, r multiples of 8, 8 <= r <= 128.
+ * The K-split fp32 partial sums go to a fixed 16 MiB array inside the library
+ * (4 Mi floats, held on every GPU that loads the library until the process exits);
+ * sizes with splits * T * rp above that are rejected with LORA_ERR_UNSUPPORTED.
+ * No cudaMalloc/cudaFree or other allocation is made.  The first call on each
+ * device looks up that array's device address (cudaGetSymbolAddress, with the
+ * device current) and caches it; make that first call before any stream capture.
+ * All calls share the array: calls that can overlap on the GPU (different streams,
+ * or several host threads) race on it and must be serialised by the caller.  Every
+ * partial-sum element is rewritten by each call, so nothing has to be cleared. */
+int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, const void* X, const void* A,
+                              void* P, void* stream);
+
 /* Per-phase timing.  With timing enabled, every kernel launch of the calls above
  * is bracketed by CUDA events on the caller's stream.  lora_mlp_timing_collect()
  * synchronises those events and returns, per phase id, the summed milliseconds and

@@ -428,6 +428,36 @@ void choose_splits(GemmArgs& a, long long K) {
 
 }  // namespace
 
+// ---------------------------------------------------- allocation-free variant
+// Scratch for lora_lowrank_proj_noalloc: the K-split fp32 partial sums live in a
+// file-scope device array instead of caller memory.  Every GPU that loads this
+// library holds it until the process exits.
+constexpr size_t kNoAllocScratchFloats = size_t(4) << 20;  // 16 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Host code may not use &g_noalloc_scratch as a device address (in host code the
+// name denotes a host-side stand-in), so the device address is looked up once per
+// device, with that device current, and cached.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(float** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(LORA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(LORA_ERR_CUDA, "cudaGetSymbolAddress(no-alloc scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return LORA_OK;
+}
+
 // ======================================================================= ABI
 extern "C" {
 
@@ -802,6 +832,33 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DA_D)));
   }
   return end_call(status, st);
+}
+
+int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, const void* X, const void* A,
+                              void* P, void* stream) {
+  if (T < 1 || T >= (1LL << 31) || K < 8 || r < 8 || r > 128)
+    return fail(LORA_ERR_INVALID_ARG, "bad T/K/r (%lld, %d, %d)", (long long)T, K, r);
+  if (K % 8 || r % 8) return fail(LORA_ERR_ALIGNMENT, "K and r must be multiples of 8");
+  TRY(check_ptrs({X, A, P}));
+  const int rp = round_up(r, 16);
+  const int splits = proj_splits(T, K);
+  const size_t need = static_cast<size_t>(splits) * static_cast<size_t>(T) * rp;
+  if (need > kNoAllocScratchFloats)
+    return fail(LORA_ERR_UNSUPPORTED,
+                "T x rp x splits = %lld x %d x %d fp32 partial sums exceed the %zu-float no-alloc scratch",
+                (long long)T, rp, splits, kNoAllocScratchFloats);
+  float* part = nullptr;
+  TRY(noalloc_scratch(&part));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every partial-sum element is overwritten by the split GEMM (all T rows and rp
+  // columns of each split), so the scratch needs no clearing between calls.
+  GemmArgs a = new_args(nullptr);
+  TRY(map_k(&a.maps[0], X, T, K, K, 128));
+  TRY(map_k(&a.maps[1], A, r, K, K, rp));
+  set_seg(a, 0, 0, 0, 1, 0, -1, 0, K);
+  a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
+  a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
+  return launch_proj<0, 1>(a, T, K, rp, part, P, scale, st, PH_OTHER);
 }
 
 }  // extern "C"

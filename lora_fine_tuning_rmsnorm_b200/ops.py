@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         "lora_rmsnorm_bwd": [i64, i32, vp, vp, vp, vp, vp, vp],
         "lora_quantize_4bit": [vp, i64, i32, vp, vp, vp, vp],
         "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, i32, vp],
+        "lora_lowrank_proj_noalloc": [i64, i32, i32, f32, vp, vp, vp, vp],
         "lora_mlp_timing_enable": [i32],
         "lora_mlp_timing_collect": [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
     }
@@ -201,6 +202,13 @@ def lora_gemm_bf16(A, a_mn, B, b_mn, C, pair=False, stream=None):
     K = A.shape[0] if a_mn else A.shape[1]
     _check(lib().lora_gemm_bf16(M, N, K, _p(A), int(a_mn), _p(B), int(b_mn), _p(C),
                                 GEMM_CTA_PAIR if pair else 0, _stream(stream)))
+
+
+def lora_lowrank_proj_noalloc(X, A, P, scale, stream=None):
+    """P[T x rp] = scale * X A^T using the library's fixed device scratch (no allocation)."""
+    T, K = X.shape
+    r = A.shape[0]
+    _check(lib().lora_lowrank_proj_noalloc(T, K, r, scale, _p(X), _p(A), _p(P), _stream(stream)))
 
 
 def timing_enable(on: bool = True):
