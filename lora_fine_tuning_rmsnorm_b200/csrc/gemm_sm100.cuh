@@ -44,12 +44,15 @@ enum Epi : int {
   EPI_ATOMIC = 4       // accumulator a atomically added into fp32 output rng[a] (split-K reductions)
 };
 
+enum Hint : int { HINT_NONE = 0, HINT_EVICT_FIRST = 1, HINT_EVICT_LAST = 2 };
+
 struct Seg {
   int a_map;
   int a_k0;
   int b_map[2];  // -1: this segment does not feed that accumulator
   int b_k0[2];
   int k_len;
+  int a_hint, b_hint;  // L2 eviction priority of the A / B loads (Hint)
 };
 
 struct OutRange {
@@ -66,6 +69,9 @@ struct GemmArgs {
   int M, N;  // valid rows / valid columns per accumulator
   int bn;    // N tile per accumulator (multiple of 16; multiple of 64 when B is MN-major)
   int tiles_m, tiles_n, splits;
+  int raster_n;    // 0: M-fastest tile order; 1: N-fastest
+  int mn3d_a, mn3d_b;  // 1: that MN-major operand's maps are 3-D {64, K, MN/64} views (one box per tile)
+  int stream_out;  // 1: epilogue stores are streaming (evict-first in L2)
   int k_chunk;  // split-K chunk in elements (multiple of BK) when splits > 1
   int stages;
   uint32_t stage_bytes;
@@ -85,10 +91,17 @@ struct GemmArgs {
 
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
 __device__ __forceinline__ void decode_tile(const GemmArgs& p, int t, int& mt, int& nt, int& ks) {
-  mt = t % p.tiles_m;
-  t /= p.tiles_m;
-  nt = t % p.tiles_n;
-  ks = t / p.tiles_n;
+  if (p.raster_n) {
+    nt = t % p.tiles_n;
+    t /= p.tiles_n;
+    mt = t % p.tiles_m;
+    ks = t / p.tiles_m;
+  } else {
+    mt = t % p.tiles_m;
+    t /= p.tiles_m;
+    nt = t % p.tiles_n;
+    ks = t / p.tiles_n;
+  }
 }
 
 __device__ __forceinline__ void seg_kb_range(const GemmArgs& p, int s, int ks, int& lo, int& hi) {
@@ -128,6 +141,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   uint32_t issued_mask = 0, issued_par = 0;
   const uint32_t a_bytes = BM * BK * 2;
   const uint32_t b_bytes = static_cast<uint32_t>(bnl) * BK * 2;
+  const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
   bool ok = true;
   for (int t = unit0; t < total && ok; t += nunits) {
     int mt, nt, ks;
@@ -142,13 +156,17 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
       auto bytes_of = [&](uint32_t rr) -> uint32_t {
         const int m0r = mbase + static_cast<int>(rr) * BM;
         uint32_t by = 0;
-        if (A_MN) by += (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
+        if (A_MN) by += p.mn3d_a ? (m0r < p.M ? 16384u : 0u) : (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
         else by += (m0r < p.M ? a_bytes : 0u);
         const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rr) * bnl;
         uint32_t bb = 0;
         if (B_MN) {
-          for (int c = 0; c < bnl / 64; ++c)
-            if (nb0 + 64 * c < p.N) bb += 8192u;
+          if (p.mn3d_b) {
+            bb = nb0 < p.N ? b_bytes : 0u;
+          } else {
+            for (int c = 0; c < bnl / 64; ++c)
+              if (nb0 + 64 * c < p.N) bb += 8192u;
+          }
         } else {
           bb = nb0 < p.N ? b_bytes : 0u;
         }
@@ -171,16 +189,31 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
         const int k = kb * BK;
         const CUtensorMap* am = &p.maps[sg.a_map];
+        int hint = sg.a_hint;
         auto load = [&](uint32_t dst, const CUtensorMap* m, int x, int y) {
-          if (PAIR == 1) tma_load_2d(dst, m, bar, x, y);
-          else tma_load_2d_pair(dst, m, bar, x, y);
+          if (hint == HINT_NONE) {
+            if (PAIR == 1) tma_load_2d(dst, m, bar, x, y);
+            else tma_load_2d_pair(dst, m, bar, x, y);
+          } else {
+            const uint64_t pol = hint == HINT_EVICT_LAST ? pol_last : pol_first;
+            if (PAIR == 1) tma_load_2d_hint(dst, m, bar, x, y, pol);
+            else tma_load_2d_pair_hint(dst, m, bar, x, y, pol);
+          }
         };
-        if (A_MN) {
+        // one 3-D box = all 64-column chunks of an MN-major operand tile, K rows [y, y + 64)
+        auto load3 = [&](uint32_t dst, const CUtensorMap* m, int y, int z) {
+          if (PAIR == 1) tma_load_3d(dst, m, bar, 0, y, z);
+          else tma_load_3d_pair(dst, m, bar, 0, y, z);
+        };
+        if (A_MN && p.mn3d_a) {
+          if (m0 < p.M) load3(sA, am, sg.a_k0 + k, m0 / 64);
+        } else if (A_MN) {
           if (m0 < p.M) load(sA, am, m0, sg.a_k0 + k);
           if (m0 + 64 < p.M) load(sA + 8192, am, m0 + 64, sg.a_k0 + k);
         } else if (m0 < p.M) {
           load(sA, am, sg.a_k0 + k, m0);
         }
+        hint = sg.b_hint;
         if (FUSE) {
           // branch r fills B rows [r * bn, (r + 1) * bn) of the wide tile; a CTA of a
           // pair holds only its own branch
@@ -197,7 +230,9 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
             if (sg.b_map[a] < 0) continue;
             const uint32_t sB = sA + a_bytes + a * b_bytes;
             const CUtensorMap* bm = &p.maps[sg.b_map[a]];
-            if (B_MN) {
+            if (B_MN && p.mn3d_b) {
+              if (nb0 < p.N) load3(sB, bm, sg.b_k0[a] + k, nb0 / 64);
+            } else if (B_MN) {
               for (int c = 0; c < bnl / 64; ++c)
                 if (nb0 + 64 * c < p.N) load(sB + c * 8192, bm, nb0 + 64 * c, sg.b_k0[a] + k);
             } else if (nb0 < p.N) {
@@ -308,6 +343,12 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
   }
 }
 
+template <class V>
+__device__ __forceinline__ void st_out(V* ptr, const V& v, int streaming) {
+  if (streaming) __stcs(ptr, v);
+  else *ptr = v;
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -360,7 +401,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
                                        __uint_as_float(r[4 * h + 1]) * p.alpha,
                                        __uint_as_float(r[4 * h + 2]) * p.alpha,
                                        __uint_as_float(r[4 * h + 3]) * p.alpha);
-                *reinterpret_cast<float4*>(o + 4 * h) = v;
+                st_out(reinterpret_cast<float4*>(o + 4 * h), v, p.stream_out);
               }
             }
           } else {
@@ -373,7 +414,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
                 v.y = pack_bf16x2(__uint_as_float(r[8 * h + 2]) * p.alpha, __uint_as_float(r[8 * h + 3]) * p.alpha);
                 v.z = pack_bf16x2(__uint_as_float(r[8 * h + 4]) * p.alpha, __uint_as_float(r[8 * h + 5]) * p.alpha);
                 v.w = pack_bf16x2(__uint_as_float(r[8 * h + 6]) * p.alpha, __uint_as_float(r[8 * h + 7]) * p.alpha);
-                *reinterpret_cast<uint4*>(o + 8 * h) = v;
+                st_out(reinterpret_cast<uint4*>(o + 8 * h), v, p.stream_out);
               }
             }
           }
@@ -401,9 +442,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             pu[j] = pack_bf16x2(u0, u1);
             pa[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
           }
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[2]) + off + 8 * h) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h), make_uint4(pg[0], pg[1], pg[2], pg[3]), p.stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h), make_uint4(pu[0], pu[1], pu[2], pu[3]), p.stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[2]) + off + 8 * h), make_uint4(pa[0], pa[1], pa[2], pa[3]), p.stream_out);
         }
       }
     } else if (EPI == EPI_SWIGLU_BWD) {
@@ -448,8 +489,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             pdg[j] = pack_bf16x2(dg[0], dg[1]);
             pdu[j] = pack_bf16x2(du[0], du[1]);
           }
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h) = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h) = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h), make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]), p.stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h), make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]), p.stream_out);
         }
       }
     } else if (EPI == EPI_ATOMIC) {

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -103,6 +104,22 @@ int map_k(CUtensorMap* m, const void* p, uint64_t rows, uint64_t K, uint64_t ld,
 // Operand with M/N contiguous: [K x MN], box 64 (MN) x 64 (K).
 int map_mn(CUtensorMap* m, const void* p, uint64_t K, uint64_t MN, uint64_t ld) {
   return make_map(m, p, MN, K, ld, 64, 64);
+}
+// The same operand as a 3-D view {64 elements, K rows, MN/64 chunks} (MN % 64 == 0),
+// box {64, 64, chunks}: one load fills `chunks` chunk-major 8 KB sub-tiles.
+int map_mn3(CUtensorMap* m, const void* p, uint64_t K, uint64_t MN, uint64_t ld, uint32_t chunks) {
+  TRY(get_encoder());
+  cuuint64_t dims[3] = {64, K, MN / 64};
+  cuuint64_t strides[2] = {ld * 2, 128};
+  cuuint32_t box[3] = {64, 64, chunks};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d): K=%llu MN=%llu ld=%llu chunks=%u",
+                static_cast<int>(r), (unsigned long long)K, (unsigned long long)MN, (unsigned long long)ld, chunks);
+  return LORA_OK;
 }
 
 // --------------------------------------------------------------------- timing
@@ -276,15 +293,29 @@ struct WsLayout {
 
 // K-split count of a rank-r projection: about two waves of CTAs on a 148-SM part,
 // at most 8 splits (fixed, so workspace sizes do not depend on the device).
-constexpr int kProjTargetCtas = 296;
-constexpr int kProjMaxSplits = 8;
+constexpr int kProjMaxSplits = 16;
+// Number of K splits for `tiles` output tiles over nkb k-blocks: the split that
+// fills whole waves of a 148-SM part best (at most max_splits), preferring fewer
+// splits among those within 3 % of the best.  Depends only on the sizes, so
+// workspace sizes do not depend on the device.
+int balanced_splits(long long tiles, long long nkb, int max_splits) {
+  const double sms = 148.0;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= max_splits && s <= nkb; ++s) {
+    const long long per = (nkb + s - 1) / s;
+    const long long ss = (nkb + per - 1) / per;        // splits actually formed
+    const double w = static_cast<double>(tiles * ss) / sms;
+    double eff = w / std::ceil(w);
+    if (tiles * ss < sms) eff = w;                      // a partial single wave
+    if (eff > best_eff + 0.03) { best_eff = eff; best = static_cast<int>(ss); }
+  }
+  return best;
+}
 int proj_splits(long long T, long long K) {
   const long long tiles = (T + 127) / 128;
   const long long nkb = (K + 63) / 64;
-  long long s = std::max<long long>(1, (kProjTargetCtas + tiles - 1) / tiles);
-  s = std::min<long long>(std::min<long long>(s, kProjMaxSplits), nkb);
-  const long long per = (nkb + s - 1) / s;
-  return static_cast<int>((nkb + per - 1) / per);
+  return balanced_splits(tiles, nkb, kProjMaxSplits);
 }
 
 int check_dims(const lora_mlp_dims* D) {
@@ -380,6 +411,13 @@ GemmArgs new_args(int* status) {
   return a;
 }
 
+void set_hints(GemmArgs& a, int a_hint, int b_hint) {
+  for (int s = 0; s < a.nseg; ++s) {
+    a.seg[s].a_hint = a_hint;
+    a.seg[s].b_hint = b_hint;
+  }
+}
+
 void set_seg(GemmArgs& a, int s, int amap, int ak0, int b0, int bk0, int b1, int bk1, int klen) {
   a.seg[s].a_map = amap;
   a.seg[s].a_k0 = ak0;
@@ -415,13 +453,13 @@ int launch_proj(GemmArgs& a, long long T, long long K, int cols, float* part, vo
   return LORA_OK;
 }
 
-// Split the T reduction so that roughly two CTAs per SM are busy.
+// Split the T reduction of an adapter-gradient GEMM so that the tiles fill whole
+// waves (at most 12 splits: every split adds one set of fp32 atomics per output).
 void choose_splits(GemmArgs& a, long long K) {
   const long long tiles = static_cast<long long>(a.tiles_m) * a.tiles_n;
   const long long nkb = (K + BK - 1) / BK;
-  long long want = std::max<long long>(1, (2LL * sm_count() + tiles - 1) / tiles);
-  want = std::min(want, nkb);
-  long long per = (nkb + want - 1) / want;
+  const int s = balanced_splits(tiles, nkb, 12);
+  const long long per = (nkb + s - 1) / s;
   a.k_chunk = static_cast<int>(per * BK);
   a.splits = static_cast<int>((nkb + per - 1) / per);
 }
@@ -557,8 +595,15 @@ int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn,
   int bn = b_mn ? (N >= 256 ? 256 : round_up(static_cast<int>(N), 64))
                 : (N >= 256 ? 256 : round_up(static_cast<int>(N), 16));
   if (pair == 2) bn = b_mn ? std::min(256, round_up(static_cast<int>(N), 128)) : std::max(bn, 32);
-  if (a_mn) TRY(map_mn(&a.maps[0], A, K, M, M)); else TRY(map_k(&a.maps[0], A, M, K, K, 128));
-  if (b_mn) TRY(map_mn(&a.maps[1], B, K, N, N)); else TRY(map_k(&a.maps[1], B, N, K, K, bn / pair));
+  // MN-major operands whose contiguous extent is a multiple of 64 load one 3-D box per tile
+  a.mn3d_a = a_mn && M % 64 == 0;
+  a.mn3d_b = b_mn && N % 64 == 0;
+  if (a.mn3d_a) TRY(map_mn3(&a.maps[0], A, K, M, M, 2));
+  else if (a_mn) TRY(map_mn(&a.maps[0], A, K, M, M));
+  else TRY(map_k(&a.maps[0], A, M, K, K, 128));
+  if (a.mn3d_b) TRY(map_mn3(&a.maps[1], B, K, N, N, bn / pair / 64));
+  else if (b_mn) TRY(map_mn(&a.maps[1], B, K, N, N));
+  else TRY(map_k(&a.maps[1], B, N, K, K, bn / pair));
   set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(K));
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
@@ -632,6 +677,8 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
+    set_hints(a, HINT_EVICT_LAST, HINT_NONE);  // H is re-read by every N tile: keep it in L2
+    a.stream_out = 1;
     if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1>(a, st, PH_GATEUP)));
     else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1>(a, st, PH_GATEUP)));
   }
@@ -659,6 +706,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
+    a.stream_out = 1;
     if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_DOWN)));
     else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_DOWN)));
   }
@@ -712,9 +760,15 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     const int bn = f >= 256 ? 256 : round_up(f, 64);
     const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
     TRY(map_k(&a.maps[0], dY, T, d, d, 128));
-    TRY(map_mn(&a.maps[1], W->Wd, d, f, f));
     TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
-    TRY(map_mn(&a.maps[3], A->Ad, r, f, f));
+    a.mn3d_b = f % 64 == 0;
+    if (a.mn3d_b) {
+      TRY(map_mn3(&a.maps[1], W->Wd, d, f, f, bn / pair / 64));
+      TRY(map_mn3(&a.maps[3], A->Ad, r, f, f, bn / pair / 64));
+    } else {
+      TRY(map_mn(&a.maps[1], W->Wd, d, f, f));
+      TRY(map_mn(&a.maps[3], A->Ad, r, f, f));
+    }
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
     a.M = static_cast<int>(T); a.N = f; a.bn = bn;
@@ -742,12 +796,20 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     const int bn = d >= 256 ? 256 : round_up(d, 64);
     const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
     TRY(map_k(&a.maps[0], dG, T, f, f, 128));
-    TRY(map_mn(&a.maps[1], W->Wg, f, d, d));
     TRY(map_k(&a.maps[2], dU, T, f, f, 128));
-    TRY(map_mn(&a.maps[3], W->Wu, f, d, d));
     TRY(map_k(&a.maps[4], Q, T, 2 * rp, 2 * rp, 128));
-    TRY(map_mn(&a.maps[5], A->Ag, r, d, d));
-    TRY(map_mn(&a.maps[6], A->Au, r, d, d));
+    a.mn3d_b = d % 64 == 0;
+    if (a.mn3d_b) {
+      TRY(map_mn3(&a.maps[1], W->Wg, f, d, d, bn / pair / 64));
+      TRY(map_mn3(&a.maps[3], W->Wu, f, d, d, bn / pair / 64));
+      TRY(map_mn3(&a.maps[5], A->Ag, r, d, d, bn / pair / 64));
+      TRY(map_mn3(&a.maps[6], A->Au, r, d, d, bn / pair / 64));
+    } else {
+      TRY(map_mn(&a.maps[1], W->Wg, f, d, d));
+      TRY(map_mn(&a.maps[3], W->Wu, f, d, d));
+      TRY(map_mn(&a.maps[5], A->Ag, r, d, d));
+      TRY(map_mn(&a.maps[6], A->Au, r, d, d));
+    }
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, f);
     set_seg(a, 2, 4, 0, 5, 0, -1, 0, rp);
@@ -780,7 +842,9 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // S9: dAg = Q_g^T H, dAu = Q_u^T H   ([r x d], written transposed from [d x r] tiles)
   {
     GemmArgs a = new_args(status);
-    TRY(map_mn(&a.maps[0], H, T, d, d));
+    a.mn3d_a = d % 64 == 0;
+    if (a.mn3d_a) TRY(map_mn3(&a.maps[0], H, T, d, d, 2));
+    else TRY(map_mn(&a.maps[0], H, T, d, d));
     TRY(map_mn(&a.maps[1], Q, T, r, 2 * rp));
     TRY(map_mn(&a.maps[2], static_cast<const char*>(Q) + rp * 2, T, r, 2 * rp));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, static_cast<int>(T));
@@ -794,8 +858,14 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // S7b: dBg = dG^T P_g, dBu = dU^T P_u  ([f x r])
   {
     GemmArgs a = new_args(status);
-    TRY(map_mn(&a.maps[0], dG, T, f, f));
-    TRY(map_mn(&a.maps[1], dU, T, f, f));
+    a.mn3d_a = f % 64 == 0;
+    if (a.mn3d_a) {
+      TRY(map_mn3(&a.maps[0], dG, T, f, f, 2));
+      TRY(map_mn3(&a.maps[1], dU, T, f, f, 2));
+    } else {
+      TRY(map_mn(&a.maps[0], dG, T, f, f));
+      TRY(map_mn(&a.maps[1], dU, T, f, f));
+    }
     TRY(map_mn(&a.maps[2], P, T, r, 2 * rp));
     TRY(map_mn(&a.maps[3], static_cast<const char*>(P) + rp * 2, T, r, 2 * rp));
     set_seg(a, 0, 0, 0, 2, 0, -1, 0, static_cast<int>(T));
@@ -810,7 +880,9 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // S5c: dBd = dY^T Pd  ([d x r])
   {
     GemmArgs a = new_args(status);
-    TRY(map_mn(&a.maps[0], dY, T, d, d));
+    a.mn3d_a = d % 64 == 0;
+    if (a.mn3d_a) TRY(map_mn3(&a.maps[0], dY, T, d, d, 2));
+    else TRY(map_mn(&a.maps[0], dY, T, d, d));
     TRY(map_mn(&a.maps[1], Pd, T, r, rp));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
     a.M = d; a.N = r; a.bn = rbn; a.tiles_m = (d + BM - 1) / BM; a.tiles_n = 1;
@@ -822,7 +894,9 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // S6b: dAd = Qd^T Act  ([r x f], written transposed from [f x r] tiles)
   {
     GemmArgs a = new_args(status);
-    TRY(map_mn(&a.maps[0], Act, T, f, f));
+    a.mn3d_a = f % 64 == 0;
+    if (a.mn3d_a) TRY(map_mn3(&a.maps[0], Act, T, f, f, 2));
+    else TRY(map_mn(&a.maps[0], Act, T, f, f));
     TRY(map_mn(&a.maps[1], Qd, T, r, rp));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
     a.M = f; a.N = r; a.bn = rbn; a.tiles_m = (f + BM - 1) / BM; a.tiles_n = 1;
