@@ -63,7 +63,7 @@ enum lora_wfmt {
  * Limits: 1 <= T < 2^31; d, f multiples of 8 with 8 <= d <= 65536, 8 <= f;
  * r a multiple of 8 with 8 <= r <= 128.  scale = alpha / r (any finite value).
  * wfmt = LORA_WFMT_BF16 or LORA_WFMT_4BIT (then qblock must be 64 and d, f
- * multiples of 64). */
+ * multiples of 256). */
 typedef struct lora_mlp_dims {
   int64_t T;
   int32_t d, f, r;
@@ -79,6 +79,9 @@ typedef struct lora_mlp_dims {
  *                                           the row-major matrix in the low nibble
  *   absmax_g, absmax_u [f*d/64], absmax_d [d*f/64]  fp32 per-block absmax
  *   codebook [16] fp32                      code values (wfmt = LORA_WFMT_4BIT)
+ * With 4-bit weights the GEMMs stage the codes and absmax in shared memory and
+ * expand them to bf16 tiles in-kernel (w = bf16(codebook[idx] * absmax)) right
+ * before the tensor-core MMA; no bf16 copy of W is ever written to memory.
  * Unused members may be NULL. */
 typedef struct lora_mlp_weights {
   const void* Wg;

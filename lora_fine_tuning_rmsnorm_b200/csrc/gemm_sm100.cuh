@@ -32,9 +32,11 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kMaxStages = 8;
 constexpr int kMaxSegs = 4;
-constexpr int kMaxMaps = 8;
+constexpr int kMaxMaps = 10;
 constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16-column chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kDqWarps = 4;  // 4-bit weights: warps that expand codes into bf16 B tiles
+__host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps : 0); }
 
 enum Epi : int {
   EPI_F32 = 0,         // out[0] fp32 = acc_a * alpha at column a * out_acc_col (+ split * split_stride)
@@ -53,6 +55,8 @@ struct Seg {
   int b_k0[2];
   int k_len;
   int a_hint, b_hint;  // L2 eviction priority of the A / B loads (Hint)
+  int q4;              // 1: B comes from 4-bit codes (b_map = code map, b_am = absmax map)
+  int b_am[2];
 };
 
 struct OutRange {
@@ -87,6 +91,7 @@ struct GemmArgs {
   int nrng;
   int* status;
   unsigned long long limit_ns;
+  const float* codebook;  // 4-bit code values (16 fp32)
 };
 
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
@@ -130,7 +135,7 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const Wai
 // FUSE = 1 (gate/up): the two B operands of a segment are two halves of ONE
 // N = 2 * bn MMA (branch 0 -> columns [0, bn), branch 1 -> [bn, 2 bn)), so a k-step
 // issues one wide MMA instead of two; with PAIR = 2, CTA rank r loads branch r.
-template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE>
+template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                               uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
@@ -175,7 +180,16 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           if (sg.b_map[a] >= 0) by += bb;
         return by;
       };
-      const uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
+      uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
+      if (Q4 && sg.q4) {
+        // A tile + per branch: packed codes (bn x 32 B) and an absmax box (K-major:
+        // bn rows x 4 floats; MN-major: 64 K rows x 4 floats)
+        uint32_t by = a_bytes;
+#pragma unroll
+        for (int a = 0; a < (FUSE ? 2 : NACC); ++a)
+          if (sg.b_map[a] >= 0) by += p.bn * 32u + (B_MN ? 64u * 16u : p.bn * 16u);
+        stage_tx = by;
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t full = full0 + 8 * stage, empty = empty0 + 8 * stage;
         if (!mbar_wait(empty, phase ^ 1, wc, kDevTimeoutProducer)) {
@@ -214,7 +228,26 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           load(sA, am, sg.a_k0 + k, m0);
         }
         hint = sg.b_hint;
-        if (FUSE) {
+        if (Q4 && sg.q4) {
+          // 4-bit B: stage the codes and block absmax; the dequant warps expand them
+          const int nbr = FUSE ? 2 : NACC;
+          const uint32_t sQ = sA + a_bytes + nbr * b_bytes;
+          const uint32_t sM = sQ + nbr * p.bn * 32;
+#pragma unroll
+          for (int r = 0; r < (FUSE ? 2 : NACC); ++r) {
+            if (sg.b_map[r] < 0) continue;
+            const CUtensorMap* qm = &p.maps[sg.b_map[r]];
+            const CUtensorMap* mm = &p.maps[sg.b_am[r]];
+            const int kk = sg.b_k0[r] + k;
+            if (B_MN) {
+              load(sQ + r * p.bn * 32, qm, n0 / 2, kk);
+              load(sM + r * p.bn * 16, mm, (n0 / 64) & ~3, kk);
+            } else {
+              load(sQ + r * p.bn * 32, qm, kk / 2, n0);
+              load(sM + r * p.bn * 16, mm, (kk / 64) & ~3, n0);
+            }
+          }
+        } else if (FUSE) {
           // branch r fills B rows [r * bn, (r + 1) * bn) of the wide tile; a CTA of a
           // pair holds only its own branch
           const uint32_t sB = sA + a_bytes;
@@ -257,11 +290,11 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE>
+template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
 __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                          uint32_t empty0, uint32_t tfull0, uint32_t tempty0,
                                          uint32_t drain_bar, uint32_t tmem_base,
-                                         const WaitCtl& wc) {
+                                         const WaitCtl& wc, uint32_t dq0) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const uint32_t idesc = idesc_bf16(BM * PAIR, FUSE ? 2 * p.bn : p.bn, A_MN, B_MN);
@@ -287,6 +320,10 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
       seg_kb_range(p, s, ks, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        if (Q4 && !mbar_wait(dq0 + 8 * stage, phase, wc, kDevTimeoutMma)) {  // B tiles expanded
           ok = false;
           break;
         }
@@ -532,9 +569,93 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
+// 4-bit B producer (kDqWarps warps): for every stage, wait for the staged codes
+// and absmax, expand each 64-element block row w = code[idx] * absmax (fp32 product,
+// rounded once to bf16) into the 128-byte-swizzled bf16 B tile, make the writes
+// visible to the tensor core (async proxy) and arrive on the stage's dq barrier.
+// tab[b] = (code[b & 15], code[b >> 4]): both nibbles of one packed byte.
+template <int B_MN, int NACC, int FUSE>
+__device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, uint32_t full0, uint32_t dq0,
+                                             const float2* tab, const WaitCtl& wc) {
+  const int tid = threadIdx.x - kGemmThreads;  // 0 .. 32 * kDqWarps - 1
+  const int lane = threadIdx.x % 32;
+  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const uint32_t a_bytes = BM * BK * 2;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
+  const int nbr = FUSE ? 2 : NACC;
+  int stage = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    int mt, nt, ks;
+    decode_tile(p, t, mt, nt, ks);
+    const int n0 = nt * p.bn;
+    for (int s = 0; s < p.nseg && ok; ++s) {
+      const Seg& sg = p.seg[s];
+      int kb0, kb1;
+      seg_kb_range(p, s, ks, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutProducer) ? 1 : 0;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        if (sg.q4) {
+          uint8_t* base = tiles + static_cast<size_t>(stage) * p.stage_bytes;
+          const uint8_t* sQ = base + a_bytes + nbr * b_bytes;
+          const float* sM = reinterpret_cast<const float*>(sQ + nbr * p.bn * 32);
+          const int kk = kb * BK;
+          const int rows = p.bn;  // K-major: bn W rows; MN-major: 64 K rows x bn/64 chunks
+          for (int r = 0; r < nbr; ++r) {
+            if (sg.b_map[r] < 0) continue;
+            const uint8_t* q = sQ + r * p.bn * 32;
+            const float* am = sM + r * p.bn * 4;
+            uint8_t* dst = base + a_bytes + r * b_bytes;
+            for (int i = tid; i < rows; i += 32 * kDqWarps) {
+              const uint4* src;
+              float scale;
+              if (B_MN) {
+                const int c = i >> 6, krow = i & 63, chunks = p.bn >> 6;
+                src = reinterpret_cast<const uint4*>(q + krow * (chunks * 32) + c * 32);
+                scale = am[krow * 4 + ((n0 >> 6) & 3) + c];
+              } else {
+                src = reinterpret_cast<const uint4*>(q + i * 32);
+                scale = am[i * 4 + ((kk >> 6) & 3)];
+              }
+              const uint4 c0 = src[0], c1 = src[1];
+              const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+              uint8_t* row = dst + static_cast<size_t>(i) * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {  // 16-byte piece j = elements 8j .. 8j+7
+                uint32_t o[4];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  const float2 v = tab[(wv[j] >> (8 * b)) & 0xFF];
+                  o[b] = pack_bf16x2(v.x * scale, v.y * scale);
+                }
+                *reinterpret_cast<uint4*>(row + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq0 + 8 * stage);
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  }
+}
+
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE, int Q4>
+__global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
   static_assert(!FUSE || (NACC == 2 && !B_MN), "fused wide MMA: two K-major B halves");
+  static_assert(!Q4 || (PAIR == 1 && !A_MN), "4-bit B: single-CTA tiles, K-major A");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + static_cast<size_t>(p.stages) * p.stage_bytes);
@@ -544,8 +665,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const uint32_t tfull0 = empty0 + 8 * S;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t drain_bar = tempty0 + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  const uint32_t dq0 = drain_bar + 8;  // Q4: one barrier per stage (kDqWarps arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? S : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* tab = reinterpret_cast<float2*>(tmem_slot + 4);  // Q4: 256-entry nibble-pair table (8-byte aligned)
+  if (Q4)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) tab[i] = make_float2(p.codebook[i & 15], p.codebook[i >> 4]);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = PAIR == 1 ? 0u : cluster_ctarank();
 
@@ -559,6 +684,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     mbar_init(tempty0, kEpiWarps * PAIR);
     mbar_init(tempty0 + 8, kEpiWarps * PAIR);
     mbar_init(drain_bar, 1);
+    if (Q4)
+      for (int s = 0; s < S; ++s) mbar_init(dq0 + 8 * s, kDqWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -582,14 +709,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const WaitCtl wc{abort_flag, p.status, p.limit_ns};
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE>(p, tiles, full0, empty0, wc, rank);
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, wc, rank);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
-      gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc);
+      gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc, dq0);
     __syncwarp();
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     gemm_epilogue<NACC, EPI, PAIR>(p, tfull0, tempty0, tmem_base, wc, rank);
+  } else if (Q4) {
+    gemm_dequant<B_MN, NACC, FUSE>(p, tiles, full0, dq0, tab, wc);
   }
   tc_fence_before();
   __syncthreads();

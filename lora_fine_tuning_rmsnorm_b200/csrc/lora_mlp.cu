@@ -97,6 +97,37 @@ int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, ui
                 (unsigned long long)ld, box_inner, box_outer);
   return LORA_OK;
 }
+// Untyped 2-D map without swizzle (4-bit codes as bytes, block absmax as fp32).
+int make_map_raw(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint32_t esize, uint64_t inner,
+                 uint64_t outer, uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
+  TRY(get_encoder());
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * esize};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled (raw) failed (%d): inner=%llu outer=%llu box=%ux%u",
+                static_cast<int>(r), (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+  return LORA_OK;
+}
+// 4-bit weight W [rows x cols] (codes: rows x cols/2 bytes; absmax: rows x cols/64 fp32)
+// read with K = cols contiguous (forward use): boxes {32 B, n_rows} and {4 floats, n_rows}.
+int map_q4_k(CUtensorMap* mq, CUtensorMap* ma, const uint8_t* q, const float* am, uint64_t rows, uint64_t cols,
+             uint32_t n_rows) {
+  TRY(make_map_raw(mq, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cols / 2, rows, cols / 2, 32, n_rows));
+  return make_map_raw(ma, am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols / 64, rows, cols / 64, 4, n_rows);
+}
+// The same weight read with N = cols contiguous and K = rows (backward use): boxes
+// {n_cols / 2 B, 64 K rows} and {4 floats, 64 K rows}.
+int map_q4_mn(CUtensorMap* mq, CUtensorMap* ma, const uint8_t* q, const float* am, uint64_t rows, uint64_t cols,
+              uint32_t n_cols) {
+  TRY(make_map_raw(mq, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cols / 2, rows, cols / 2, n_cols / 2, 64));
+  return make_map_raw(ma, am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols / 64, rows, cols / 64, 4, 64);
+}
+
 // Operand with K contiguous: [rows x K], box 64 (K) x box_rows.
 int map_k(CUtensorMap* m, const void* p, uint64_t rows, uint64_t K, uint64_t ld, uint32_t box_rows) {
   return make_map(m, p, K, rows, ld, 64, box_rows);
@@ -182,13 +213,17 @@ constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
 
 // Launch one GEMM.  PAIR = 2 runs clusters of two CTAs sharing 256-row tiles
 // (tcgen05 cta_group::2); the caller sets tiles_m = ceil(M / (128 * PAIR)).
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1, int FUSE = 0>
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1, int FUSE = 0, int Q4 = 0>
 int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   static_assert(PAIR == 1 || (PAIR == 2 && !A_MN), "CTA pairs take a K-major A operand");
   if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
     return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
   a.stage_bytes = BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
-  const int avail = kSmemLimit - 1024 - 256;
+  // 4-bit B: per branch also the staged codes (bn x 32 B) and absmax (>= 1 KB)
+  if (Q4) a.stage_bytes += NACC * (a.bn * 32 + std::max(a.bn * 16, 1024));
+  a.stage_bytes = (a.stage_bytes + 1023) & ~1023u;
+  const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit nibble-pair table)
+  const int avail = kSmemLimit - 1024 - extra;
   a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
   static const int stage_cap = [] {
     const char* e = getenv("LORA_MLP_MAX_STAGES");  // tuning knob: cap the TMA ring depth
@@ -201,7 +236,7 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
   if (tc > 512) return fail(LORA_ERR_UNSUPPORTED, "internal: TMEM columns %d > 512", cols);
   a.tmem_cols = tc;
-  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + 256;
+  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + extra;
   // more than half of TMEM per CTA: keep one CTA per SM so allocation never waits
   if (tc > 256) smem = std::max(smem, kSmemLimit / 2 + 4096);
   a.limit_ns = wait_limit_ns();
@@ -209,15 +244,15 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   if (tiles <= 0) return LORA_OK;
   if (tiles > 0x7fffffffLL) return fail(LORA_ERR_UNSUPPORTED, "too many tiles");
   const int units = static_cast<int>(std::min<long long>(tiles, sm_count() / PAIR));
-  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR, FUSE>;
+  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR, FUSE, Q4>;
   CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   PhaseScope ps(st, phase);
   if (PAIR == 1) {
-    kern<<<units, kGemmThreads, smem, st>>>(a);
+    kern<<<units, gemm_threads(Q4), smem, st>>>(a);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(units * PAIR, 1, 1);
-    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.blockDim = dim3(gemm_threads(Q4), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -329,7 +364,7 @@ int check_dims(const lora_mlp_dims* D) {
   if (D->wfmt != LORA_WFMT_BF16 && D->wfmt != LORA_WFMT_4BIT) return fail(LORA_ERR_INVALID_ARG, "bad wfmt");
   if (D->wfmt == LORA_WFMT_4BIT) {
     if (D->qblock != 64) return fail(LORA_ERR_UNSUPPORTED, "qblock must be 64");
-    if (D->d % 64 || D->f % 64) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights need d, f multiples of 64");
+    if (D->d % 256 || D->f % 256) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights need d, f multiples of 256");
   }
   return LORA_OK;
 }
@@ -626,8 +661,10 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
                  const lora_mlp_adapters* A, void* Y, void* ctx, void* workspace, void* stream) {
   TRY(check_dims(D));
   if (!W || !A) return fail(LORA_ERR_INVALID_ARG, "weights/adapters is NULL");
-  if (D->wfmt != LORA_WFMT_BF16) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights are not built into this entry point yet");
-  TRY(check_ptrs({X, rms_w, Y, ctx, workspace, W->Wg, W->Wu, W->Wd, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd}));
+  const bool q4 = D->wfmt == LORA_WFMT_4BIT;
+  TRY(check_ptrs({X, rms_w, Y, ctx, workspace, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd}));
+  if (q4) TRY(check_ptrs({W->Qg, W->Qu, W->Qd, W->absmax_g, W->absmax_u, W->absmax_d, W->codebook}));
+  else TRY(check_ptrs({W->Wg, W->Wu, W->Wd}));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long T = D->T;
   const int d = D->d, f = D->f, r = D->r, rp = rp_of(D);
@@ -663,7 +700,26 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
   // One N = 256 MMA per k-step covers 128 gate and 128 up columns; the LoRA term is
   // one K = 2rp extension [P_g | P_u] x [[Bg | 0]; [0 | Bu]]^T, the zero blocks
   // coming from TMA out-of-range fill (Bu is read from column -rp).
-  {
+  if (q4) {
+    // 4-bit frozen weights: the codes are expanded to bf16 B tiles in shared memory
+    // by dequant warps inside the GEMM (single-CTA tiles)
+    GemmArgs a = new_args(status);
+    TRY(map_k(&a.maps[0], H, T, d, d, 128));
+    TRY(map_q4_k(&a.maps[1], &a.maps[6], W->Qg, W->absmax_g, f, d, 128));
+    TRY(map_q4_k(&a.maps[2], &a.maps[7], W->Qu, W->absmax_u, f, d, 128));
+    TRY(map_k(&a.maps[3], P, T, 2 * rp, 2 * rp, 128));
+    TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128));
+    TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
+    set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
+    a.seg[0].q4 = 1; a.seg[0].b_am[0] = 6; a.seg[0].b_am[1] = 7;
+    set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
+    a.codebook = W->codebook;
+    a.M = static_cast<int>(T); a.N = f; a.bn = 128;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (f + 127) / 128;
+    a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
+    a.stream_out = 1;
+    TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1, 1>(a, st, PH_GATEUP)));
+  } else {
     GemmArgs a = new_args(status);
     const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
@@ -693,7 +749,23 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     TRY((launch_proj<0, 1>(a, T, f, rp, part, Pd, s, st, PH_P_D)));
   }
   // S4b: Y = Act Wd^T + Pd Bd^T
-  {
+  if (q4) {
+    GemmArgs a = new_args(status);
+    const int bn = d >= 256 ? 256 : round_up(d, 16);
+    TRY(map_k(&a.maps[0], Act, T, f, f, 128));
+    TRY(map_q4_k(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn));
+    TRY(map_k(&a.maps[2], Pd, T, rp, rp, 128));
+    TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
+    a.seg[0].q4 = 1; a.seg[0].b_am[0] = 4;
+    set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    a.codebook = W->codebook;
+    a.M = static_cast<int>(T); a.N = d; a.bn = bn;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
+    a.out[0] = Y; a.ld_out = d;
+    a.stream_out = 1;
+    TRY((launch_gemm<0, 0, 1, EPI_BF16, 1, 0, 1>(a, st, PH_DOWN)));
+  } else   {
     GemmArgs a = new_args(status);
     const int bn = d >= 256 ? 256 : round_up(d, 16);
     const int pair = (T > 128 && bn >= 32) ? 2 : 1;
@@ -718,9 +790,11 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
                  void* stream) {
   TRY(check_dims(D));
   if (!W || !A || !gr) return fail(LORA_ERR_INVALID_ARG, "weights/adapters/grads is NULL");
-  if (D->wfmt != LORA_WFMT_BF16) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights are not built into this entry point yet");
-  TRY(check_ptrs({dY, X, rms_w, ctx, dX, workspace, W->Wg, W->Wu, W->Wd, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd,
+  const bool q4 = D->wfmt == LORA_WFMT_4BIT;
+  TRY(check_ptrs({dY, X, rms_w, ctx, dX, workspace, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd,
                   gr->dAg, gr->dBg, gr->dAu, gr->dBu, gr->dAd, gr->dBd}));
+  if (q4) TRY(check_ptrs({W->Qg, W->Qu, W->Qd, W->absmax_g, W->absmax_u, W->absmax_d, W->codebook}));
+  else TRY(check_ptrs({W->Wg, W->Wu, W->Wd}));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long T = D->T;
   const int d = D->d, f = D->f, r = D->r, rp = rp_of(D);
@@ -755,7 +829,25 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY((launch_proj<1, 1>(a, T, d, rp, part, Qd, s, st, PH_Q_D)));
   }
   // S5b + S6: dAct = dY Wd + Qd Ad  ->  dG = dAct U silu'(G), dU = dAct silu(G)
-  {
+  if (q4) {
+    GemmArgs a = new_args(status);
+    const int bn = 256;
+    TRY(map_k(&a.maps[0], dY, T, d, d, 128));
+    TRY(map_q4_mn(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn));
+    TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
+    a.mn3d_b = 1;
+    TRY(map_mn3(&a.maps[3], A->Ad, r, f, f, bn / 64));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
+    a.seg[0].q4 = 1; a.seg[0].b_am[0] = 4;
+    set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    a.codebook = W->codebook;
+    a.M = static_cast<int>(T); a.N = f; a.bn = bn;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (f + bn - 1) / bn;
+    a.in[0] = G; a.in[1] = U; a.ld_in = f;
+    a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
+    a.stream_out = 1;
+    TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 1, 0, 1>(a, st, PH_DACT)));
+  } else   {
     GemmArgs a = new_args(status);
     const int bn = f >= 256 ? 256 : round_up(f, 64);
     const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
@@ -791,7 +883,29 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY((launch_proj<1, 2>(a, T, f, 2 * rp, part, Q, s, st, PH_Q_GU)));
   }
   // S8: dH = dG Wg + dU Wu + Q_g Ag + Q_u Au   (fp32)
-  {
+  if (q4) {
+    GemmArgs a = new_args(status);
+    const int bn = 256;
+    TRY(map_k(&a.maps[0], dG, T, f, f, 128));
+    TRY(map_q4_mn(&a.maps[1], &a.maps[7], W->Qg, W->absmax_g, f, d, bn));
+    TRY(map_k(&a.maps[2], dU, T, f, f, 128));
+    TRY(map_q4_mn(&a.maps[3], &a.maps[8], W->Qu, W->absmax_u, f, d, bn));
+    TRY(map_k(&a.maps[4], Q, T, 2 * rp, 2 * rp, 128));
+    a.mn3d_b = 1;
+    TRY(map_mn3(&a.maps[5], A->Ag, r, d, d, bn / 64));
+    TRY(map_mn3(&a.maps[6], A->Au, r, d, d, bn / 64));
+    set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
+    a.seg[0].q4 = 1; a.seg[0].b_am[0] = 7;
+    set_seg(a, 1, 2, 0, 3, 0, -1, 0, f);
+    a.seg[1].q4 = 1; a.seg[1].b_am[0] = 8;
+    set_seg(a, 2, 4, 0, 5, 0, -1, 0, rp);
+    set_seg(a, 3, 4, rp, 6, 0, -1, 0, rp);
+    a.codebook = W->codebook;
+    a.M = static_cast<int>(T); a.N = d; a.bn = bn;
+    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
+    a.out[0] = dH; a.ld_out = d;
+    TRY((launch_gemm<0, 1, 1, EPI_F32, 1, 0, 1>(a, st, PH_DH)));
+  } else   {
     GemmArgs a = new_args(status);
     const int bn = d >= 256 ? 256 : round_up(d, 64);
     const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;

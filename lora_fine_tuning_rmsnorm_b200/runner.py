@@ -12,6 +12,16 @@ ADAPTERS = ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")
 GRADS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
 
 
+def load_codebook() -> list:
+    """The 16-entry 4-bit codebook written by tests/golden/make_codebook.py."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "tests", "golden",
+                        "codebook16.json")
+    with open(path) as fh:
+        return [float.fromhex(h) for h in json.load(fh)["codebook_f32_hex"]]
+
+
 def bf16_tensor(bits: np.ndarray, device="cuda", pin=False) -> torch.Tensor:
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
     if device == "cpu":
@@ -40,13 +50,25 @@ class Problem:
         self.ctx = ops.alloc_ctx(self.dims, device)
         self.ws = ops.alloc_workspace(self.dims, device)
 
-    def use_4bit(self, codes: dict, absmax: dict, codebook: torch.Tensor):
-        """Switch the frozen weights to 4-bit codes (dict keys g, u, d)."""
+    def use_4bit(self, codebook, drop_bf16: bool = True):
+        """Quantise the frozen Wg, Wu, Wd to 4-bit blockwise codes on the GPU (one-off
+        set-up, lora_quantize_4bit) and switch the weights to them.  `codebook` is the
+        16-entry fp32 code table (an input of the method)."""
+        cb = torch.as_tensor(np.asarray(codebook, dtype=np.float32)).to(self.device)
+        codes, absmax = {}, {}
+        for k, name in (("g", "Wg"), ("u", "Wu"), ("d", "Wd")):
+            W = self.t[name]
+            codes[k] = torch.empty(W.numel() // 2, dtype=torch.uint8, device=self.device)
+            absmax[k] = torch.empty(W.numel() // 64, dtype=torch.float32, device=self.device)
+            ops.lora_quantize_4bit(W, cb, codes[k], absmax[k])
         self.dims.wfmt = ops.WFMT_4BIT
         self.dims.qblock = 64
-        self._q = (codes, absmax, codebook)
+        self.q4 = (codes, absmax, cb)
         self.weights = ops.make_weights(Qg=codes["g"], Qu=codes["u"], Qd=codes["d"], absmax_g=absmax["g"],
-                                        absmax_u=absmax["u"], absmax_d=absmax["d"], codebook=codebook)
+                                        absmax_u=absmax["u"], absmax_d=absmax["d"], codebook=cb)
+        if drop_bf16:  # the bf16 copies are no longer needed on the device
+            for name in ("Wg", "Wu", "Wd"):
+                self.t[name] = None
 
     def forward(self, X=None, stream=None):
         ops.lora_mlp_fwd(self.dims, self.t["X"] if X is None else X, self.t["w"], self.weights, self.adapters,

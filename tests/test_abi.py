@@ -80,12 +80,14 @@ def test_null_and_misaligned_pointers_rejected(L):
 
 
 def test_4bit_dims_rules(L):
-    dims = ops.make_dims(64, 128, 344, 8, wfmt=ops.WFMT_4BIT)
+    dims = ops.make_dims(64, 256, 344, 8, wfmt=ops.WFMT_4BIT)
     out = ctypes.c_size_t()
-    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3   # f % 64 != 0
-    dims = ops.make_dims(64, 128, 384, 8, wfmt=ops.WFMT_4BIT, qblock=32)
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3   # f % 256 != 0
+    dims = ops.make_dims(64, 128, 512, 8, wfmt=ops.WFMT_4BIT)
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3   # d % 256 != 0
+    dims = ops.make_dims(64, 256, 512, 8, wfmt=ops.WFMT_4BIT, qblock=32)
     assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3
-    dims = ops.make_dims(64, 128, 384, 8, wfmt=ops.WFMT_4BIT)
+    dims = ops.make_dims(64, 256, 512, 8, wfmt=ops.WFMT_4BIT)
     assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == 0
 
 

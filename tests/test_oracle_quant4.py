@@ -103,3 +103,12 @@ def test_pack_nibble_order_roundtrip():
     p = q4.pack(idx)
     assert p[0] == (0 | (1 << 4)) and p[7] == (14 | (15 << 4))
     np.testing.assert_array_equal(q4.unpack(p), idx)
+
+
+def test_golden_codebook_file_matches_oracle():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "codebook16.json")) as fh:
+        j = json.load(fh)
+    got = np.array([float.fromhex(h) for h in j["codebook_f32_hex"]], dtype=np.float64)
+    np.testing.assert_array_equal(got, q4.codebook16().astype(np.float64))
