@@ -42,7 +42,8 @@ def peaks():
 def shape_for(name, T=None):
     import dataclasses
     from lora_fine_tuning_rmsnorm_b200 import configs
-    s = {"8b": configs.LLAMA3_8B, "1b": configs.LLAMA32_1B, "tiny": configs.TINY}[name]
+    s = {"8b": configs.LLAMA3_8B, "8b-4bit": configs.LLAMA3_8B, "1b": configs.LLAMA32_1B,
+         "tiny": configs.TINY}[name]
     return dataclasses.replace(s, T=T) if T else s
 
 
@@ -157,13 +158,15 @@ def ours_arm(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from lora_fine_tuning_rmsnorm_b200 import configs, ops, synth
-    from lora_fine_tuning_rmsnorm_b200.runner import GRADS, Problem, bf16_tensor
+    from lora_fine_tuning_rmsnorm_b200.runner import GRADS, Problem, bf16_tensor, load_codebook
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     shape = shape_for(args.config, args.T)
     bits = synth.make_inputs_bits(shape)
     pb = Problem(shape, bits, device=dev)
+    if args.config == "8b-4bit":
+        pb.use_4bit(load_codebook())  # one-off quantisation of the frozen weights (set-up)
     # one flat fp32 buffer for the six adapter gradients -> one all-reduce per step
     sizes = {"dAg": (shape.r, shape.d), "dBg": (shape.f, shape.r), "dAu": (shape.r, shape.d),
              "dBu": (shape.f, shape.r), "dAd": (shape.r, shape.f), "dBd": (shape.d, shape.r)}
@@ -279,7 +282,8 @@ def ours_arm(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; bf16 weights/activations, fp32 accumulate)",
         "config": {"workload": f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape: T={T} (batch 4 x seq 2048) d={d} f={f} "
-                               f"r={r} alpha={shape.alpha:g}" if args.config == "8b" else
+                               f"r={r} alpha={shape.alpha:g}" + (", 4-bit frozen W (blocksize 64)" if args.config == "8b-4bit" else "")
+                   if args.config in ("8b", "8b-4bit") else
                                f"LoRA-MLP fwd+bwd {args.config}: T={T} d={d} f={f} r={r}",
                    "global_batch": T * world, "seq_len": 2048, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (weights 336 MB + activations), no flush"},
@@ -314,7 +318,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="8b", choices=["8b", "1b", "tiny"])
+    ap.add_argument("--config", default="8b", choices=["8b", "8b-4bit", "1b", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling on small cases)")

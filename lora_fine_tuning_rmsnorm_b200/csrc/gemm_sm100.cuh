@@ -35,7 +35,7 @@ constexpr int kMaxSegs = 4;
 constexpr int kMaxMaps = 10;
 constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16-column chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
-constexpr int kDqWarps = 4;  // 4-bit weights: warps that expand codes into bf16 B tiles
+constexpr int kDqWarps = 8;  // 4-bit weights: warps that expand codes into bf16 B tiles
 __host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps : 0); }
 
 enum Epi : int {
@@ -573,10 +573,11 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 // and absmax, expand each 64-element block row w = code[idx] * absmax (fp32 product,
 // rounded once to bf16) into the 128-byte-swizzled bf16 B tile, make the writes
 // visible to the tensor core (async proxy) and arrive on the stage's dq barrier.
-// tab[b] = (code[b & 15], code[b >> 4]): both nibbles of one packed byte.
+// The 16 code values are replicated per lane, tab[e * 32 + lane], so each lookup
+// reads bank `lane`: a warp's 32 lookups are one conflict-free shared-memory access.
 template <int B_MN, int NACC, int FUSE>
 __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, uint32_t full0, uint32_t dq0,
-                                             const float2* tab, const WaitCtl& wc) {
+                                             const float* tab, const WaitCtl& wc) {
   const int tid = threadIdx.x - kGemmThreads;  // 0 .. 32 * kDqWarps - 1
   const int lane = threadIdx.x % 32;
   const int total = p.tiles_m * p.tiles_n * p.splits;
@@ -627,13 +628,15 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
               const uint4 c0 = src[0], c1 = src[1];
               const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
               uint8_t* row = dst + static_cast<size_t>(i) * 128;
+              const float* tl = tab + lane;
 #pragma unroll
               for (int j = 0; j < 8; ++j) {  // 16-byte piece j = elements 8j .. 8j+7
                 uint32_t o[4];
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                  const float2 v = tab[(wv[j] >> (8 * b)) & 0xFF];
-                  o[b] = pack_bf16x2(v.x * scale, v.y * scale);
+                for (int b = 0; b < 4; ++b) {  // byte b: even element in the low nibble
+                  const float lo = tl[((wv[j] >> (8 * b)) & 0xF) * 32];
+                  const float hi = tl[((wv[j] >> (8 * b + 4)) & 0xF) * 32];
+                  o[b] = pack_bf16x2(lo * scale, hi * scale);
                 }
                 *reinterpret_cast<uint4*>(row + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
               }
@@ -668,9 +671,9 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   const uint32_t dq0 = drain_bar + 8;  // Q4: one barrier per stage (kDqWarps arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? S : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float2* tab = reinterpret_cast<float2*>(tmem_slot + 4);  // Q4: 256-entry nibble-pair table (8-byte aligned)
+  float* tab = reinterpret_cast<float*>(tmem_slot + 4);  // Q4: code values replicated per lane, [16][32]
   if (Q4)
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) tab[i] = make_float2(p.codebook[i & 15], p.codebook[i >> 4]);
+    for (int i = threadIdx.x; i < 16 * 32; i += blockDim.x) tab[i] = p.codebook[i / 32];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = PAIR == 1 ? 0u : cluster_ctarank();
 
