@@ -312,6 +312,40 @@ def ours_arm(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def sweep(args):
+    """Rank / length sweep at d = 4096, f = 14336 (alpha = 16): one JSON line per
+    point with tokens/s and the dense-GEMM vs memory-bound phase split."""
+    import torch
+    from lora_fine_tuning_rmsnorm_b200 import configs, ops, synth
+    from lora_fine_tuning_rmsnorm_b200.runner import Problem
+    torch.cuda.set_device(0)
+    gemm_names = ("gemm_gate_up_swiglu", "gemm_down", "gemm_dact_swiglu_bwd", "gemm_dH")
+    for s in configs.SWEEP:
+        bits = synth.make_inputs_bits(s)
+        pb = Problem(s, bits)
+        for _ in range(args.warmup):
+            pb.step()
+        torch.cuda.synchronize()
+        ops.timing_enable(True)
+        ops.timing_collect()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            pb.step()
+        e1.record()
+        torch.cuda.synchronize()
+        ph = ops.timing_collect()
+        ops.timing_enable(False)
+        ms = e0.elapsed_time(e1) / args.steps
+        gemm = sum(ph.get(k, (0.0, 0))[0] for k in gemm_names) / args.steps
+        other = sum(v[0] for k, v in ph.items() if k not in gemm_names) / args.steps
+        print(json.dumps({"sweep": True, "T": s.T, "r": s.r, "tokens_per_s": s.T / (ms / 1e3), "ms_per_step": ms,
+                          "tflops": configs.algorithmic_flops(s) / (ms / 1e3) / 1e12,
+                          "gemm_ms": gemm, "memory_bound_ms": other}), flush=True)
+        del pb
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -322,6 +356,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling on small cases)")
+    ap.add_argument("--sweep", action="store_true", help="rank/length sweep, one JSON line per point")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -329,6 +364,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         reference_arm(args, rank, world)
+        return
+    if args.sweep:
+        sweep(args)
         return
     if world > 1:
         import datetime

@@ -142,3 +142,45 @@ def fwd_bwd(inp: dict, s: float, eps: float, chunk: int = 2048, keep=("Y", "dX")
     out = {k: np.concatenate(v, axis=0) for k, v in rows.items()}
     out.update(grads)
     return out
+
+
+def sampled(inp: dict, s: float, eps: float, rows, cols, chunk: int = 4096):
+    """Selected outputs of the same forward/backward, computed without the full
+    [T x f] products, for long inputs:
+
+      Y[rows], dX[rows]                 (every step is row-local given the weights)
+      dBg[cols], dBu[cols], dAd[:, cols] (need only the columns `cols` of G, U, Act
+                                          and dAct, over all T rows)
+
+    Written from the same definitions as forward()/backward(), restricted to the
+    requested rows / columns.
+    """
+    X, dY = inp["X"], inp["dY"]
+    w, Wg, Wu, Wd = inp["w"], inp["Wg"], inp["Wu"], inp["Wd"]
+    Ag, Bg, Au, Bu, Ad, Bd = (inp[k] for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd"))
+    rows = np.asarray(rows)
+    cols = np.asarray(cols)
+    # row-local outputs
+    fw = forward(X[rows], w, eps, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s)
+    bw = backward(fw, dY[rows], X[rows], w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s)
+    out = {"Y": fw["Y"], "dX": bw["dX"]}
+    # column-restricted reductions over all rows
+    dBg = np.zeros((cols.size, Bg.shape[1]))
+    dBu = np.zeros((cols.size, Bu.shape[1]))
+    dAd = np.zeros((Ad.shape[0], cols.size))
+    for t0 in range(0, X.shape[0], chunk):
+        H, _ = rmsnorm_fwd(X[t0:t0 + chunk], w, eps)
+        dy = dY[t0:t0 + chunk]
+        Pg, Pu = H @ Ag.T, H @ Au.T
+        G = H @ Wg[cols].T + s * (Pg @ Bg[cols].T)
+        U = H @ Wu[cols].T + s * (Pu @ Bu[cols].T)
+        Act = silu(G) * U
+        Qd = dy @ Bd
+        dAct = dy @ Wd[:, cols] + s * (Qd @ Ad[:, cols])
+        dG = dAct * U * silu_grad(G)
+        dU = dAct * silu(G)
+        dBg += s * (dG.T @ Pg)
+        dBu += s * (dU.T @ Pu)
+        dAd += s * (Qd.T @ Act)
+    out.update(dBg=dBg, dBu=dBu, dAd=dAd)
+    return out

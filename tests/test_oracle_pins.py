@@ -256,3 +256,16 @@ def test_page_numbers_lora_shapes():
     fw = ref.forward(inp["X"], inp["w"], 1e-6, *(inp[k] for k in NAMES[1:]), s2.scale)
     frac = fw["Pg"].size / inp["X"].size
     assert round(100 * frac, 1) == xa["percent"]
+
+
+def test_sampled_outputs_equal_full_oracle():
+    s, inp = tiny_inputs(T=37, d=16, f=24, r=3, seed=41)
+    full = ref.fwd_bwd(inp, s.scale, 1e-6, chunk=1000, keep=("Y", "dX"))
+    rows = [0, 5, 36]
+    cols = [1, 7, 23]
+    smp = ref.sampled(inp, s.scale, 1e-6, rows, cols, chunk=10)
+    np.testing.assert_allclose(smp["Y"], full["Y"][rows], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(smp["dX"], full["dX"][rows], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(smp["dBg"], full["dBg"][cols], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(smp["dBu"], full["dBu"][cols], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(smp["dAd"], full["dAd"][:, cols], rtol=1e-12, atol=1e-15)
