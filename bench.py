@@ -158,7 +158,8 @@ def ours_arm(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from lora_fine_tuning_rmsnorm_b200 import configs, ops, synth
-    from lora_fine_tuning_rmsnorm_b200.runner import GRADS, Problem, bf16_tensor, load_codebook
+    from lora_fine_tuning_rmsnorm_b200 import dist as ldist
+    from lora_fine_tuning_rmsnorm_b200.runner import GRADS, HostPipeline, Problem, bf16_tensor, load_codebook
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -168,23 +169,15 @@ def ours_arm(args, rank, world, local_rank):
     if args.config == "8b-4bit":
         pb.use_4bit(load_codebook())  # one-off quantisation of the frozen weights (set-up)
     # one flat fp32 buffer for the six adapter gradients -> one all-reduce per step
-    sizes = {"dAg": (shape.r, shape.d), "dBg": (shape.f, shape.r), "dAu": (shape.r, shape.d),
-             "dBu": (shape.f, shape.r), "dAd": (shape.r, shape.f), "dBd": (shape.d, shape.r)}
-    total = sum(a * b for a, b in sizes.values())
-    flat = torch.zeros(total, dtype=torch.float32, device=dev)
-    off = 0
-    for k in GRADS:
-        n = sizes[k][0] * sizes[k][1]
-        pb.g[k] = flat[off:off + n].view(*sizes[k])
-        off += n
+    flat, views = ldist.flat_grads(shape.d, shape.f, shape.r, device=dev)
+    pb.g = views
     pb.grads = ops.make_grads(*(pb.g[k] for k in GRADS))
     stream = torch.cuda.current_stream(dev)
 
     def step():
         pb.forward(stream=stream)
         pb.backward(stream=stream)
-        if world > 1:
-            dist.all_reduce(flat)
+        ldist.allreduce_grads(flat)
 
     def barrier():
         if world > 1:
@@ -222,41 +215,30 @@ def ours_arm(args, rank, world, local_rank):
     tokens = world * shape.T * args.steps
     value = tokens / (ms / 1e3)
 
-    # ---- end-to-end through the C ABI with host buffers (pinned), copies inside the timed region
+    # ---- end-to-end through the C ABI with host buffers (pinned): every step copies its
+    # inputs in and its results (Y, dX, gradients) out inside the timed region; the copies
+    # are double-buffered on a second stream and overlap the neighbouring steps' compute
     hX = bf16_tensor(bits["X"], "cpu", pin=True)
     hdY = bf16_tensor(bits["dY"], "cpu", pin=True)
-    dX_in = torch.empty_like(pb.t["X"])
-    dY_in = torch.empty_like(pb.t["dY"])
-    hY = torch.empty(pb.Y.shape, dtype=torch.bfloat16, pin_memory=True)
-    hdX = torch.empty(pb.dX.shape, dtype=torch.bfloat16, pin_memory=True)
-    hflat = torch.empty(flat.shape, dtype=torch.float32, pin_memory=True)
-
-    def e2e_step():
-        dX_in.copy_(hX, non_blocking=True)
-        dY_in.copy_(hdY, non_blocking=True)
-        pb.forward(X=dX_in, stream=stream)
-        pb.backward(dY=dY_in, X=dX_in, stream=stream)
-        if world > 1:
-            dist.all_reduce(flat)
-        hY.copy_(pb.Y, non_blocking=True)
-        hdX.copy_(pb.dX, non_blocking=True)
-        hflat.copy_(flat, non_blocking=True)
-
-    e2e_step()
+    pipe = HostPipeline(pb, hX, hdY, reduce=ldist.allreduce_grads if world > 1 else None)
+    pipe.start()
+    for i in range(2):
+        pipe.step(i, 2)
     torch.cuda.synchronize(dev)
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    f1.record(stream)
+    f0.record(pipe.xs)
+    pipe.start()
+    for i in range(args.steps):
+        pipe.step(i, args.steps)
+    f1.record(pipe.xs)
     torch.cuda.synchronize(dev)
     barrier()
     ms_e2e = max_over_ranks(f0.elapsed_time(f1))
     e2e_value = world * shape.T * args.steps / (ms_e2e / 1e3)
     clocks = clk.stop() if clk else None
-    h2d = hX.numel() * 2 + hdY.numel() * 2
-    d2h = hY.numel() * 2 + hdX.numel() * 2 + hflat.numel() * 4
+    h2d = pipe.h2d_bytes
+    d2h = pipe.d2h_bytes
 
     if rank != 0:
         return

@@ -464,6 +464,30 @@ void set_seg(GemmArgs& a, int s, int amap, int ak0, int b0, int bk0, int b1, int
   a.nseg = std::max(a.nseg, s + 1);
 }
 
+// Tile shape of a dense GEMM (M = T rows, N columns): CTA pair (256-row tiles) or
+// single CTA, N tile 256 or 128 — the option that fills whole waves of the 148 SMs
+// best (ties within 2 % go to the larger tile, then to the pair).
+struct TileChoice { int pair, bn; };
+TileChoice pick_tiles(long long T, int N, bool mn_major) {
+  TileChoice best{T > 128 ? 2 : 1, N >= 256 ? 256 : (mn_major ? round_up(N, 64) : round_up(N, 16))};
+  if (N < 256 || T <= 128) return best;
+  double best_eff = -1.0;
+  const int bns[2] = {256, 128};
+  for (int pair = 2; pair >= 1; --pair) {
+    for (int bn : bns) {
+      const long long units = ((T + 128LL * pair - 1) / (128LL * pair)) * ((N + bn - 1) / bn);
+      const double per_wave = 148.0 / pair;
+      const double waves = units / per_wave;
+      const double eff = waves / std::ceil(waves);
+      if (eff > best_eff + 0.02) {
+        best_eff = eff;
+        best = TileChoice{pair, bn};
+      }
+    }
+  }
+  return best;
+}
+
 // Rank-r projection out[T x cols] (bf16) = scale * sum of K-split fp32 partials.
 // The GEMM args must already hold maps/segments/M/N/bn/tiles and NACC columns.
 template <int B_MN, int NACC>
@@ -765,10 +789,11 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.out[0] = Y; a.ld_out = d;
     a.stream_out = 1;
     TRY((launch_gemm<0, 0, 1, EPI_BF16, 1, 0, 1>(a, st, PH_DOWN)));
-  } else   {
+  } else {
     GemmArgs a = new_args(status);
-    const int bn = d >= 256 ? 256 : round_up(d, 16);
-    const int pair = (T > 128 && bn >= 32) ? 2 : 1;
+    const TileChoice tcx = pick_tiles(T, d, false);
+    const int bn = tcx.bn;
+    const int pair = (tcx.pair == 2 && bn >= 32) ? 2 : 1;
     TRY(map_k(&a.maps[0], Act, T, f, f, 128));
     TRY(map_k(&a.maps[1], W->Wd, d, f, f, bn / pair));
     TRY(map_k(&a.maps[2], Pd, T, rp, rp, 128));
@@ -847,10 +872,11 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
     a.stream_out = 1;
     TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 1, 0, 1>(a, st, PH_DACT)));
-  } else   {
+  } else {
     GemmArgs a = new_args(status);
-    const int bn = f >= 256 ? 256 : round_up(f, 64);
-    const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
+    const TileChoice tcx = pick_tiles(T, f, true);
+    const int bn = tcx.bn;
+    const int pair = (tcx.pair == 2 && bn % 128 == 0) ? 2 : 1;
     TRY(map_k(&a.maps[0], dY, T, d, d, 128));
     TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
     a.mn3d_b = f % 64 == 0;
@@ -905,10 +931,11 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
     TRY((launch_gemm<0, 1, 1, EPI_F32, 1, 0, 1>(a, st, PH_DH)));
-  } else   {
+  } else {
     GemmArgs a = new_args(status);
-    const int bn = d >= 256 ? 256 : round_up(d, 64);
-    const int pair = (T > 128 && bn % 128 == 0) ? 2 : 1;
+    const TileChoice tcx = pick_tiles(T, d, true);
+    const int bn = tcx.bn;
+    const int pair = (tcx.pair == 2 && bn % 128 == 0) ? 2 : 1;
     TRY(map_k(&a.maps[0], dG, T, f, f, 128));
     TRY(map_k(&a.maps[2], dU, T, f, f, 128));
     TRY(map_k(&a.maps[4], Q, T, 2 * rp, 2 * rp, 128));

@@ -84,3 +84,64 @@ class Problem:
 
     def saved(self) -> dict:
         return ops.ctx_views(self.dims, self.ctx)
+
+
+class HostPipeline:
+    """Training-step driver for inputs and results in pinned HOST memory.
+
+    Every step copies its X and dY host -> device, runs lora_mlp_fwd + lora_mlp_bwd,
+    and copies Y, dX and the packed adapter gradients device -> host.  The copies
+    run on a second stream and are double-buffered, so step i's results go back and
+    step i+2's inputs come in while step i+1 computes.  `reduce` (optional) is called
+    on the packed gradient buffer on the compute stream after each backward (the
+    data-parallel all-reduce).
+    """
+
+    def __init__(self, pb: "Problem", hX: torch.Tensor, hdY: torch.Tensor, reduce=None):
+        from . import dist as ldist
+        s = pb.shape
+        self.pb, self.hX, self.hdY, self.reduce = pb, hX, hdY, reduce
+        dev = pb.Y.device
+        self.cs = torch.cuda.current_stream(dev)
+        self.xs = torch.cuda.Stream(dev)
+        self.bufs = []
+        for _ in range(2):
+            flat, views = ldist.flat_grads(s.d, s.f, s.r, device=dev)
+            self.bufs.append(dict(X=torch.empty_like(hX, device=dev), dY=torch.empty_like(hdY, device=dev),
+                                  Y=torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev),
+                                  dX=torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev), flat=flat,
+                                  grads=ops.make_grads(*(views[k] for k in GRADS)),
+                                  ready=torch.cuda.Event(), done=torch.cuda.Event()))
+        self.hY = torch.empty(s.T, s.d, dtype=torch.bfloat16, pin_memory=True)
+        self.hdX = torch.empty(s.T, s.d, dtype=torch.bfloat16, pin_memory=True)
+        self.hflat = torch.empty(self.bufs[0]["flat"].numel(), dtype=torch.float32, pin_memory=True)
+        self.h2d_bytes = hX.numel() * hX.element_size() + hdY.numel() * hdY.element_size()
+        self.d2h_bytes = 2 * self.hY.numel() * 2 + self.hflat.numel() * 4
+
+    def _load(self, b):
+        with torch.cuda.stream(self.xs):
+            b["X"].copy_(self.hX, non_blocking=True)
+            b["dY"].copy_(self.hdY, non_blocking=True)
+            b["ready"].record(self.xs)
+
+    def start(self):
+        for b in self.bufs:
+            self._load(b)
+
+    def step(self, i: int, n_steps: int | None = None):
+        """Run step i; with n_steps given, inputs are not prefetched past the last step."""
+        pb, b = self.pb, self.bufs[i % 2]
+        self.cs.wait_event(b["ready"])
+        ops.lora_mlp_fwd(pb.dims, b["X"], pb.t["w"], pb.weights, pb.adapters, b["Y"], pb.ctx, pb.ws, self.cs)
+        ops.lora_mlp_bwd(pb.dims, b["dY"], b["X"], pb.t["w"], pb.weights, pb.adapters, pb.ctx, b["dX"],
+                         b["grads"], pb.ws, self.cs)
+        if self.reduce is not None:
+            self.reduce(b["flat"])
+        b["done"].record(self.cs)
+        self.xs.wait_event(b["done"])
+        with torch.cuda.stream(self.xs):
+            self.hY.copy_(b["Y"], non_blocking=True)
+            self.hdX.copy_(b["dX"], non_blocking=True)
+            self.hflat.copy_(b["flat"], non_blocking=True)
+        if n_steps is None or i + 2 < n_steps:
+            self._load(b)  # inputs of step i + 2 (after this step's compute has read them)

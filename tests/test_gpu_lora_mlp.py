@@ -106,3 +106,26 @@ def test_fwd_bwd_parity_llama3_8b(cuda_ok):
     pb = run_gpu(shape, bits, poison=False)
     R = oracle_all(shape, bits, keep=("Y", "dX"))
     compare(pb, R)
+
+
+def test_host_pipeline_matches_device_step(cuda_ok):
+    """Host-buffer driver (double-buffered copies on a second stream) returns the same
+    Y, dX and gradients as the device-resident step."""
+    from lora_fine_tuning_rmsnorm_b200 import dist as ldist
+    from lora_fine_tuning_rmsnorm_b200.runner import HostPipeline, bf16_tensor
+    shape = synth.Shape(T=384, d=256, f=512, r=16)
+    bits = synth.make_inputs_bits(shape)
+    pb = run_gpu(shape, bits, poison=False)
+    pipe = HostPipeline(pb, bf16_tensor(bits["X"], "cpu", pin=True), bf16_tensor(bits["dY"], "cpu", pin=True))
+    pipe.start()
+    for i in range(3):
+        pipe.step(i, 3)
+    torch.cuda.synchronize()
+    assert torch.equal(pipe.hY, pb.Y.cpu()) and torch.equal(pipe.hdX, pb.dX.cpu())
+    _, views = ldist.flat_grads(shape.d, shape.f, shape.r)
+    off = 0
+    for k in ldist.GRAD_ORDER:
+        n = views[k].numel()
+        got = pipe.hflat[off:off + n].view_as(views[k])
+        torch.testing.assert_close(got, pb.g[k].cpu(), rtol=1e-5, atol=1e-6 * float(pb.g[k].abs().max()))
+        off += n
