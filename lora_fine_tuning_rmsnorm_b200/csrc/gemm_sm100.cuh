@@ -73,7 +73,8 @@ struct GemmArgs {
   int M, N;  // valid rows / valid columns per accumulator
   int bn;    // N tile per accumulator (multiple of 16; multiple of 64 when B is MN-major)
   int tiles_m, tiles_n, splits;
-  int raster_n;    // 0: M-fastest tile order; 1: N-fastest
+  int raster;      // 0: M-fastest tile order; 1: N-fastest; 2: bands of group_m row tiles, N swept per band
+  int group_m;
   int mn3d_a, mn3d_b;  // 1: that MN-major operand's maps are 3-D {64, K, MN/64} views (one box per tile)
   int stream_out;  // 1: epilogue stores are streaming (evict-first in L2)
   int k_chunk;  // split-K chunk in elements (multiple of BK) when splits > 1
@@ -96,7 +97,18 @@ struct GemmArgs {
 
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
 __device__ __forceinline__ void decode_tile(const GemmArgs& p, int t, int& mt, int& nt, int& ks) {
-  if (p.raster_n) {
+  if (p.raster == 2) {
+    // a band of group_m row tiles stays in L2 while the wave sweeps the N tiles
+    const int per_split = p.tiles_m * p.tiles_n;
+    ks = t / per_split;
+    const int u = t - ks * per_split;
+    const int g = u / (p.group_m * p.tiles_n);
+    const int m_base = g * p.group_m;
+    const int gsz = min(p.group_m, p.tiles_m - m_base);
+    const int r = u - g * p.group_m * p.tiles_n;
+    mt = m_base + r % gsz;
+    nt = r / gsz;
+  } else if (p.raster == 1) {
     nt = t % p.tiles_n;
     t /= p.tiles_n;
     mt = t % p.tiles_m;

@@ -446,6 +446,19 @@ GemmArgs new_args(int* status) {
   return a;
 }
 
+// Banded tile order for a dense GEMM: `group_m` row tiles per band (the band's A
+// panels are re-read from L2 by every N tile).  LORA_MLP_RASTER=0 selects the plain
+// M-fastest order instead (tuning comparison).
+void set_band(GemmArgs& a, int group_m) {
+  static const int off = [] {
+    const char* e = getenv("LORA_MLP_RASTER");
+    return e && e[0] == '0' ? 1 : 0;
+  }();
+  if (off || group_m >= a.tiles_m) return;
+  a.raster = 2;
+  a.group_m = group_m;
+}
+
 void set_hints(GemmArgs& a, int a_hint, int b_hint) {
   for (int s = 0; s < a.nseg; ++s) {
     a.seg[s].a_hint = a_hint;
@@ -758,6 +771,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);  // H is re-read by every N tile: keep it in L2
+    set_band(a, 16);
     a.stream_out = 1;
     if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1>(a, st, PH_GATEUP)));
     else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1>(a, st, PH_GATEUP)));
@@ -804,6 +818,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
     a.stream_out = 1;
+    set_band(a, 8);
     if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_DOWN)));
     else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_DOWN)));
   }
@@ -893,6 +908,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
+    set_band(a, 16);
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
     else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
   }
@@ -958,6 +974,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
+    set_band(a, 4);
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_DH)));
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
   }
