@@ -38,6 +38,24 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kDqWarps = 8;  // 4-bit weights: warps that expand codes into bf16 B tiles
 __host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps : 0); }
 
+// Shared-memory layout of one 4-bit stage in one CTA (host and device use the same):
+// [A 16 KB][expanded bf16 B: slots x b_unit][codes: slots x q_unit][absmax: slots x m_unit].
+// A unit is one B operand (one accumulator, or one gate/up branch) as held by this CTA:
+// `cols` B rows (K-major) or B columns (MN-major) by 64 K, i.e. `cols` 128-byte smem rows.
+struct Q4Layout {
+  uint32_t b_unit, q_unit, m_unit;
+  int slots, cols;
+};
+__host__ __device__ inline Q4Layout q4_layout(int bn, int pair, int fuse, int b_mn, int nacc) {
+  Q4Layout L;
+  L.cols = fuse ? bn : bn / pair;
+  L.slots = fuse ? (pair == 1 ? 2 : 1) : nacc;
+  L.b_unit = static_cast<uint32_t>(L.cols) * 128u;
+  L.q_unit = static_cast<uint32_t>(L.cols) * 32u;
+  L.m_unit = b_mn ? 1024u : static_cast<uint32_t>(L.cols) * 16u;  // absmax box {4 floats} x rows
+  return L;
+}
+
 enum Epi : int {
   EPI_F32 = 0,         // out[0] fp32 = acc_a * alpha at column a * out_acc_col (+ split * split_stride)
   EPI_BF16 = 1,        // out[0] bf16 = acc_a * alpha, accumulator a at column a * out_acc_col
@@ -149,7 +167,8 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const Wai
 // issues one wide MMA instead of two; with PAIR = 2, CTA rank r loads branch r.
 template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
-                                              uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
+                                              uint32_t empty0, const WaitCtl& wc, uint32_t rank,
+                                              uint32_t cfull0) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const int bnl = p.bn / PAIR;  // B rows (N) held by this CTA
@@ -187,20 +206,22 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         } else {
           bb = nb0 < p.N ? b_bytes : 0u;
         }
+        if (!(Q4 && sg.q4)) {  // 4-bit B is staged on this CTA's own code barrier instead
 #pragma unroll
-        for (int a = 0; a < NACC; ++a)
-          if (sg.b_map[a] >= 0) by += bb;
+          for (int a = 0; a < NACC; ++a)
+            if (sg.b_map[a] >= 0) by += bb;
+        }
         return by;
       };
-      uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
+      const uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
+      // 4-bit: codes + absmax of the units this CTA expands, on its own code barrier
+      const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
+      uint32_t code_tx = 0;
       if (Q4 && sg.q4) {
-        // A tile + per branch: packed codes (bn x 32 B) and an absmax box (K-major:
-        // bn rows x 4 floats; MN-major: 64 K rows x 4 floats)
-        uint32_t by = a_bytes;
-#pragma unroll
-        for (int a = 0; a < (FUSE ? 2 : NACC); ++a)
-          if (sg.b_map[a] >= 0) by += p.bn * 32u + (B_MN ? 64u * 16u : p.bn * 16u);
-        stage_tx = by;
+        for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
+          if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
+          if (sg.b_map[u] >= 0) code_tx += QL.q_unit + QL.m_unit;
+        }
       }
       for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t full = full0 + 8 * stage, empty = empty0 + 8 * stage;
@@ -209,6 +230,10 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           break;
         }
         if (stage_tx) mbar_expect_tx(full, stage_tx);
+        if (Q4) {  // the code barrier completes every stage (no bytes for bf16 segments)
+          if (code_tx) mbar_expect_tx(cfull0 + 8 * stage, code_tx);
+          else mbar_arrive(cfull0 + 8 * stage);
+        }
         const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);
         const int m0 = mbase + static_cast<int>(rank) * BM;
         const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rank) * bnl;
@@ -241,22 +266,26 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         }
         hint = sg.b_hint;
         if (Q4 && sg.q4) {
-          // 4-bit B: stage the codes and block absmax; the dequant warps expand them
-          const int nbr = FUSE ? 2 : NACC;
-          const uint32_t sQ = sA + a_bytes + nbr * b_bytes;
-          const uint32_t sM = sQ + nbr * p.bn * 32;
+          // 4-bit B: stage the codes and block absmax of this CTA's units (own barrier);
+          // the dequant warps expand them into the B slots
+          const uint32_t sQ = sA + a_bytes + QL.slots * QL.b_unit;
+          const uint32_t sM = sQ + QL.slots * QL.q_unit;
+          const uint32_t cbar = cfull0 + 8 * stage;
 #pragma unroll
-          for (int r = 0; r < (FUSE ? 2 : NACC); ++r) {
-            if (sg.b_map[r] < 0) continue;
-            const CUtensorMap* qm = &p.maps[sg.b_map[r]];
-            const CUtensorMap* mm = &p.maps[sg.b_am[r]];
-            const int kk = sg.b_k0[r] + k;
+          for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
+            if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
+            if (sg.b_map[u] < 0) continue;
+            const int slot = (FUSE && PAIR == 2) ? 0 : u;
+            const int nq = FUSE ? n0 : nb0;  // first B row / column of this unit in this CTA
+            const CUtensorMap* qm = &p.maps[sg.b_map[u]];
+            const CUtensorMap* mm = &p.maps[sg.b_am[u]];
+            const int kk = sg.b_k0[u] + k;
             if (B_MN) {
-              load(sQ + r * p.bn * 32, qm, n0 / 2, kk);
-              load(sM + r * p.bn * 16, mm, (n0 / 64) & ~3, kk);
+              tma_load_2d(sQ + slot * QL.q_unit, qm, cbar, nq / 2, kk);
+              tma_load_2d(sM + slot * QL.m_unit, mm, cbar, (nq / 64) & ~3, kk);
             } else {
-              load(sQ + r * p.bn * 32, qm, kk / 2, n0);
-              load(sM + r * p.bn * 16, mm, (kk / 64) & ~3, n0);
+              tma_load_2d(sQ + slot * QL.q_unit, qm, cbar, kk / 2, nq);
+              tma_load_2d(sM + slot * QL.m_unit, mm, cbar, (kk / 64) & ~3, nq);
             }
           }
         } else if (FUSE) {
@@ -294,11 +323,14 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
       }
     }
   }
-  if (!ok && rank == 0) {
+  if (!ok) {
     // Aborting: make sure no TMA write into shared memory is still in flight (the
-    // even CTA's full barriers also count the odd CTA's bytes).
-    for (int s = 0; s < p.stages; ++s)
-      if (issued_mask & (1u << s)) drain_wait(full0 + 8 * s, (issued_par >> s) & 1, wc);
+    // even CTA's full barriers also count the odd CTA's bytes; code barriers are local).
+    for (int s = 0; s < p.stages; ++s) {
+      if (!(issued_mask & (1u << s))) continue;
+      if (rank == 0) drain_wait(full0 + 8 * s, (issued_par >> s) & 1, wc);
+      if (Q4) drain_wait(cfull0 + 8 * s, (issued_par >> s) & 1, wc);
+    }
   }
 }
 
@@ -335,9 +367,13 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
           ok = false;
           break;
         }
-        if (Q4 && !mbar_wait(dq0 + 8 * stage, phase, wc, kDevTimeoutMma)) {  // B tiles expanded
-          ok = false;
-          break;
+        if (Q4) {  // B tiles expanded (by both CTAs of a pair: cluster-scope acquire)
+          const bool got = PAIR == 1 ? mbar_wait(dq0 + 8 * stage, phase, wc, kDevTimeoutMma)
+                                     : mbar_wait_cluster(dq0 + 8 * stage, phase, wc, kDevTimeoutMma);
+          if (!got) {
+            ok = false;
+            break;
+          }
         }
         tc_fence_after();
         const int rem = sg.k_len - kb * BK;
@@ -581,25 +617,28 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   }
 }
 
-// 4-bit B producer (kDqWarps warps): for every stage, wait for the staged codes
-// and absmax, expand each 64-element block row w = code[idx] * absmax (fp32 product,
-// rounded once to bf16) into the 128-byte-swizzled bf16 B tile, make the writes
-// visible to the tensor core (async proxy) and arrive on the stage's dq barrier.
+// 4-bit B producer (kDqWarps warps per CTA): for every stage, wait for this CTA's
+// staged codes and absmax, expand each 64-element block row w = code[idx] * absmax
+// (fp32 product, rounded once to bf16) into the 128-byte-swizzled bf16 B tile, make the
+// writes visible to the tensor core (async proxy) and arrive on the MMA issuer's dq
+// barrier (the even CTA's, with a cluster-scope release, when CTAs are paired).  Each
+// warp waits and arrives on its own: a group barrier per stage (one wait, one arrive
+// per CTA) measured slower, since it keeps the warps from drifting across stages.
 // The 16 code values are replicated per lane, tab[e * 32 + lane], so each lookup
 // reads bank `lane`: a warp's 32 lookups are one conflict-free shared-memory access.
-template <int B_MN, int NACC, int FUSE>
-__device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, uint32_t full0, uint32_t dq0,
-                                             const float* tab, const WaitCtl& wc) {
+template <int B_MN, int NACC, int FUSE, int PAIR>
+__device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, uint32_t cfull0, uint32_t dq0,
+                                             const float* tab, const WaitCtl& wc, uint32_t rank) {
   const int tid = threadIdx.x - kGemmThreads;  // 0 .. 32 * kDqWarps - 1
   const int lane = threadIdx.x % 32;
   const int total = p.tiles_m * p.tiles_n * p.splits;
+  const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const uint32_t a_bytes = BM * BK * 2;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
-  const int nbr = FUSE ? 2 : NACC;
+  const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
   int stage = 0;
   uint32_t phase = 0;
   bool ok = true;
-  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+  for (int t = unit0; t < total && ok; t += nunits) {
     int mt, nt, ks;
     decode_tile(p, t, mt, nt, ks);
     const int n0 = nt * p.bn;
@@ -609,7 +648,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
       seg_kb_range(p, s, ks, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
         int w = 1;
-        if (lane == 0) w = mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutProducer) ? 1 : 0;
+        if (lane == 0) w = mbar_wait(cfull0 + 8 * stage, phase, wc, kDevTimeoutProducer) ? 1 : 0;
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) {
           ok = false;
@@ -617,47 +656,72 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
         }
         if (sg.q4) {
           uint8_t* base = tiles + static_cast<size_t>(stage) * p.stage_bytes;
-          const uint8_t* sQ = base + a_bytes + nbr * b_bytes;
-          const float* sM = reinterpret_cast<const float*>(sQ + nbr * p.bn * 32);
+          const uint8_t* sQ = base + a_bytes + QL.slots * QL.b_unit;
+          const float* sM = reinterpret_cast<const float*>(sQ + QL.slots * QL.q_unit);
           const int kk = kb * BK;
-          const int rows = p.bn;  // K-major: bn W rows; MN-major: 64 K rows x bn/64 chunks
-          for (int r = 0; r < nbr; ++r) {
-            if (sg.b_map[r] < 0) continue;
-            const uint8_t* q = sQ + r * p.bn * 32;
-            const float* am = sM + r * p.bn * 4;
-            uint8_t* dst = base + a_bytes + r * b_bytes;
-            for (int i = tid; i < rows; i += 32 * kDqWarps) {
-              const uint4* src;
-              float scale;
-              if (B_MN) {
-                const int c = i >> 6, krow = i & 63, chunks = p.bn >> 6;
-                src = reinterpret_cast<const uint4*>(q + krow * (chunks * 32) + c * 32);
-                scale = am[krow * 4 + ((n0 >> 6) & 3) + c];
-              } else {
-                src = reinterpret_cast<const uint4*>(q + i * 32);
-                scale = am[i * 4 + ((kk >> 6) & 3)];
-              }
-              const uint4 c0 = src[0], c1 = src[1];
-              const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-              uint8_t* row = dst + static_cast<size_t>(i) * 128;
-              const float* tl = tab + lane;
+          for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
+            if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
+            if (sg.b_map[u] < 0) continue;
+            const int slot = (FUSE && PAIR == 2) ? 0 : u;
+            const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (p.bn / PAIR);
+            const uint8_t* q = sQ + slot * QL.q_unit;
+            const float* am = sM + slot * (QL.m_unit / 4);
+            uint8_t* dst = base + a_bytes + slot * QL.b_unit;
+            const int chunks = QL.cols >> 6;
+            // Work item = one 16-byte piece (8 elements) of one 128-byte B row, so a
+            // warp covers 4 whole rows and every dequant warp has work.  Four items
+            // per thread per batch: all shared-memory loads before any store.
+            const int nitems = QL.cols * 8;
+            const float* tl = tab + lane;
+            for (int it0 = tid; it0 < nitems; it0 += 4 * 32 * kDqWarps) {
+              uint32_t cw[4];
+              float sc[4];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {  // 16-byte piece j = elements 8j .. 8j+7
+              for (int e = 0; e < 4; ++e) {
+                const int item = it0 + e * 32 * kDqWarps;
+                const int i = item >> 3, j = item & 7;
+                cw[e] = 0u;
+                sc[e] = 0.f;
+                if (item < nitems) {
+                  if (B_MN) {  // row i = (64-column chunk c, K row krow)
+                    const int c = i >> 6, krow = i & 63;
+                    cw[e] = *reinterpret_cast<const uint32_t*>(q + krow * (chunks * 32) + c * 32 + j * 4);
+                    sc[e] = am[krow * 4 + ((nq >> 6) & 3) + c];
+                  } else {     // row i = B row (N index), 64 K elements
+                    cw[e] = *reinterpret_cast<const uint32_t*>(q + i * 32 + j * 4);
+                    sc[e] = am[i * 4 + ((kk >> 6) & 3)];
+                  }
+                }
+              }
+              uint4 ov[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
                 uint32_t o[4];
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {  // byte b: even element in the low nibble
-                  const float lo = tl[((wv[j] >> (8 * b)) & 0xF) * 32];
-                  const float hi = tl[((wv[j] >> (8 * b + 4)) & 0xF) * 32];
-                  o[b] = pack_bf16x2(lo * scale, hi * scale);
+                  const float lo = tl[((cw[e] >> (8 * b)) & 0xF) * 32];
+                  const float hi = tl[((cw[e] >> (8 * b + 4)) & 0xF) * 32];
+                  o[b] = pack_bf16x2(lo * sc[e], hi * sc[e]);
                 }
-                *reinterpret_cast<uint4*>(row + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                ov[e] = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int item = it0 + e * 32 * kDqWarps;
+                if (item < nitems) {
+                  const int i = item >> 3, j = item & 7;
+                  *reinterpret_cast<uint4*>(dst + static_cast<size_t>(i) * 128 + ((j ^ (i & 7)) << 4)) = ov[e];
+                }
               }
             }
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(dq0 + 8 * stage);
+        if (lane == 0) {
+          if (PAIR == 1) mbar_arrive(dq0 + 8 * stage);
+          else mbar_arrive_cluster(mapa_shared(dq0 + 8 * stage, 0));
+        }
         if (++stage == p.stages) {
           stage = 0;
           phase ^= 1;
@@ -670,7 +734,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
 template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE, int Q4>
 __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
   static_assert(!FUSE || (NACC == 2 && !B_MN), "fused wide MMA: two K-major B halves");
-  static_assert(!Q4 || (PAIR == 1 && !A_MN), "4-bit B: single-CTA tiles, K-major A");
+  static_assert(!Q4 || !A_MN, "4-bit B: K-major A");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + static_cast<size_t>(p.stages) * p.stage_bytes);
@@ -680,8 +744,9 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   const uint32_t tfull0 = empty0 + 8 * S;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t drain_bar = tempty0 + 16;
-  const uint32_t dq0 = drain_bar + 8;  // Q4: one barrier per stage (kDqWarps arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? S : 0));
+  const uint32_t dq0 = drain_bar + 8;     // Q4: per stage, one arrival per dequant warp of each CTA
+  const uint32_t cfull0 = dq0 + 8 * S;    // Q4: per stage, this CTA's staged codes (TMA bytes)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? 2 * S : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tab = reinterpret_cast<float*>(tmem_slot + 4);  // Q4: code values replicated per lane, [16][32]
   if (Q4)
@@ -700,7 +765,10 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
     mbar_init(tempty0 + 8, kEpiWarps * PAIR);
     mbar_init(drain_bar, 1);
     if (Q4)
-      for (int s = 0; s < S; ++s) mbar_init(dq0 + 8 * s, kDqWarps);
+      for (int s = 0; s < S; ++s) {
+        mbar_init(dq0 + 8 * s, kDqWarps * PAIR);
+        mbar_init(cfull0 + 8 * s, 1);
+      }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -724,7 +792,7 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   const WaitCtl wc{abort_flag, p.status, p.limit_ns};
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, wc, rank);
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, wc, rank, cfull0);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
@@ -733,7 +801,7 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   } else if (warp < 2 + kEpiWarps) {
     gemm_epilogue<NACC, EPI, PAIR>(p, tfull0, tempty0, tmem_base, wc, rank);
   } else if (Q4) {
-    gemm_dequant<B_MN, NACC, FUSE>(p, tiles, full0, dq0, tab, wc);
+    gemm_dequant<B_MN, NACC, FUSE, PAIR>(p, tiles, cfull0, dq0, tab, wc, rank);
   }
   tc_fence_before();
   __syncthreads();

@@ -219,8 +219,10 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
     return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
   a.stage_bytes = BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
-  // 4-bit B: per branch also the staged codes (bn x 32 B) and absmax (>= 1 KB)
-  if (Q4) a.stage_bytes += NACC * (a.bn * 32 + std::max(a.bn * 16, 1024));
+  if (Q4) {  // 4-bit B: each expanded B slot also stages its codes and block absmax
+    const Q4Layout QL = q4_layout(a.bn, PAIR, FUSE, B_MN, NACC);
+    a.stage_bytes = BM * BK * 2 + QL.slots * (QL.b_unit + QL.q_unit + QL.m_unit);
+  }
   a.stage_bytes = (a.stage_bytes + 1023) & ~1023u;
   const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit nibble-pair table)
   const int avail = kSmemLimit - 1024 - extra;
@@ -739,8 +741,9 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
   // coming from TMA out-of-range fill (Bu is read from column -rp).
   if (q4) {
     // 4-bit frozen weights: the codes are expanded to bf16 B tiles in shared memory
-    // by dequant warps inside the GEMM (single-CTA tiles)
+    // by dequant warps inside the GEMM (each CTA of a pair expands its own branch)
     GemmArgs a = new_args(status);
+    const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
     TRY(map_q4_k(&a.maps[1], &a.maps[6], W->Qg, W->absmax_g, f, d, 128));
     TRY(map_q4_k(&a.maps[2], &a.maps[7], W->Qu, W->absmax_u, f, d, 128));
@@ -752,10 +755,13 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
     a.codebook = W->codebook;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (f + 127) / 128;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
+    set_hints(a, HINT_EVICT_LAST, HINT_NONE);
+    set_band(a, 16);
     a.stream_out = 1;
-    TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1, 1>(a, st, PH_GATEUP)));
+    if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1, 1>(a, st, PH_GATEUP)));
+    else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1, 1>(a, st, PH_GATEUP)));
   } else {
     GemmArgs a = new_args(status);
     const int pair = T > 128 ? 2 : 1;
@@ -789,20 +795,23 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
   // S4b: Y = Act Wd^T + Pd Bd^T
   if (q4) {
     GemmArgs a = new_args(status);
-    const int bn = d >= 256 ? 256 : round_up(d, 16);
+    const int bn = 256;  // d is a multiple of 256 for 4-bit weights
+    const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], Act, T, f, f, 128));
-    TRY(map_q4_k(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn));
+    TRY(map_q4_k(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn / pair));
     TRY(map_k(&a.maps[2], Pd, T, rp, rp, 128));
-    TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn));
+    TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn / pair));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 4;
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
     a.codebook = W->codebook;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
     a.stream_out = 1;
-    TRY((launch_gemm<0, 0, 1, EPI_BF16, 1, 0, 1>(a, st, PH_DOWN)));
+    set_band(a, 8);
+    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 1>(a, st, PH_DOWN)));
+    else TRY((launch_gemm<0, 0, 1, EPI_BF16, 1, 0, 1>(a, st, PH_DOWN)));
   } else {
     GemmArgs a = new_args(status);
     const TileChoice tcx = pick_tiles(T, d, false);
@@ -872,21 +881,24 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   if (q4) {
     GemmArgs a = new_args(status);
     const int bn = 256;
+    const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], dY, T, d, d, 128));
-    TRY(map_q4_mn(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn));
+    TRY(map_q4_mn(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn / pair));
     TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
     a.mn3d_b = 1;
-    TRY(map_mn3(&a.maps[3], A->Ad, r, f, f, bn / 64));
+    TRY(map_mn3(&a.maps[3], A->Ad, r, f, f, bn / pair / 64));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 4;
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
     a.codebook = W->codebook;
     a.M = static_cast<int>(T); a.N = f; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (f + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
     a.stream_out = 1;
-    TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 1, 0, 1>(a, st, PH_DACT)));
+    set_band(a, 16);
+    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2, 0, 1>(a, st, PH_DACT)));
+    else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 1, 0, 1>(a, st, PH_DACT)));
   } else {
     GemmArgs a = new_args(status);
     const TileChoice tcx = pick_tiles(T, f, true);
@@ -928,14 +940,15 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   if (q4) {
     GemmArgs a = new_args(status);
     const int bn = 256;
+    const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], dG, T, f, f, 128));
-    TRY(map_q4_mn(&a.maps[1], &a.maps[7], W->Qg, W->absmax_g, f, d, bn));
+    TRY(map_q4_mn(&a.maps[1], &a.maps[7], W->Qg, W->absmax_g, f, d, bn / pair));
     TRY(map_k(&a.maps[2], dU, T, f, f, 128));
-    TRY(map_q4_mn(&a.maps[3], &a.maps[8], W->Qu, W->absmax_u, f, d, bn));
+    TRY(map_q4_mn(&a.maps[3], &a.maps[8], W->Qu, W->absmax_u, f, d, bn / pair));
     TRY(map_k(&a.maps[4], Q, T, 2 * rp, 2 * rp, 128));
     a.mn3d_b = 1;
-    TRY(map_mn3(&a.maps[5], A->Ag, r, d, d, bn / 64));
-    TRY(map_mn3(&a.maps[6], A->Au, r, d, d, bn / 64));
+    TRY(map_mn3(&a.maps[5], A->Ag, r, d, d, bn / pair / 64));
+    TRY(map_mn3(&a.maps[6], A->Au, r, d, d, bn / pair / 64));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 7;
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, f);
@@ -944,9 +957,11 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     set_seg(a, 3, 4, rp, 6, 0, -1, 0, rp);
     a.codebook = W->codebook;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
-    TRY((launch_gemm<0, 1, 1, EPI_F32, 1, 0, 1>(a, st, PH_DH)));
+    set_band(a, 4);
+    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 1>(a, st, PH_DH)));
+    else TRY((launch_gemm<0, 1, 1, EPI_F32, 1, 0, 1>(a, st, PH_DH)));
   } else {
     GemmArgs a = new_args(status);
     const TileChoice tcx = pick_tiles(T, d, true);

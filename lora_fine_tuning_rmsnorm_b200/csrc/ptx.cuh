@@ -71,6 +71,34 @@ struct WaitCtl {
   uint64_t limit_ns;
 };
 
+// try_wait with cluster-scope acquire: orders what the arriving threads of the
+// other CTA wrote (and released at cluster scope) before the caller's later work.
+__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (see mbar_wait).
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_test_cluster(bar, parity, 200000u)) return true;
+    if (*c.abort_flag) return false;
+    if (global_ns() - t0 > c.limit_ns) {
+      if (c.status) atomicCAS(c.status, 0, code);
+      *c.abort_flag = 1;
+      __threadfence_block();
+      return false;
+    }
+  }
+}
+
 // Slow path of mbar_wait: sleep in suspend-hinted try_waits, checking the abort
 // flag and the time limit between them.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
