@@ -367,13 +367,9 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
           ok = false;
           break;
         }
-        if (Q4) {  // B tiles expanded (by both CTAs of a pair: cluster-scope acquire)
-          const bool got = PAIR == 1 ? mbar_wait(dq0 + 8 * stage, phase, wc, kDevTimeoutMma)
-                                     : mbar_wait_cluster(dq0 + 8 * stage, phase, wc, kDevTimeoutMma);
-          if (!got) {
-            ok = false;
-            break;
-          }
+        if (Q4 && !mbar_wait(dq0 + 8 * stage, phase, wc, kDevTimeoutMma)) {  // B tiles expanded (both CTAs)
+          ok = false;
+          break;
         }
         tc_fence_after();
         const int rem = sg.k_len - kb * BK;

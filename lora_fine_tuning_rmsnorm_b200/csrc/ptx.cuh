@@ -71,34 +71,6 @@ struct WaitCtl {
   uint64_t limit_ns;
 };
 
-// try_wait with cluster-scope acquire: orders what the arriving threads of the
-// other CTA wrote (and released at cluster scope) before the caller's later work.
-__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(ns)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait with cluster-scope acquire (see mbar_wait).
-__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
-  const uint64_t t0 = global_ns();
-  while (true) {
-    if (mbar_test_cluster(bar, parity, 200000u)) return true;
-    if (*c.abort_flag) return false;
-    if (global_ns() - t0 > c.limit_ns) {
-      if (c.status) atomicCAS(c.status, 0, code);
-      *c.abort_flag = 1;
-      __threadfence_block();
-      return false;
-    }
-  }
-}
-
 // Slow path of mbar_wait: sleep in suspend-hinted try_waits, checking the abort
 // flag and the time limit between them.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
@@ -206,9 +178,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
+// Arrive on a barrier of another CTA of the cluster (address from mapa_shared).  The
+// default (release, CTA-scope) form, as CUTLASS's cluster pipelines use: the writes it
+// publishes are the arriving thread's own shared-memory stores, complete before the
+// remote arrive leaves the SM.  The .release.cluster form adds a cluster-wide fence
+// that measured ~1500 cycles per arrive, which serialised the per-stage hand-off of
+// expanded 4-bit tiles.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
