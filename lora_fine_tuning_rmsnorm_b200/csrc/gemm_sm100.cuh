@@ -36,6 +36,7 @@ constexpr int kMaxMaps = 10;
 constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16-column chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kDqWarps = 8;  // 4-bit weights: warps that expand codes into bf16 B tiles
+constexpr int kDqGroups = 2;  // ... in groups that take alternate stages
 __host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps : 0); }
 
 // Shared-memory layout of one 4-bit stage in one CTA (host and device use the same):
@@ -613,25 +614,35 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   }
 }
 
-// 4-bit B producer (kDqWarps warps per CTA): for every stage, wait for this CTA's
-// staged codes and absmax, expand each 64-element block row w = code[idx] * absmax
-// (fp32 product, rounded once to bf16) into the 128-byte-swizzled bf16 B tile, make the
-// writes visible to the tensor core (async proxy) and arrive on the MMA issuer's dq
-// barrier (the even CTA's, with a cluster-scope release, when CTAs are paired).  Each
-// warp waits and arrives on its own: a group barrier per stage (one wait, one arrive
-// per CTA) measured slower, since it keeps the warps from drifting across stages.
-// The 16 code values are replicated per lane, tab[e * 32 + lane], so each lookup
-// reads bank `lane`: a warp's 32 lookups are one conflict-free shared-memory access.
+// 4-bit B producer (kDqWarps warps per CTA, in kDqGroups groups that take turns:
+// group g expands the stages with running index = g mod kDqGroups, so a thread has a
+// whole 64-element row of work per stage it takes and the wait / fence / arrive cost
+// is paid once per kDqGroups stages).  For each stage the group waits for this CTA's
+// staged codes and absmax, expands every 128-byte B row (one 64-element quantisation
+// block: one absmax) into the 128-byte-swizzled bf16 tile, makes the writes visible
+// to the tensor core (async proxy) and arrives on the MMA issuer's dq barrier (the
+// even CTA's when CTAs are paired).
+//
+// Expansion of one row: the 16 products bf16(fl32(code_e * absmax)) are formed once
+// (fp32 multiply, one rounding, as every element would get alone) and kept as byte
+// planes in registers, lo[0..3] / hi[0..3] = low / high bytes of entries 4q..4q+3.
+// A code word holds 8 elements' 4-bit indices in nibble order, which is already the
+// selector layout of prmt: the low 3 bits pick one of 8 entries from a plane pair,
+// bit 3 picks the pair (entries 0..7 or 8..15) through a byte mask.
 template <int B_MN, int NACC, int FUSE, int PAIR>
 __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, uint32_t cfull0, uint32_t dq0,
                                              const float* tab, const WaitCtl& wc, uint32_t rank) {
+  constexpr int kGroupWarps = kDqWarps / kDqGroups;
   const int tid = threadIdx.x - kGemmThreads;  // 0 .. 32 * kDqWarps - 1
   const int lane = threadIdx.x % 32;
+  const int group = (tid >> 5) / kGroupWarps;
+  const int gtid = tid % (32 * kGroupWarps);
   const int total = p.tiles_m * p.tiles_n * p.splits;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const uint32_t a_bytes = BM * BK * 2;
   const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
-  int stage = 0;
+  const float* code = tab + lane;  // code value e at code[32 * e] (lane-replicated: conflict-free)
+  int stage = 0, turn = 0;
   uint32_t phase = 0;
   bool ok = true;
   for (int t = unit0; t < total && ok; t += nunits) {
@@ -643,81 +654,77 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
       int kb0, kb1;
       seg_kb_range(p, s, ks, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
-        int w = 1;
-        if (lane == 0) w = mbar_wait(cfull0 + 8 * stage, phase, wc, kDevTimeoutProducer) ? 1 : 0;
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) {
-          ok = false;
-          break;
-        }
-        if (sg.q4) {
-          uint8_t* base = tiles + static_cast<size_t>(stage) * p.stage_bytes;
-          const uint8_t* sQ = base + a_bytes + QL.slots * QL.b_unit;
-          const float* sM = reinterpret_cast<const float*>(sQ + QL.slots * QL.q_unit);
-          const int kk = kb * BK;
-          for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
-            if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
-            if (sg.b_map[u] < 0) continue;
-            const int slot = (FUSE && PAIR == 2) ? 0 : u;
-            const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (p.bn / PAIR);
-            const uint8_t* q = sQ + slot * QL.q_unit;
-            const float* am = sM + slot * (QL.m_unit / 4);
-            uint8_t* dst = base + a_bytes + slot * QL.b_unit;
+        if (turn == group) {
+          int w = 1;
+          if (lane == 0) w = mbar_wait(cfull0 + 8 * stage, phase, wc, kDevTimeoutProducer) ? 1 : 0;
+          w = __shfl_sync(0xffffffffu, w, 0);
+          if (!w) {
+            ok = false;
+            break;
+          }
+          if (sg.q4) {
+            uint8_t* base = tiles + static_cast<size_t>(stage) * p.stage_bytes;
+            const uint8_t* sQ = base + a_bytes + QL.slots * QL.b_unit;
+            const float* sM = reinterpret_cast<const float*>(sQ + QL.slots * QL.q_unit);
+            const int kk = kb * BK;
             const int chunks = QL.cols >> 6;
-            // Work item = one 16-byte piece (8 elements) of one 128-byte B row, so a
-            // warp covers 4 whole rows and every dequant warp has work.  Four items
-            // per thread per batch: all shared-memory loads before any store.
-            const int nitems = QL.cols * 8;
-            const float* tl = tab + lane;
-            for (int it0 = tid; it0 < nitems; it0 += 4 * 32 * kDqWarps) {
-              uint32_t cw[4];
-              float sc[4];
+            for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
+              if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
+              if (sg.b_map[u] < 0) continue;
+              const int slot = (FUSE && PAIR == 2) ? 0 : u;
+              const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (p.bn / PAIR);
+              const uint8_t* q = sQ + slot * QL.q_unit;
+              const float* am = sM + slot * (QL.m_unit / 4);
+              uint8_t* dst = base + a_bytes + slot * QL.b_unit;
+              for (int i = gtid; i < QL.cols; i += 32 * kGroupWarps) {
+                const uint4* src;
+                float sc;
+                if (B_MN) {  // row i = (64-column chunk c, K row krow)
+                  const int c = i >> 6, krow = i & 63;
+                  src = reinterpret_cast<const uint4*>(q + krow * (chunks * 32) + c * 32);
+                  sc = am[krow * 4 + ((nq >> 6) & 3) + c];
+                } else {     // row i = B row (N index), 64 K elements
+                  src = reinterpret_cast<const uint4*>(q + i * 32);
+                  sc = am[i * 4 + ((kk >> 6) & 3)];
+                }
+                const uint4 c0 = src[0], c1 = src[1];
+                uint32_t lo[4], hi[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int item = it0 + e * 32 * kDqWarps;
-                const int i = item >> 3, j = item & 7;
-                cw[e] = 0u;
-                sc[e] = 0.f;
-                if (item < nitems) {
-                  if (B_MN) {  // row i = (64-column chunk c, K row krow)
-                    const int c = i >> 6, krow = i & 63;
-                    cw[e] = *reinterpret_cast<const uint32_t*>(q + krow * (chunks * 32) + c * 32 + j * 4);
-                    sc[e] = am[krow * 4 + ((nq >> 6) & 3) + c];
-                  } else {     // row i = B row (N index), 64 K elements
-                    cw[e] = *reinterpret_cast<const uint32_t*>(q + i * 32 + j * 4);
-                    sc[e] = am[i * 4 + ((kk >> 6) & 3)];
+                for (int g = 0; g < 4; ++g) {
+                  const uint32_t w0 = pack_bf16x2(code[32 * (4 * g)] * sc, code[32 * (4 * g + 1)] * sc);
+                  const uint32_t w1 = pack_bf16x2(code[32 * (4 * g + 2)] * sc, code[32 * (4 * g + 3)] * sc);
+                  lo[g] = prmt(w0, w1, 0x6420u);
+                  hi[g] = prmt(w0, w1, 0x7531u);
+                }
+                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint8_t* row = dst + static_cast<size_t>(i) * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {  // word j = elements 8j .. 8j+7 = 16-byte piece j
+                  const uint32_t m8 = (cw[j] >> 3) & 0x11111111u;  // bit 3 of every index
+                  uint32_t o[4];
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {  // elements 8j + 4h .. 8j + 4h + 3
+                    const uint32_t g16 = h ? (cw[j] >> 16) : cw[j];
+                    const uint32_t sel = g16 & 0x7777u;
+                    const uint32_t msk = prmt(0x0000FF00u, 0u, h ? (m8 >> 16) : m8);  // 0xFF where index >= 8
+                    const uint32_t lb = (prmt(lo[0], lo[1], sel) & ~msk) | (prmt(lo[2], lo[3], sel) & msk);
+                    const uint32_t hb = (prmt(hi[0], hi[1], sel) & ~msk) | (prmt(hi[2], hi[3], sel) & msk);
+                    o[2 * h] = prmt(lb, hb, 0x5140u);
+                    o[2 * h + 1] = prmt(lb, hb, 0x7362u);
                   }
-                }
-              }
-              uint4 ov[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                uint32_t o[4];
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {  // byte b: even element in the low nibble
-                  const float lo = tl[((cw[e] >> (8 * b)) & 0xF) * 32];
-                  const float hi = tl[((cw[e] >> (8 * b + 4)) & 0xF) * 32];
-                  o[b] = pack_bf16x2(lo * sc[e], hi * sc[e]);
-                }
-                ov[e] = make_uint4(o[0], o[1], o[2], o[3]);
-              }
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int item = it0 + e * 32 * kDqWarps;
-                if (item < nitems) {
-                  const int i = item >> 3, j = item & 7;
-                  *reinterpret_cast<uint4*>(dst + static_cast<size_t>(i) * 128 + ((j ^ (i & 7)) << 4)) = ov[e];
+                  *reinterpret_cast<uint4*>(row + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
               }
             }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            if (PAIR == 1) mbar_arrive(dq0 + 8 * stage);
+            else mbar_arrive_cluster(mapa_shared(dq0 + 8 * stage, 0));
+          }
         }
-        __syncwarp();
-        if (lane == 0) {
-          if (PAIR == 1) mbar_arrive(dq0 + 8 * stage);
-          else mbar_arrive_cluster(mapa_shared(dq0 + 8 * stage, 0));
-        }
+        if (++turn == kDqGroups) turn = 0;
         if (++stage == p.stages) {
           stage = 0;
           phase ^= 1;
@@ -740,7 +747,7 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   const uint32_t tfull0 = empty0 + 8 * S;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t drain_bar = tempty0 + 16;
-  const uint32_t dq0 = drain_bar + 8;     // Q4: per stage, one arrival per dequant warp of each CTA
+  const uint32_t dq0 = drain_bar + 8;     // Q4: per stage, one arrival per warp of the expanding group, per CTA
   const uint32_t cfull0 = dq0 + 8 * S;    // Q4: per stage, this CTA's staged codes (TMA bytes)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? 2 * S : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -762,7 +769,7 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
     mbar_init(drain_bar, 1);
     if (Q4)
       for (int s = 0; s < S; ++s) {
-        mbar_init(dq0 + 8 * s, kDqWarps * PAIR);
+        mbar_init(dq0 + 8 * s, (kDqWarps / kDqGroups) * PAIR);
         mbar_init(cfull0 + 8 * s, 1);
       }
     *abort_flag = 0;
