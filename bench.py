@@ -273,7 +273,8 @@ def ours_arm(args, rank, world, local_rank):
         "pct_bf16_peak": flops / (step_ms / 1e3) / 1e12 / bf16_sust,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tflops, "peak": bf16_sust,
                      "unit": "TFLOP/s", "frac": (dom_tflops / bf16_sust) if dom_tflops else None,
-                     "traffic": None, "peak_source": f"bf16_tflops_sustained ({src})",
+                     "traffic": measured_traffic(dom, args.config),
+                     "peak_source": f"bf16_tflops_sustained ({src})",
                      "flops_per_launch": dom_flops},
         "phase_rooflines": {
             "gemm_phases_frac_of_bf16_sustained": gemm_flops / (gemm_ms / 1e3) / 1e12 / bf16_sust if gemm_ms else None,
@@ -292,6 +293,37 @@ def ours_arm(args, rank, world, local_rank):
         line["cpu_baseline"] = {"value": n / t, "unit": UNIT, "cores": ot.cores, "kind": "oracle",
                                 "sample": f"{n} of {T} rows, fp64 NumPy oracle fwd+bwd over all weights ({t:.1f} s)"}
     print(json.dumps(line), flush=True)
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_lora_mlp_8b.md")
+KERNEL_SOURCES = ("gemm_sm100.cuh", "ptx.cuh", "lora_mlp.cu")
+
+
+def sources_digest() -> str:
+    """sha256 over the sources the GEMM kernels and their launches are built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "lora_fine_tuning_rmsnorm_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, config: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken
+    on the current kernel sources (a `traffic-record:` line); None otherwise."""
+    try:
+        lines = open(TRAFFIC_FILE).read().splitlines()
+    except OSError:
+        return None
+    digest = sources_digest()
+    for ln in lines:
+        if "traffic-record:" not in ln:
+            continue
+        kv = dict(x.split("=", 1) for x in ln.split("traffic-record:", 1)[1].split() if "=" in x)
+        if kv.get("kernel") == kernel and kv.get("config") == config and kv.get("sources") == digest:
+            return float(kv["bytes_per_launch"])
+    return None
 
 
 def sweep(args):
