@@ -37,10 +37,13 @@ constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kDqWarps = 8;  // 4-bit weights: warps that expand codes into bf16 B tiles
 constexpr int kDqGroups = 2;  // ... in groups that take alternate stages
-__host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps : 0); }
+constexpr int kCodeRing = 8;  // 4-bit weights: entries of the code ring (codes + absmax of one stage)
+// 4-bit CTAs add the dequant warps and one warp that fills the code ring
+__host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps + 32 : 0); }
 
-// Shared-memory layout of one 4-bit stage in one CTA (host and device use the same):
-// [A 16 KB][expanded bf16 B: slots x b_unit][codes: slots x q_unit][absmax: slots x m_unit].
+// Shared-memory layout of the 4-bit operand in one CTA (host and device use the same):
+// each stage is [A 16 KB][expanded bf16 B: slots x b_unit]; each of the kCodeRing code-ring
+// entries is [codes: slots x q_unit][absmax: slots x m_unit] (cr_bytes, 1 KB aligned).
 // A unit is one B operand (one accumulator, or one gate/up branch) as held by this CTA:
 // `cols` B rows (K-major) or B columns (MN-major) by 64 K, i.e. `cols` 128-byte smem rows.
 struct Q4Layout {
@@ -112,6 +115,7 @@ struct GemmArgs {
   int* status;
   unsigned long long limit_ns;
   const float* codebook;  // 4-bit code values (16 fp32)
+  uint32_t cr_bytes;      // 4-bit: bytes of one code-ring entry
 };
 
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
@@ -168,8 +172,7 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const Wai
 // issues one wide MMA instead of two; with PAIR = 2, CTA rank r loads branch r.
 template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
-                                              uint32_t empty0, const WaitCtl& wc, uint32_t rank,
-                                              uint32_t cfull0) {
+                                              uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
   const int total = p.tiles_m * p.tiles_n * p.splits;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const int bnl = p.bn / PAIR;  // B rows (N) held by this CTA
@@ -207,7 +210,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         } else {
           bb = nb0 < p.N ? b_bytes : 0u;
         }
-        if (!(Q4 && sg.q4)) {  // 4-bit B is staged on this CTA's own code barrier instead
+        if (!(Q4 && sg.q4)) {  // 4-bit B is written by the dequant warps instead
 #pragma unroll
           for (int a = 0; a < NACC; ++a)
             if (sg.b_map[a] >= 0) by += bb;
@@ -215,15 +218,6 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         return by;
       };
       const uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
-      // 4-bit: codes + absmax of the units this CTA expands, on its own code barrier
-      const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
-      uint32_t code_tx = 0;
-      if (Q4 && sg.q4) {
-        for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
-          if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
-          if (sg.b_map[u] >= 0) code_tx += QL.q_unit + QL.m_unit;
-        }
-      }
       for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t full = full0 + 8 * stage, empty = empty0 + 8 * stage;
         if (!mbar_wait(empty, phase ^ 1, wc, kDevTimeoutProducer)) {
@@ -231,10 +225,6 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           break;
         }
         if (stage_tx) mbar_expect_tx(full, stage_tx);
-        if (Q4) {  // the code barrier completes every stage (no bytes for bf16 segments)
-          if (code_tx) mbar_expect_tx(cfull0 + 8 * stage, code_tx);
-          else mbar_arrive(cfull0 + 8 * stage);
-        }
         const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);
         const int m0 = mbase + static_cast<int>(rank) * BM;
         const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rank) * bnl;
@@ -267,28 +257,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         }
         hint = sg.b_hint;
         if (Q4 && sg.q4) {
-          // 4-bit B: stage the codes and block absmax of this CTA's units (own barrier);
-          // the dequant warps expand them into the B slots
-          const uint32_t sQ = sA + a_bytes + QL.slots * QL.b_unit;
-          const uint32_t sM = sQ + QL.slots * QL.q_unit;
-          const uint32_t cbar = cfull0 + 8 * stage;
-#pragma unroll
-          for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
-            if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
-            if (sg.b_map[u] < 0) continue;
-            const int slot = (FUSE && PAIR == 2) ? 0 : u;
-            const int nq = FUSE ? n0 : nb0;  // first B row / column of this unit in this CTA
-            const CUtensorMap* qm = &p.maps[sg.b_map[u]];
-            const CUtensorMap* mm = &p.maps[sg.b_am[u]];
-            const int kk = sg.b_k0[u] + k;
-            if (B_MN) {
-              tma_load_2d(sQ + slot * QL.q_unit, qm, cbar, nq / 2, kk);
-              tma_load_2d(sM + slot * QL.m_unit, mm, cbar, (nq / 64) & ~3, kk);
-            } else {
-              tma_load_2d(sQ + slot * QL.q_unit, qm, cbar, kk / 2, nq);
-              tma_load_2d(sM + slot * QL.m_unit, mm, cbar, (kk / 64) & ~3, nq);
-            }
-          }
+          // 4-bit B: the dequant warps fill the B slots from the code ring
         } else if (FUSE) {
           // branch r fills B rows [r * bn, (r + 1) * bn) of the wide tile; a CTA of a
           // pair holds only its own branch
@@ -326,11 +295,10 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   }
   if (!ok) {
     // Aborting: make sure no TMA write into shared memory is still in flight (the
-    // even CTA's full barriers also count the odd CTA's bytes; code barriers are local).
+    // even CTA's full barriers also count the odd CTA's bytes).
     for (int s = 0; s < p.stages; ++s) {
       if (!(issued_mask & (1u << s))) continue;
       if (rank == 0) drain_wait(full0 + 8 * s, (issued_par >> s) & 1, wc);
-      if (Q4) drain_wait(cfull0 + 8 * s, (issued_par >> s) & 1, wc);
     }
   }
 }
@@ -345,10 +313,12 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
   const uint32_t idesc = idesc_bf16(BM * PAIR, FUSE ? 2 * p.bn : p.bn, A_MN, B_MN);
   const uint32_t a_bytes = BM * BK * 2;
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn / PAIR) * BK * 2;
+  const uint32_t tiles_u32 = smem_u32(tiles);
   int stage = 0;
   uint32_t phase = 0;
   uint32_t it = 0;
   bool ok = true, issued_any = false;
+  bool ready = false;  // the current stage's full barrier was seen complete by a peek
   for (int t = unit0; t < total && ok; t += nunits, ++it) {
     int mt, nt, ks;
     decode_tile(p, t, mt, nt, ks);
@@ -364,7 +334,7 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
       int kb0, kb1;
       seg_kb_range(p, s, ks, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutMma)) {
+        if (!ready && !mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutMma)) {
           ok = false;
           break;
         }
@@ -374,7 +344,15 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
         }
         tc_fence_after();
         const int rem = sg.k_len - kb * BK;
-        const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
+        const uint32_t sA = tiles_u32 + static_cast<uint32_t>(stage) * p.stage_bytes;
+        // Peek at the next stage of the ring (the next tile's first, at a tile's end)
+        // while the MMAs below issue: when its copies have landed no wait separates
+        // these MMAs from the next ones, and the tensor pipe does not drain between
+        // stages.
+        {
+          const int ns = stage + 1 == p.stages ? 0 : stage + 1;
+          ready = mbar_peek(full0 + 8 * ns, ns == 0 ? phase ^ 1u : phase);
+        }
         // descriptors of k-step 0; later k-steps only move the start address
         // (+32 B in a K-major 128-byte row, +2048 B = 16 rows for MN-major)
         const uint64_t ad0 = A_MN ? sdesc_sw128(sA, 8192, 1024) : sdesc_sw128(sA, 16, 1024);
@@ -614,11 +592,82 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   }
 }
 
+// 4-bit code-ring producer (one thread of the code warp): for every stage of a 4-bit
+// segment, copies this CTA's codes and block absmax into the next of kCodeRing ring
+// entries once the dequant group that read the entry before has released it.  The copies
+// thus run up to kCodeRing stages ahead of the expansion, outside the per-stage loop of
+// A copy -> expansion -> MMA -> free.
+template <int B_MN, int NACC, int PAIR, int FUSE>
+__device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* ring, uint32_t crfull0,
+                                                   uint32_t crempty0, const WaitCtl& wc, uint32_t rank) {
+  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
+  const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
+  int e = 0;
+  uint32_t phase = 0, issued_mask = 0, issued_par = 0;
+  bool ok = true;
+  for (int t = unit0; t < total && ok; t += nunits) {
+    int mt, nt, ks;
+    decode_tile(p, t, mt, nt, ks);
+    const int n0 = nt * p.bn;
+    for (int s = 0; s < p.nseg && ok; ++s) {
+      const Seg& sg = p.seg[s];
+      if (!sg.q4) continue;
+      int kb0, kb1;
+      seg_kb_range(p, s, ks, kb0, kb1);
+      uint32_t code_tx = 0;
+      for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
+        if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
+        if (sg.b_map[u] >= 0) code_tx += QL.q_unit + QL.m_unit;
+      }
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(crempty0 + 8 * e, phase ^ 1, wc, kDevTimeoutProducer)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bar = crfull0 + 8 * e;
+        if (code_tx) mbar_expect_tx(bar, code_tx);
+        else mbar_arrive(bar);
+        const uint32_t sQ = smem_u32(ring + static_cast<size_t>(e) * p.cr_bytes);
+        const uint32_t sM = sQ + QL.slots * QL.q_unit;
+#pragma unroll
+        for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
+          if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
+          if (sg.b_map[u] < 0) continue;
+          const int slot = (FUSE && PAIR == 2) ? 0 : u;
+          const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (p.bn / PAIR);  // first B row / column here
+          const CUtensorMap* qm = &p.maps[sg.b_map[u]];
+          const CUtensorMap* mm = &p.maps[sg.b_am[u]];
+          const int kk = sg.b_k0[u] + kb * BK;
+          if (B_MN) {
+            tma_load_2d(sQ + slot * QL.q_unit, qm, bar, nq / 2, kk);
+            tma_load_2d(sM + slot * QL.m_unit, mm, bar, (nq / 64) & ~3, kk);
+          } else {
+            tma_load_2d(sQ + slot * QL.q_unit, qm, bar, kk / 2, nq);
+            tma_load_2d(sM + slot * QL.m_unit, mm, bar, (kk / 64) & ~3, nq);
+          }
+        }
+        issued_mask |= 1u << e;
+        issued_par = (issued_par & ~(1u << e)) | (phase << e);
+        if (++e == kCodeRing) {
+          e = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  }
+  if (!ok) {  // aborting: no copy into the ring may still be in flight
+    for (int i = 0; i < kCodeRing; ++i)
+      if (issued_mask & (1u << i)) drain_wait(crfull0 + 8 * i, (issued_par >> i) & 1, wc);
+  }
+}
+
 // 4-bit B producer (kDqWarps warps per CTA, in kDqGroups groups that take turns:
 // group g expands the stages with running index = g mod kDqGroups, so a thread has a
 // whole 64-element row of work per stage it takes and the wait / fence / arrive cost
-// is paid once per kDqGroups stages).  For each stage the group waits for this CTA's
-// staged codes and absmax, expands every 128-byte B row (one 64-element quantisation
+// is paid once per kDqGroups stages).  For each stage the group waits until the MMA has
+// released the stage (its B slot is free) and for the stage's code-ring entry, expands
+// every 128-byte B row (one 64-element quantisation
 // block: one absmax) into the 128-byte-swizzled bf16 tile, makes the writes visible
 // to the tensor core (async proxy) and arrives on the MMA issuer's dq barrier (the
 // even CTA's when CTAs are paired).
@@ -630,8 +679,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 // selector layout of prmt: the low 3 bits pick one of 8 entries from a plane pair,
 // bit 3 picks the pair (entries 0..7 or 8..15) through a byte mask.
 template <int B_MN, int NACC, int FUSE, int PAIR>
-__device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, uint32_t cfull0, uint32_t dq0,
-                                             const float* tab, const WaitCtl& wc, uint32_t rank) {
+__device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, const uint8_t* ring,
+                                             uint32_t empty0, uint32_t crfull0, uint32_t crempty0,
+                                             uint32_t dq0, const float* tab, const WaitCtl& wc, uint32_t rank) {
   constexpr int kGroupWarps = kDqWarps / kDqGroups;
   const int tid = threadIdx.x - kGemmThreads;  // 0 .. 32 * kDqWarps - 1
   const int lane = threadIdx.x % 32;
@@ -642,8 +692,8 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
   const uint32_t a_bytes = BM * BK * 2;
   const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
   const float* code = tab + lane;  // code value e at code[32 * e] (lane-replicated: conflict-free)
-  int stage = 0, turn = 0;
-  uint32_t phase = 0;
+  int stage = 0, turn = 0, e = 0;
+  uint32_t phase = 0, cphase = 0;
   bool ok = true;
   for (int t = unit0; t < total && ok; t += nunits) {
     int mt, nt, ks;
@@ -655,8 +705,12 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
       seg_kb_range(p, s, ks, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (turn == group) {
+          // the stage's previous contents consumed by the MMA (B slot free), codes landed
           int w = 1;
-          if (lane == 0) w = mbar_wait(cfull0 + 8 * stage, phase, wc, kDevTimeoutProducer) ? 1 : 0;
+          if (lane == 0) {
+            w = mbar_wait(empty0 + 8 * stage, phase ^ 1, wc, kDevTimeoutProducer) ? 1 : 0;
+            if (w && sg.q4) w = mbar_wait(crfull0 + 8 * e, cphase, wc, kDevTimeoutProducer) ? 1 : 0;
+          }
           w = __shfl_sync(0xffffffffu, w, 0);
           if (!w) {
             ok = false;
@@ -664,7 +718,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
           }
           if (sg.q4) {
             uint8_t* base = tiles + static_cast<size_t>(stage) * p.stage_bytes;
-            const uint8_t* sQ = base + a_bytes + QL.slots * QL.b_unit;
+            const uint8_t* sQ = ring + static_cast<size_t>(e) * p.cr_bytes;
             const float* sM = reinterpret_cast<const float*>(sQ + QL.slots * QL.q_unit);
             const int kk = kb * BK;
             const int chunks = QL.cols >> 6;
@@ -720,9 +774,14 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
           }
           __syncwarp();
           if (lane == 0) {
+            if (sg.q4) mbar_arrive(crempty0 + 8 * e);  // ring entry read: free for the next copy
             if (PAIR == 1) mbar_arrive(dq0 + 8 * stage);
             else mbar_arrive_cluster(mapa_shared(dq0 + 8 * stage, 0));
           }
+        }
+        if (sg.q4 && ++e == kCodeRing) {
+          e = 0;
+          cphase ^= 1;
         }
         if (++turn == kDqGroups) turn = 0;
         if (++stage == p.stages) {
@@ -740,16 +799,18 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   static_assert(!Q4 || !A_MN, "4-bit B: K-major A");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + static_cast<size_t>(p.stages) * p.stage_bytes);
+  uint8_t* ring = tiles + static_cast<size_t>(p.stages) * p.stage_bytes;  // Q4: code ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (Q4 ? static_cast<size_t>(kCodeRing) * p.cr_bytes : 0));
   const int S = p.stages;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * S;
   const uint32_t tfull0 = empty0 + 8 * S;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t drain_bar = tempty0 + 16;
-  const uint32_t dq0 = drain_bar + 8;     // Q4: per stage, one arrival per warp of the expanding group, per CTA
-  const uint32_t cfull0 = dq0 + 8 * S;    // Q4: per stage, this CTA's staged codes (TMA bytes)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? 2 * S : 0));
+  const uint32_t dq0 = drain_bar + 8;             // Q4: per stage, one arrival per warp of the expanding group, per CTA
+  const uint32_t crfull0 = dq0 + 8 * S;           // Q4: per ring entry, the code copy (TMA bytes)
+  const uint32_t crempty0 = crfull0 + 8 * kCodeRing;  // Q4: per ring entry, released by the expanding group
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? S + 2 * kCodeRing : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tab = reinterpret_cast<float*>(tmem_slot + 4);  // Q4: code values replicated per lane, [16][32]
   if (Q4)
@@ -767,11 +828,13 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
     mbar_init(tempty0, kEpiWarps * PAIR);
     mbar_init(tempty0 + 8, kEpiWarps * PAIR);
     mbar_init(drain_bar, 1);
-    if (Q4)
-      for (int s = 0; s < S; ++s) {
-        mbar_init(dq0 + 8 * s, (kDqWarps / kDqGroups) * PAIR);
-        mbar_init(cfull0 + 8 * s, 1);
+    if (Q4) {
+      for (int s = 0; s < S; ++s) mbar_init(dq0 + 8 * s, (kDqWarps / kDqGroups) * PAIR);
+      for (int i = 0; i < kCodeRing; ++i) {
+        mbar_init(crfull0 + 8 * i, 1);
+        mbar_init(crempty0 + 8 * i, kDqWarps / kDqGroups);
       }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -795,7 +858,7 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
   const WaitCtl wc{abort_flag, p.status, p.limit_ns};
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, wc, rank, cfull0);
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, wc, rank);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
@@ -803,8 +866,11 @@ __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp < 2 + kEpiWarps) {
     gemm_epilogue<NACC, EPI, PAIR>(p, tfull0, tempty0, tmem_base, wc, rank);
+  } else if (Q4 && warp < 2 + kEpiWarps + kDqWarps) {
+    gemm_dequant<B_MN, NACC, FUSE, PAIR>(p, tiles, ring, empty0, crfull0, crempty0, dq0, tab, wc, rank);
   } else if (Q4) {
-    gemm_dequant<B_MN, NACC, FUSE, PAIR>(p, tiles, cfull0, dq0, tab, wc, rank);
+    if (lane == 0) gemm_code_producer<B_MN, NACC, PAIR, FUSE>(p, ring, crfull0, crempty0, wc, rank);
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -219,13 +219,16 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
     return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
   a.stage_bytes = BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
-  if (Q4) {  // 4-bit B: each expanded B slot also stages its codes and block absmax
+  a.cr_bytes = 0;
+  if (Q4) {  // 4-bit B: expanded B slots per stage; codes + absmax in a ring of their own
     const Q4Layout QL = q4_layout(a.bn, PAIR, FUSE, B_MN, NACC);
-    a.stage_bytes = BM * BK * 2 + QL.slots * (QL.b_unit + QL.q_unit + QL.m_unit);
+    a.stage_bytes = BM * BK * 2 + QL.slots * QL.b_unit;
+    a.cr_bytes = (QL.slots * (QL.q_unit + QL.m_unit) + 1023) & ~1023u;
   }
   a.stage_bytes = (a.stage_bytes + 1023) & ~1023u;
-  const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit nibble-pair table)
-  const int avail = kSmemLimit - 1024 - extra;
+  const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit code table)
+  const int ring = Q4 ? kCodeRing * static_cast<int>(a.cr_bytes) : 0;
+  const int avail = kSmemLimit - 1024 - extra - ring;
   a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
   static const int stage_cap = [] {
     const char* e = getenv("LORA_MLP_MAX_STAGES");  // tuning knob: cap the TMA ring depth
@@ -238,7 +241,7 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
   if (tc > 512) return fail(LORA_ERR_UNSUPPORTED, "internal: TMEM columns %d > 512", cols);
   a.tmem_cols = tc;
-  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + extra;
+  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + ring + extra;
   // more than half of TMEM per CTA: keep one CTA per SM so allocation never waits
   if (tc > 256) smem = std::max(smem, kSmemLimit / 2 + 4096);
   a.limit_ns = wait_limit_ns();

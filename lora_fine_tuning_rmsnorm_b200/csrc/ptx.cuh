@@ -50,6 +50,18 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking look at a phase (test_wait never suspends the thread).
+__device__ __forceinline__ bool mbar_peek(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // try_wait with a suspend-time hint: the thread sleeps (no issue slots) until the
 // phase completes or about `ns` nanoseconds pass, instead of spinning.
 __device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
