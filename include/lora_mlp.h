@@ -79,9 +79,10 @@ typedef struct lora_mlp_dims {
  *                                           the row-major matrix in the low nibble
  *   absmax_g, absmax_u [f*d/64], absmax_d [d*f/64]  fp32 per-block absmax
  *   codebook [16] fp32                      code values (wfmt = LORA_WFMT_4BIT)
- * With 4-bit weights the GEMMs stage the codes and absmax in shared memory and
- * expand them to bf16 tiles in-kernel (w = bf16(codebook[idx] * absmax)) right
- * before the tensor-core MMA; no bf16 copy of W is ever written to memory.
+ * With 4-bit weights the GEMMs copy the codes and absmax into shared memory and
+ * expand them to bf16 tiles in-kernel (w = bf16(codebook[idx] * absmax), fp32
+ * product rounded once) right before the tensor-core MMA; no bf16 copy of W is
+ * ever written to memory.
  * Unused members may be NULL. */
 typedef struct lora_mlp_weights {
   const void* Wg;

@@ -49,7 +49,7 @@ def run(shape, keep=("Y", "dX")):
 @pytest.mark.parametrize("shape", [
     synth.Shape(T=200, d=256, f=512, r=16, alpha=16.0),
     synth.Shape(T=300, d=512, f=768, r=32, alpha=16.0),
-    synth.Shape(T=64, d=256, f=256, r=8, alpha=16.0),     # one M tile: single-CTA tiles
+    synth.Shape(T=64, d=256, f=256, r=8, alpha=16.0),     # T <= 128: single-CTA tiles (no pairs)
     synth.Shape(T=2200, d=256, f=512, r=16, alpha=16.0),  # CTA pairs, banded tile order, ragged T
 ], ids=lambda s: f"T{s.T}_d{s.d}_f{s.f}_r{s.r}")
 def test_fwd_bwd_parity_4bit_small(cuda_ok, shape):
