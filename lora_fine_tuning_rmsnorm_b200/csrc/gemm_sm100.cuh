@@ -314,6 +314,10 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
   const uint32_t a_bytes = BM * BK * 2;
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn / PAIR) * BK * 2;
   const uint32_t tiles_u32 = smem_u32(tiles);
+  // launch constants in registers: the asm statements below clobber memory, which would
+  // otherwise make the compiler re-read them from the parameter space in the issue loop
+  const int nstages = p.stages, nseg = p.nseg, bn = p.bn;
+  const uint32_t stage_bytes = p.stage_bytes;
   int stage = 0;
   uint32_t phase = 0;
   uint32_t it = 0;
@@ -329,10 +333,15 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
     }
     tc_fence_after();
     uint32_t started = 0;
-    for (int s = 0; s < p.nseg && ok; ++s) {
+    for (int s = 0; s < nseg && ok; ++s) {
       const Seg& sg = p.seg[s];
       int kb0, kb1;
       seg_kb_range(p, s, ks, kb0, kb1);
+      const int k_len = sg.k_len;
+      uint32_t bmask = 0;  // accumulators this segment feeds
+#pragma unroll
+      for (int a = 0; a < NACC; ++a)
+        if (sg.b_map[a] >= 0) bmask |= 1u << a;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!ready && !mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutMma)) {
           ok = false;
@@ -343,14 +352,14 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
           break;
         }
         tc_fence_after();
-        const int rem = sg.k_len - kb * BK;
-        const uint32_t sA = tiles_u32 + static_cast<uint32_t>(stage) * p.stage_bytes;
+        const int rem = k_len - kb * BK;
+        const uint32_t sA = tiles_u32 + static_cast<uint32_t>(stage) * stage_bytes;
         // Peek at the next stage of the ring (the next tile's first, at a tile's end)
         // while the MMAs below issue: when its copies have landed no wait separates
         // these MMAs from the next ones, and the tensor pipe does not drain between
         // stages.
         {
-          const int ns = stage + 1 == p.stages ? 0 : stage + 1;
+          const int ns = stage + 1 == nstages ? 0 : stage + 1;
           ready = mbar_peek(full0 + 8 * ns, ns == 0 ? phase ^ 1u : phase);
         }
         // descriptors of k-step 0; later k-steps only move the start address
@@ -360,10 +369,10 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
         constexpr uint32_t b_step = B_MN ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
         for (int a = 0; a < (FUSE ? 1 : NACC); ++a) {
-          if (sg.b_map[a] < 0) continue;
+          if (!((bmask >> a) & 1u)) continue;
           const uint32_t sB = sA + a_bytes + a * b_bytes;
           const uint64_t bd0 = B_MN ? sdesc_sw128(sB, 8192, 1024) : sdesc_sw128(sB, 16, 1024);
-          const uint32_t d = tmem_base + buf * (NACC * p.bn) + a * p.bn;
+          const uint32_t d = tmem_base + buf * (NACC * bn) + a * bn;
           const uint32_t acc0 = (started >> a) & 1;
           if (rem >= BK) {
 #pragma unroll
@@ -384,7 +393,7 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
         // frees the smem stage (in both CTAs of a pair) once these MMAs finish
         if (PAIR == 1) mma_commit(empty0 + 8 * stage);
         else mma_commit_pair(empty0 + 8 * stage, 0x3);
-        if (++stage == p.stages) {
+        if (++stage == nstages) {
           stage = 0;
           phase ^= 1;
         }
