@@ -83,6 +83,18 @@ class OracleTimer:
         return max(16, min(n, len(self.inp["X"])))
 
 
+def config_for(args, shape, world):
+    """The workload description both arms print (same sizes, same wording)."""
+    T, d, f, r = shape.T, shape.d, shape.f, shape.r
+    if args.config in ("8b", "8b-4bit"):
+        wl = (f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape: T={T} (batch 4 x seq 2048) d={d} f={f} "
+              f"r={r} alpha={shape.alpha:g}" + (", 4-bit frozen W (blocksize 64)" if args.config == "8b-4bit" else ""))
+    else:
+        wl = f"LoRA-MLP fwd+bwd {args.config}: T={T} d={d} f={f} r={r}"
+    return {"workload": wl, "global_batch": T * world, "seq_len": 2048, "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2 (weights 336 MB + activations), no flush"}
+
+
 def reference_arm(args, rank, world):
     if rank != 0:
         return
@@ -102,8 +114,7 @@ def reference_arm(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_med,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, bf16-rounded)",
-        "config": {"workload": f"LoRA-MLP {args.config} T={shape.T} d={shape.d} f={shape.f} r={shape.r}",
-                   "global_batch": shape.T, "seq_len": 2048, "parallelism": "cpu"},
+        "config": config_for(args, shape, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": ot.cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -263,12 +274,7 @@ def ours_arm(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; bf16 weights/activations, fp32 accumulate)",
-        "config": {"workload": f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape: T={T} (batch 4 x seq 2048) d={d} f={f} "
-                               f"r={r} alpha={shape.alpha:g}" + (", 4-bit frozen W (blocksize 64)" if args.config == "8b-4bit" else "")
-                   if args.config in ("8b", "8b-4bit") else
-                               f"LoRA-MLP fwd+bwd {args.config}: T={T} d={d} f={f} r={r}",
-                   "global_batch": T * world, "seq_len": 2048, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (weights 336 MB + activations), no flush"},
+        "config": config_for(args, shape, world),
         "tflops": flops / (step_ms / 1e3) / 1e12,
         "pct_bf16_peak": flops / (step_ms / 1e3) / 1e12 / bf16_sust,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tflops, "peak": bf16_sust,
