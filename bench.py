@@ -306,12 +306,17 @@ KERNEL_SOURCES = ("gemm_sm100.cuh", "ptx.cuh", "lora_mlp.cu")
 
 
 def sources_digest() -> str:
-    """sha256 over the sources the GEMM kernels and their launches are built from."""
+    """sha256 over the code (comments and blank space removed) of the sources the GEMM
+    kernels and their launches are built from."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "lora_fine_tuning_rmsnorm_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "lora_fine_tuning_rmsnorm_b200", "csrc", name)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

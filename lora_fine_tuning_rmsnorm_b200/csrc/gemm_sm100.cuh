@@ -22,7 +22,9 @@
 // TMEM and issues tcgen05.mma from one thread, warps 2..9 drain the double-
 // buffered TMEM accumulators (tcgen05.ld) through the epilogue while the next
 // tile's main loop runs (two warps per TMEM lane quarter, alternating 16-column
-// chunks).  Tile order is M-fastest over a persistent grid.
+// chunks).  With 4-bit weights (Q4 = 1) warps 10..17 expand the codes into the bf16
+// B tiles and warp 18 fills the code ring.  Tiles are handed out over a persistent
+// grid, M-fastest or in bands of group_m row tiles with N swept per band.
 #pragma once
 #include "ptx.cuh"
 
