@@ -489,16 +489,18 @@ struct TileChoice { int pair, bn; };
 TileChoice pick_tiles(long long T, int N, bool mn_major) {
   TileChoice best{T > 128 ? 2 : 1, N >= 256 ? 256 : (mn_major ? round_up(N, 64) : round_up(N, 16))};
   if (N < 256 || T <= 128) return best;
-  double best_eff = -1.0;
+  // Cost = whole waves x time of one tile.  A tile of N = 128 takes about 0.8 of an
+  // N = 256 tile's time (measured: the per-k-block issue and barrier work of the MMA
+  // thread does not shrink with N), so N = 128 only pays where it saves many waves.
+  double best_cost = 1e30;
   const int bns[2] = {256, 128};
   for (int pair = 2; pair >= 1; --pair) {
     for (int bn : bns) {
       const long long units = ((T + 128LL * pair - 1) / (128LL * pair)) * ((N + bn - 1) / bn);
-      const double per_wave = 148.0 / pair;
-      const double waves = units / per_wave;
-      const double eff = waves / std::ceil(waves);
-      if (eff > best_eff + 0.02) {
-        best_eff = eff;
+      const double waves = std::ceil(units / (148.0 / pair));
+      const double cost = waves * (bn == 256 ? 1.0 : 0.8);
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
         best = TileChoice{pair, bn};
       }
     }
