@@ -26,6 +26,19 @@ are taken exactly):
   page, and the SiLU derivative, "Unsloth提速秘诀…", §2.2); gradients for X and for
   the six adapter matrices only (W and the norm weight are frozen).
 
+Variants around the path (off by default):
+
+  residual: the decoder layer adds the sub-block's output to its input, Y = X + MLP(RMSNorm(X)),
+  so the backward adds dY to dX ("Unsloth加速原理揭秘", §3.1, the LoRA forward that ends in a
+  residual add; the Llama residual stream).
+
+  dw: gradient of the norm weight, for a trainable-norm variant (the norm weight is frozen in
+  LoRA fine-tuning): H = X * rstd * w gives dw_j = sum_t dH_tj x_tj rstd_t
+  ("Unsloth提速秘诀…", §3.2, the norm kernel's weight operand).
+
+  merge: the adapter folded into the frozen weight for export, W + s B A ("Unsloth提速秘诀…",
+  §3.1, "LoRA Update + Weight Merge"; "Unsloth 深度实战", §5.1, the merged 16-bit save).
+
 Rows are independent in every step except the adapter-gradient reductions over T,
 so long inputs are processed in row chunks with fp64 accumulation across chunks.
 """
@@ -72,8 +85,15 @@ def lora_linear(x, W, A, B, s):
     return x @ W.T + s * ((x @ A.T) @ B.T)
 
 
-def forward(X, w, eps, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
-    """Full forward; returns every intermediate the backward needs."""
+def merge(W, A, B, s):
+    """The adapter folded into the frozen weight: W + s B A (W [out x in], B [out x r],
+    A [r x in])."""
+    return W + s * (B @ A)
+
+
+def forward(X, w, eps, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual=False):
+    """Full forward; returns every intermediate the backward needs.  With `residual`
+    the sub-block's input is added to its output."""
     H, rstd = rmsnorm_fwd(X, w, eps)
     Pg = H @ Ag.T
     Pu = H @ Au.T
@@ -82,11 +102,14 @@ def forward(X, w, eps, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
     Act = silu(G) * U
     Pd = Act @ Ad.T
     Y = Act @ Wd.T + s * (Pd @ Bd.T)
+    if residual:
+        Y = Y + X
     return dict(rstd=rstd, H=H, G=G, U=U, Act=Act, Pg=Pg, Pu=Pu, Pd=Pd, Y=Y)
 
 
-def backward(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
-    """Gradients of <dY, Y> w.r.t. X and the six adapter matrices."""
+def backward(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual=False):
+    """Gradients of <dY, Y> w.r.t. X, the six adapter matrices and the norm weight (dw,
+    for the trainable-norm variant)."""
     H, G, U, Act = fw["H"], fw["G"], fw["U"], fw["Act"]
     Pg, Pu, Pd = fw["Pg"], fw["Pu"], fw["Pd"]
     # down projection  Y = Act Wd^T + s (Act Ad^T) Bd^T
@@ -106,19 +129,22 @@ def backward(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
     dAu = s * (Qu.T @ H)
     dH = dG @ Wg + dU @ Wu + s * (Qg @ Ag + Qu @ Au)
     dX = rmsnorm_bwd(dH, X, w, fw["rstd"])
-    return dict(dX=dX, dAg=dAg, dBg=dBg, dAu=dAu, dBu=dBu, dAd=dAd, dBd=dBd,
+    if residual:
+        dX = dX + dY
+    dw = np.sum(dH * X * fw["rstd"][:, None], axis=0)
+    return dict(dX=dX, dAg=dAg, dBg=dBg, dAu=dAu, dBu=dBu, dAd=dAd, dBd=dBd, dw=dw,
                 dAct=dAct, dG=dG, dU=dU, dH=dH, Qd=Qd, Qg=Qg, Qu=Qu)
 
 
-_GRADS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
+_GRADS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd", "dw")
 
 
-def fwd_bwd(inp: dict, s: float, eps: float, chunk: int = 2048, keep=("Y", "dX")):
+def fwd_bwd(inp: dict, s: float, eps: float, chunk: int = 2048, keep=("Y", "dX"), residual=False):
     """Forward + backward over all rows in chunks of `chunk` tokens.
 
     `inp` holds fp64 arrays X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, dY.
     Returns the per-row tensors named in `keep` (concatenated over chunks) and the
-    six adapter gradients summed over all rows.
+    six adapter gradients and dw summed over all rows.
     """
     X, dY = inp["X"], inp["dY"]
     W = {k: inp[k] for k in ("w", "Wg", "Wu", "Wd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
@@ -128,9 +154,9 @@ def fwd_bwd(inp: dict, s: float, eps: float, chunk: int = 2048, keep=("Y", "dX")
     for t0 in range(0, T, chunk):
         xs, dys = X[t0:t0 + chunk], dY[t0:t0 + chunk]
         fw = forward(xs, W["w"], eps, W["Wg"], W["Wu"], W["Wd"], W["Ag"], W["Bg"],
-                     W["Au"], W["Bu"], W["Ad"], W["Bd"], s)
+                     W["Au"], W["Bu"], W["Ad"], W["Bd"], s, residual)
         bw = backward(fw, dys, xs, W["w"], W["Wg"], W["Wu"], W["Wd"], W["Ag"], W["Bg"],
-                      W["Au"], W["Bu"], W["Ad"], W["Bd"], s)
+                      W["Au"], W["Bu"], W["Ad"], W["Bd"], s, residual)
         both = {**fw, **bw}
         for k in keep:
             rows[k].append(both[k])

@@ -7,28 +7,28 @@ from oracle import lora_mlp_ref as ref
 from tests.test_oracle_pins import fd_errors, tiny_inputs
 
 
-def _bwd_drop_lora_dH(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
-    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s)
+def _bwd_drop_lora_dH(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual=False):
+    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual)
     dH = out["dG"] @ Wg + out["dU"] @ Wu          # missing s (Qg Ag + Qu Au)
     out["dX"] = ref.rmsnorm_bwd(dH, X, w, fw["rstd"])
     return out
 
 
-def _bwd_swap_pg_pu(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
-    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s)
+def _bwd_swap_pg_pu(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual=False):
+    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual)
     out["dBg"] = s * (out["dG"].T @ fw["Pu"])      # wrong index (up instead of gate)
     return out
 
 
-def _bwd_transposed_dAd(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
-    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s)
+def _bwd_transposed_dAd(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual=False):
+    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual)
     Qd = dY @ Bd
     out["dAd"] = s * (Qd.T @ (out["dAct"]))        # wrong operand
     return out
 
 
-def _bwd_no_scale_dBd(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s):
-    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s)
+def _bwd_no_scale_dBd(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual=False):
+    out = ORIG_BWD(fw, dY, X, w, Wg, Wu, Wd, Ag, Bg, Au, Bu, Ad, Bd, s, residual)
     out["dBd"] = dY.T @ fw["Pd"]                    # dropped scaling
     return out
 

@@ -23,30 +23,31 @@ def tiny_inputs(T=5, d=8, f=12, r=3, seed=11, bf16=False):
     return s, {k: synth.tensor_f64(k, s, seed) for k in synth.TENSOR_ORDER}
 
 
-def run(inp, s, eps=1e-6):
-    fw = ref.forward(inp["X"], inp["w"], eps, *(inp[k] for k in NAMES[1:]), s.scale)
-    bw = ref.backward(fw, inp["dY"], inp["X"], *(inp[k] for k in NAMES), s.scale)
+def run(inp, s, eps=1e-6, residual=False):
+    fw = ref.forward(inp["X"], inp["w"], eps, *(inp[k] for k in NAMES[1:]), s.scale, residual)
+    bw = ref.backward(fw, inp["dY"], inp["X"], *(inp[k] for k in NAMES), s.scale, residual)
     return fw, bw
 
 
-def loss(inp, s, eps=1e-6):
-    fw = ref.forward(inp["X"], inp["w"], eps, *(inp[k] for k in NAMES[1:]), s.scale)
+def loss(inp, s, eps=1e-6, residual=False):
+    fw = ref.forward(inp["X"], inp["w"], eps, *(inp[k] for k in NAMES[1:]), s.scale, residual)
     return float(np.sum(inp["dY"] * fw["Y"]))
 
 
-GRAD_OF = {"X": "dX", "Ag": "dAg", "Bg": "dBg", "Au": "dAu", "Bu": "dBu", "Ad": "dAd", "Bd": "dBd"}
+GRAD_OF = {"X": "dX", "Ag": "dAg", "Bg": "dBg", "Au": "dAu", "Bu": "dBu", "Ad": "dAd", "Bd": "dBd",
+           "w": "dw"}
 
 
-def fd_errors(inp, s, eps=1e-6, h=1e-5, seed=5):
+def fd_errors(inp, s, eps=1e-6, h=1e-5, seed=5, residual=False):
     """Relative error of <grad, V> against a central difference of L = <dY, Y>."""
-    _, bw = run(inp, s, eps)
+    _, bw = run(inp, s, eps, residual)
     rng = np.random.default_rng(seed)
     errs = {}
     for name, gname in GRAD_OF.items():
         V = rng.standard_normal(inp[name].shape)
         plus = dict(inp); plus[name] = inp[name] + h * V
         minus = dict(inp); minus[name] = inp[name] - h * V
-        fd = (loss(plus, s, eps) - loss(minus, s, eps)) / (2 * h)
+        fd = (loss(plus, s, eps, residual) - loss(minus, s, eps, residual)) / (2 * h)
         an = float(np.sum(bw[gname] * V))
         errs[name] = abs(fd - an) / max(abs(fd), 1e-300)
     return errs
@@ -58,6 +59,47 @@ def test_backward_matches_finite_differences():
     s, inp = tiny_inputs()
     errs = fd_errors(inp, s)
     assert max(errs.values()) < 1e-7, errs
+
+
+def test_residual_variant_matches_finite_differences():
+    """Y = X + MLP(RMSNorm(X)): the dY term in dX (and every other gradient) against FD."""
+    s, inp = tiny_inputs(seed=31)
+    errs = fd_errors(inp, s, residual=True)
+    # <dY, X> adds a large constant to L for every direction but X, so the central
+    # difference cancels more digits there; the X direction carries the residual term
+    assert errs["X"] < 1e-8, errs
+    assert max(errs.values()) < 5e-6, errs
+    fr, br = run(inp, s, residual=True)
+    f0, b0 = run(inp, s)
+    np.testing.assert_allclose(fr["Y"] - f0["Y"], inp["X"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(br["dX"] - b0["dX"], inp["dY"], rtol=1e-12, atol=1e-14)
+    for k in ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd", "dw"):
+        np.testing.assert_array_equal(br[k], b0[k])
+
+
+def test_norm_weight_grad_closed_form_scale_invariance():
+    """With eps = 0 the norm output does not depend on the scale of a row, so dw from
+    rows scaled by c > 0 equals dw of the unscaled rows."""
+    s, inp = tiny_inputs(seed=32)
+    _, b1 = run(inp, s, eps=0.0)
+    scaled = dict(inp)
+    scaled["X"] = inp["X"] * np.linspace(0.5, 3.0, inp["X"].shape[0])[:, None]
+    _, b2 = run(scaled, s, eps=0.0)
+    np.testing.assert_allclose(b2["dw"], b1["dw"], rtol=1e-11, atol=1e-14)
+
+
+def test_merge_brute_force_loops():
+    """ref.merge against an element-by-element loop of W_ij + s sum_k B_ik A_kj."""
+    rng = np.random.default_rng(33)
+    W, A, B = rng.standard_normal((5, 7)), rng.standard_normal((3, 7)), rng.standard_normal((5, 3))
+    s = 0.75
+    M = ref.merge(W, A, B, s)
+    for i in range(5):
+        for j in range(7):
+            acc = 0.0
+            for k in range(3):
+                acc += B[i, k] * A[k, j]
+            assert abs(M[i, j] - (W[i, j] + s * acc)) < 1e-13
 
 
 def test_backward_matches_finite_differences_bf16_inputs_eps_large():
@@ -167,9 +209,9 @@ def test_merge_equivalence():
     sc = s.scale
     fw, bw = run(inp, s)
     merged = dict(inp)
-    merged["Wg"] = inp["Wg"] + sc * inp["Bg"] @ inp["Ag"]
-    merged["Wu"] = inp["Wu"] + sc * inp["Bu"] @ inp["Au"]
-    merged["Wd"] = inp["Wd"] + sc * inp["Bd"] @ inp["Ad"]
+    merged["Wg"] = ref.merge(inp["Wg"], inp["Ag"], inp["Bg"], sc)
+    merged["Wu"] = ref.merge(inp["Wu"], inp["Au"], inp["Bu"], sc)
+    merged["Wd"] = ref.merge(inp["Wd"], inp["Ad"], inp["Bd"], sc)
     for k in ("Ag", "Au", "Ad", "Bg", "Bu", "Bd"):
         merged[k] = np.zeros_like(inp[k])
     fm, bm = run(merged, s)
