@@ -337,6 +337,67 @@ def measured_traffic(kernel: str, config: str):
     return None
 
 
+def extras(args):
+    """The variants around the path at the 8B shape, one JSON line: a step with the
+    residual connection and the norm-weight gradient against the plain step, the dw
+    kernel and the weight merge of a [f x d] matrix against the HBM roofline."""
+    import torch
+    from lora_fine_tuning_rmsnorm_b200 import ops, synth
+    from lora_fine_tuning_rmsnorm_b200.runner import Problem
+    torch.cuda.set_device(0)
+    hbm = peaks()[0]
+    shape = shape_for("8b", args.T)
+    T, d, f, r = shape.T, shape.d, shape.f, shape.r
+    bits = synth.make_inputs_bits(shape)
+    out = {"extras": True, "config": config_for(args, shape, 1)}
+
+    def timed_steps(pb):
+        for _ in range(args.warmup):
+            pb.step()
+        torch.cuda.synchronize()
+        ops.timing_enable(True)
+        ops.timing_collect()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            pb.step()
+        e1.record()
+        torch.cuda.synchronize()
+        ph = ops.timing_collect()
+        ops.timing_enable(False)
+        return e0.elapsed_time(e1) / args.steps, ph
+
+    plain = Problem(shape, bits)
+    ms_plain, _ = timed_steps(plain)
+    del plain
+    var = Problem(shape, bits, residual=True, norm_grad=True)
+    ms_var, ph = timed_steps(var)
+    dw_ms, dw_n = ph.get("norm_weight_grad", (0.0, 0))
+    dw_bytes = T * (4 * d + 2 * d + 4) + 4 * d   # dH fp32 + X bf16 + rstd read, dw written
+    dw_gbs = dw_bytes / (dw_ms / dw_n / 1e3) / 1e9 if dw_n else None
+    out["residual_and_norm_grad"] = {"ms_per_step": ms_var, "plain_ms_per_step": ms_plain,
+                                     "overhead_ms": ms_var - ms_plain}
+    out["norm_weight_grad"] = {"us_per_launch": 1e3 * dw_ms / dw_n if dw_n else None, "algorithmic_bytes": dw_bytes,
+                               "GB/s": dw_gbs, "frac_of_hbm": dw_gbs / hbm if dw_gbs else None}
+    W, A, B = var.t["Wg"], var.t["Ag"], var.t["Bg"]
+    Wm = torch.empty_like(W)
+    for _ in range(3):
+        ops.merge_weights(W, A, B, shape.scale, out=Wm)
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ops.merge_weights(W, A, B, shape.scale, out=Wm)
+    e1.record()
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / reps
+    mb = f * d * 4 + (r * d + f * r) * 2          # W read + Wm written (+ A, B)
+    out["merge_weights"] = {"rows": f, "cols": d, "r": r, "us_per_launch": us, "algorithmic_bytes": mb,
+                            "GB/s": mb / (us / 1e6) / 1e9, "frac_of_hbm": mb / (us / 1e6) / 1e9 / hbm}
+    out["hbm_peak_gbs"] = hbm
+    print(json.dumps(out), flush=True)
+
+
 def sweep(args):
     """Rank / length sweep at d = 4096, f = 14336 (alpha = 16): one JSON line per
     point with tokens/s and the dense-GEMM vs memory-bound phase split."""
@@ -382,6 +443,8 @@ def main():
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling on small cases)")
     ap.add_argument("--sweep", action="store_true", help="rank/length sweep, one JSON line per point")
+    ap.add_argument("--extras", action="store_true",
+                    help="residual / norm-weight-gradient step and weight merge, one JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -392,6 +455,9 @@ def main():
         return
     if args.sweep:
         sweep(args)
+        return
+    if args.extras:
+        extras(args)
         return
     if world > 1:
         import datetime

@@ -63,7 +63,9 @@ enum lora_wfmt {
  * Limits: 1 <= T < 2^31; d, f multiples of 8 with 8 <= d <= 65536, 8 <= f;
  * r a multiple of 8 with 8 <= r <= 128.  scale = alpha / r (any finite value).
  * wfmt = LORA_WFMT_BF16 or LORA_WFMT_4BIT (then qblock must be 64 and d, f
- * multiples of 256). */
+ * multiples of 256).  residual = 1 adds the decoder layer's residual connection
+ * around the sub-block ("Unsloth加速原理揭秘", §3.1, the LoRA forward ending in a
+ * residual add): Y = X + MLP(RMSNorm(X)) and dX gets + dY; 0 = the sub-block alone. */
 typedef struct lora_mlp_dims {
   int64_t T;
   int32_t d, f, r;
@@ -71,6 +73,7 @@ typedef struct lora_mlp_dims {
   float scale;
   int32_t wfmt;
   int32_t qblock;
+  int32_t residual;
 } lora_mlp_dims;
 
 /* Frozen base weights, nn.Linear layout (out x in):
@@ -109,7 +112,11 @@ typedef struct lora_mlp_adapters {
 
 /* Adapter gradients, fp32, same shapes as the adapters.  OVERWRITTEN by the
  * backward (not accumulated).  Sums over T are formed with fp32 atomics, so the
- * last bits may differ between runs. */
+ * last bits may differ between runs.
+ * dw [d] fp32: gradient of the norm weight, dw_j = sum_t dH_tj x_tj rstd_t, for a
+ * trainable-norm variant ("Unsloth提速秘诀：Triton内核如何加速反向传播", §3.2, the norm
+ * kernel's weight operand); NULL = the norm weight is frozen (LoRA) and dw is not
+ * computed.  Overwritten, fp32 atomics as above. */
 typedef struct lora_mlp_grads {
   float* dAg;
   float* dBg;
@@ -117,6 +124,7 @@ typedef struct lora_mlp_grads {
   float* dBu;
   float* dAd;
   float* dBd;
+  float* dw;
 } lora_mlp_grads;
 
 /* Byte offsets of the saved-activation context (one caller-owned device buffer,
@@ -167,6 +175,17 @@ int lora_rmsnorm_fwd(int64_t T, int32_t d, float eps, const void* X, const void*
 int lora_rmsnorm_bwd(int64_t T, int32_t d, const float* dH, const void* X, const void* w,
                      const float* rstd, void* dX, void* stream);
 
+/* Adapter folded into its frozen weight for export ("Unsloth提速秘诀…", §3.1, "LoRA
+ * Update + Weight Merge"; "Unsloth 深度实战", §5.1, the merged 16-bit save):
+ *   Wm[o][i] = bf16( W[o][i] + scale * sum_{k<r} B[o][k] A[k][i] )
+ * with the sum in fp32 over k = 0..r-1, then one fp32 fma (scale * sum + W), then
+ * one rounding to bf16 (RN).
+ * W, Wm [rows x cols] bf16 row-major (Wm may equal W: in place); A [r x cols], B
+ * [rows x r] bf16 row-major.  cols a multiple of 8, 1 <= r <= 256, pointers 16-byte
+ * aligned (B: 2-byte).  Asynchronous on `stream`; nothing is allocated. */
+int lora_merge_weights(int64_t rows, int64_t cols, int32_t r, float scale, const void* W, const void* A,
+                       const void* B, void* Wm, void* stream);
+
 /* 4-bit blockwise quantisation of a bf16 matrix (flattened row-major, numel a
  * multiple of block = 64): per block absmax = max|w| (fp32); code index
  * idx = #{ i in 0..14 : w > absmax * m_i }, m_i = fl32((c_i + c_{i+1}) / 2), decided
@@ -210,7 +229,7 @@ int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, cons
  * is bracketed by CUDA events on the caller's stream.  lora_mlp_timing_collect()
  * synchronises those events and returns, per phase id, the summed milliseconds and
  * the number of launches since the previous collect (arrays of LORA_NUM_PHASES). */
-#define LORA_NUM_PHASES 16
+#define LORA_NUM_PHASES 17
 int lora_mlp_timing_enable(int32_t on);
 int lora_mlp_timing_collect(double* ms, int64_t* launches);
 const char* lora_mlp_phase_name(int32_t phase);

@@ -64,7 +64,7 @@ __host__ __device__ inline Q4Layout q4_layout(int bn, int pair, int fuse, int b_
 
 enum Epi : int {
   EPI_F32 = 0,         // out[0] fp32 = acc_a * alpha at column a * out_acc_col (+ split * split_stride)
-  EPI_BF16 = 1,        // out[0] bf16 = acc_a * alpha, accumulator a at column a * out_acc_col
+  EPI_BF16 = 1,        // out[0] bf16 = acc_a * alpha (+ in[0] when set), accumulator a at column a * out_acc_col
   EPI_SWIGLU_FWD = 2,  // acc0 = G, acc1 = U -> out[0] G, out[1] U, out[2] silu(G) * U (bf16)
   EPI_SWIGLU_BWD = 3,  // acc0 = dAct; in[0] G, in[1] U -> out[0] dG, out[1] dU (bf16)
   EPI_ATOMIC = 4       // accumulator a atomically added into fp32 output rng[a] (split-K reductions)
@@ -480,11 +480,23 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               if (n + 8 * h < p.N) {
+                float v8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(r[8 * h + e]) * p.alpha;
+                if (p.in[0]) {  // residual input (bf16, same layout as the output) added in fp32
+                  float x8[8];
+                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.in[0]) +
+                                                                       row * p.ld_in + n + 8 * h));
+                  x8[0] = bf16lo(xv.x); x8[1] = bf16hi(xv.x); x8[2] = bf16lo(xv.y); x8[3] = bf16hi(xv.y);
+                  x8[4] = bf16lo(xv.z); x8[5] = bf16hi(xv.z); x8[6] = bf16lo(xv.w); x8[7] = bf16hi(xv.w);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) v8[e] += x8[e];
+                }
                 uint4 v;
-                v.x = pack_bf16x2(__uint_as_float(r[8 * h + 0]) * p.alpha, __uint_as_float(r[8 * h + 1]) * p.alpha);
-                v.y = pack_bf16x2(__uint_as_float(r[8 * h + 2]) * p.alpha, __uint_as_float(r[8 * h + 3]) * p.alpha);
-                v.z = pack_bf16x2(__uint_as_float(r[8 * h + 4]) * p.alpha, __uint_as_float(r[8 * h + 5]) * p.alpha);
-                v.w = pack_bf16x2(__uint_as_float(r[8 * h + 6]) * p.alpha, __uint_as_float(r[8 * h + 7]) * p.alpha);
+                v.x = pack_bf16x2(v8[0], v8[1]);
+                v.y = pack_bf16x2(v8[2], v8[3]);
+                v.z = pack_bf16x2(v8[4], v8[5]);
+                v.w = pack_bf16x2(v8[6], v8[7]);
                 st_out(reinterpret_cast<uint4*>(o + 8 * h), v, p.stream_out);
               }
             }

@@ -158,10 +158,10 @@ const char* kPhaseNames[LORA_NUM_PHASES] = {
     "rmsnorm_fwd", "proj_P_gate_up", "gemm_gate_up_swiglu", "proj_P_down", "gemm_down",
     "proj_Q_down", "gemm_dact_swiglu_bwd", "proj_Q_gate_up", "gemm_dH", "rmsnorm_bwd",
     "zero_grads", "reduce_dA_gate_up", "reduce_dB_gate_up", "reduce_dB_down", "reduce_dA_down",
-    "other"};
+    "norm_weight_grad", "other"};
 enum Phase {
   PH_RMS_FWD = 0, PH_P_GU, PH_GATEUP, PH_P_D, PH_DOWN, PH_Q_D, PH_DACT, PH_Q_GU, PH_DH,
-  PH_RMS_BWD, PH_ZERO, PH_RED_DA_GU, PH_RED_DB_GU, PH_RED_DB_D, PH_RED_DA_D, PH_OTHER
+  PH_RMS_BWD, PH_ZERO, PH_RED_DA_GU, PH_RED_DB_GU, PH_RED_DB_D, PH_RED_DA_D, PH_DW, PH_OTHER
 };
 
 struct Timing {
@@ -301,7 +301,7 @@ int launch_rms_fwd(cudaStream_t st, const void* X, const void* w, void* H, float
 }
 
 int launch_rms_bwd(cudaStream_t st, const float* dH, const void* X, const void* w, const float* rstd, void* dX,
-                   long long T, int d) {
+                   long long T, int d, const void* dY = nullptr) {
   const int nvec = d / 8;
   int threads = kRowThreads, vpt = (nvec + threads - 1) / threads;
   if (vpt > 4) {
@@ -313,13 +313,14 @@ int launch_rms_bwd(cudaStream_t st, const float* dH, const void* X, const void* 
   auto X16 = static_cast<const uint16_t*>(X);
   auto w16 = static_cast<const uint16_t*>(w);
   auto dX16 = static_cast<uint16_t*>(dX);
+  auto dY16 = static_cast<const uint16_t*>(dY);
   PhaseScope ps(st, PH_RMS_BWD);
   for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
     unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
     switch (v) {
-      case 1: rmsnorm_bwd_kernel<1><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dX16 + r0 * d, d); break;
-      case 2: rmsnorm_bwd_kernel<2><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dX16 + r0 * d, d); break;
-      default: rmsnorm_bwd_kernel<4><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dX16 + r0 * d, d); break;
+      case 1: rmsnorm_bwd_kernel<1><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
+      case 2: rmsnorm_bwd_kernel<2><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
+      default: rmsnorm_bwd_kernel<4><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
     }
   }
   CUDA_TRY(cudaGetLastError());
@@ -367,6 +368,7 @@ int check_dims(const lora_mlp_dims* D) {
   if (D->d > 65536) return fail(LORA_ERR_UNSUPPORTED, "d = %d > 65536", D->d);
   if (D->r > 128) return fail(LORA_ERR_UNSUPPORTED, "r = %d > 128", D->r);
   if (D->wfmt != LORA_WFMT_BF16 && D->wfmt != LORA_WFMT_4BIT) return fail(LORA_ERR_INVALID_ARG, "bad wfmt");
+  if (D->residual != 0 && D->residual != 1) return fail(LORA_ERR_INVALID_ARG, "residual must be 0 or 1");
   if (D->wfmt == LORA_WFMT_4BIT) {
     if (D->qblock != 64) return fail(LORA_ERR_UNSUPPORTED, "qblock must be 64");
     if (D->d % 256 || D->f % 256) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights need d, f multiples of 256");
@@ -646,6 +648,25 @@ int lora_rmsnorm_bwd(int64_t T, int32_t d, const float* dH, const void* X, const
   return launch_rms_bwd(static_cast<cudaStream_t>(stream), dH, X, w, rstd, dX, T, d);
 }
 
+int lora_merge_weights(int64_t rows, int64_t cols, int32_t r, float scale, const void* W, const void* A,
+                       const void* B, void* Wm, void* stream) {
+  if (rows < 1 || cols < 8 || cols % 8) return fail(LORA_ERR_INVALID_ARG, "bad rows/cols (%lld, %lld)", (long long)rows, (long long)cols);
+  if (r < 1 || r > 256) return fail(LORA_ERR_UNSUPPORTED, "r = %d outside 1..256", r);
+  if (!std::isfinite(scale)) return fail(LORA_ERR_INVALID_ARG, "scale is not finite");
+  TRY(check_ptrs({W, A, Wm}));
+  if (!B) return fail(LORA_ERR_INVALID_ARG, "B is NULL");
+  if (reinterpret_cast<uintptr_t>(B) % 2) return fail(LORA_ERR_ALIGNMENT, "B is not 2-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>((cols / 8 + 127) / 128),
+                  static_cast<unsigned>(std::min<long long>((rows + 3) / 4, 65535)));
+  PhaseScope ps(st, PH_OTHER);
+  merge_weights_kernel<<<grid, 128, 0, st>>>(static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(A),
+                                             static_cast<const uint16_t*>(B), static_cast<uint16_t*>(Wm), rows,
+                                             cols, r, scale);
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
+
 int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float* codebook16, uint8_t* codes,
                        float* absmax, void* stream) {
   if (block != 64) return fail(LORA_ERR_UNSUPPORTED, "block must be 64");
@@ -813,6 +834,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
+    if (D->residual) { a.in[0] = X; a.ld_in = d; }  // Y = X + ...
     a.stream_out = 1;
     set_band(a, 8);
     if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 1>(a, st, PH_DOWN)));
@@ -831,6 +853,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
+    if (D->residual) { a.in[0] = X; a.ld_in = d; }  // Y = X + ...
     a.stream_out = 1;
     set_band(a, 8);
     if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_DOWN)));
@@ -847,6 +870,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   const bool q4 = D->wfmt == LORA_WFMT_4BIT;
   TRY(check_ptrs({dY, X, rms_w, ctx, dX, workspace, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd,
                   gr->dAg, gr->dBg, gr->dAu, gr->dBu, gr->dAd, gr->dBd}));
+  if (gr->dw) TRY(check_ptrs({gr->dw}));
   if (q4) TRY(check_ptrs({W->Qg, W->Qu, W->Qd, W->absmax_g, W->absmax_u, W->absmax_d, W->codebook}));
   else TRY(check_ptrs({W->Wg, W->Wu, W->Wd}));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -999,7 +1023,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
   }
   // S10: dX = RMSNorm backward (cached rstd)
-  TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));
+  TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d, D->residual ? dY : nullptr));
 
   // adapter gradients: overwrite semantics -> zero, then split-T atomic reductions
   {
@@ -1010,8 +1034,17 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     z.p[3] = gr->dBu; z.n[3] = static_cast<long long>(f) * r;
     z.p[4] = gr->dAd; z.n[4] = static_cast<long long>(r) * f;
     z.p[5] = gr->dBd; z.n[5] = static_cast<long long>(d) * r;
+    z.p[6] = gr->dw;  z.n[6] = gr->dw ? d : 0;
     PhaseScope ps(st, PH_ZERO);
-    zero6_kernel<<<296, 256, 0, st>>>(z);
+    zero_grads_kernel<<<296, 256, 0, st>>>(z);
+    CUDA_TRY(cudaGetLastError());
+  }
+  // norm-weight gradient (trainable-norm variant only): dw_j = sum_t dH_tj x_tj rstd_t
+  if (gr->dw) {
+    const int rows = static_cast<int>(std::max<long long>(64, (T + 65534) / 65535));
+    const dim3 grid(static_cast<unsigned>((d / 4 + 255) / 256), static_cast<unsigned>((T + rows - 1) / rows));
+    PhaseScope ps(st, PH_DW);
+    norm_weight_grad_kernel<<<grid, 256, 0, st>>>(dH, static_cast<const uint16_t*>(X), rstd, gr->dw, T, d, rows);
     CUDA_TRY(cudaGetLastError());
   }
   // Adapter-gradient reductions over T: accumulator rows are the big dimension

@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restri
                                                            const uint16_t* __restrict__ X,
                                                            const uint16_t* __restrict__ w,
                                                            const float* __restrict__ rstd,
+                                                           const uint16_t* __restrict__ dY,
                                                            uint16_t* __restrict__ dX, int d) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
@@ -118,6 +119,12 @@ __global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restri
     float o[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j] = rs * (g[i][j] - xh[i][j] * c);
+    if (dY) {  // residual connection: the sub-block's input gradient also gets dY
+      float yf[8];
+      unpack8(__ldcs(reinterpret_cast<const uint4*>(dY + row * d) + v), yf);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] += yf[j];
+    }
     uint4 ov;
     ov.x = pack_bf16x2(o[0], o[1]);
     ov.y = pack_bf16x2(o[2], o[3]);
@@ -173,15 +180,87 @@ __global__ void splitk_finalize_kernel(const float* __restrict__ part, int split
   *reinterpret_cast<uint2*>(out + i4) = o;
 }
 
+constexpr int kZeroMax = 7;
 struct ZeroList {
-  float* p[6];
-  long long n[6];
+  float* p[kZeroMax];  // NULL entries (n = 0) are skipped
+  long long n[kZeroMax];
 };
-__global__ void zero6_kernel(ZeroList z) {
+__global__ void zero_grads_kernel(ZeroList z) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (int k = 0; k < 6; ++k)
+  for (int k = 0; k < kZeroMax; ++k)
     for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < z.n[k]; i += stride)
       z.p[k][i] = 0.f;
+}
+
+// Norm-weight gradient of H = X * rstd * w: dw_j += sum over a chunk of `rows` rows of
+// dH_tj * x_tj * rstd_t, added to dw (zeroed by the caller) with fp32 atomics.  A thread
+// owns 4 consecutive columns, so every row of dH / X is read coalesced.
+__global__ void __launch_bounds__(256) norm_weight_grad_kernel(const float* __restrict__ dH,
+                                                               const uint16_t* __restrict__ X,
+                                                               const float* __restrict__ rstd,
+                                                               float* __restrict__ dw, long long T, int d,
+                                                               int rows) {
+  const long long c = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (c >= d) return;
+  const long long t0 = static_cast<long long>(blockIdx.y) * rows;
+  const long long t1 = t0 + rows < T ? t0 + rows : T;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (long long t = t0; t < t1; ++t) {
+    const float rs = __ldg(rstd + t);
+    const float4 h = __ldcs(reinterpret_cast<const float4*>(dH + t * d + c));
+    const uint2 xv = __ldcs(reinterpret_cast<const uint2*>(X + t * d + c));
+    a0 = fmaf(h.x * bf16lo(xv.x), rs, a0);
+    a1 = fmaf(h.y * bf16hi(xv.x), rs, a1);
+    a2 = fmaf(h.z * bf16lo(xv.y), rs, a2);
+    a3 = fmaf(h.w * bf16hi(xv.y), rs, a3);
+  }
+  atomicAdd(dw + c, a0);
+  atomicAdd(dw + c + 1, a1);
+  atomicAdd(dw + c + 2, a2);
+  atomicAdd(dw + c + 3, a3);
+}
+
+// Adapter folded into its weight: Wm = bf16(fma(s, sum_k B[o][k] A[k][j], W[o][j])), the sum
+// in fp32 over k = 0..r-1.  A thread owns 4 rows x 8 consecutive columns, so each A
+// vector it loads serves 4 rows; the B values of the block's rows are shared by all of its
+// threads (broadcast loads).  W and Wm may alias: each element is read and written by
+// one thread only.
+__global__ void __launch_bounds__(128) merge_weights_kernel(const uint16_t* W, const uint16_t* __restrict__ A,
+                                                            const uint16_t* __restrict__ B, uint16_t* Wm,
+                                                            long long rows, long long cols, int r, float s) {
+  const long long j = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (j >= cols) return;
+  for (long long o0 = static_cast<long long>(blockIdx.y) * 4; o0 < rows; o0 += static_cast<long long>(gridDim.y) * 4) {
+    float acc[4][8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[q][e] = 0.f;
+    for (int k = 0; k < r; ++k) {
+      float a[8];
+      unpack8(__ldg(reinterpret_cast<const uint4*>(A + static_cast<long long>(k) * cols + j)), a);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (o0 + q >= rows) break;
+        const float b = __uint_as_float(static_cast<uint32_t>(__ldg(B + (o0 + q) * r + k)) << 16);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[q][e] = fmaf(b, a[e], acc[q][e]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (o0 + q >= rows) break;
+      const long long off = (o0 + q) * cols + j;
+      float w[8];
+      unpack8(*reinterpret_cast<const uint4*>(W + off), w);
+      uint4 ov;
+      ov.x = pack_bf16x2(fmaf(s, acc[q][0], w[0]), fmaf(s, acc[q][1], w[1]));
+      ov.y = pack_bf16x2(fmaf(s, acc[q][2], w[2]), fmaf(s, acc[q][3], w[3]));
+      ov.z = pack_bf16x2(fmaf(s, acc[q][4], w[4]), fmaf(s, acc[q][5], w[5]));
+      ov.w = pack_bf16x2(fmaf(s, acc[q][6], w[6]), fmaf(s, acc[q][7], w[7]));
+      *reinterpret_cast<uint4*>(Wm + off) = ov;
+    }
+  }
 }
 
 }  // namespace lm

@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "lora_mlp.h")
 LORA_OK = 0
 ERRORS = {-1: "INVALID_ARG", -2: "ALIGNMENT", -3: "UNSUPPORTED", -4: "CUDA", -5: "TIMEOUT"}
 WFMT_BF16, WFMT_4BIT = 0, 1
-NUM_PHASES = 16
+NUM_PHASES = 17
 
 
 class LoraError(RuntimeError):
@@ -29,7 +29,7 @@ class LoraError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("f", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("eps", ctypes.c_float), ("scale", ctypes.c_float), ("wfmt", ctypes.c_int32),
-                ("qblock", ctypes.c_int32)]
+                ("qblock", ctypes.c_int32), ("residual", ctypes.c_int32)]
 
 
 class Weights(ctypes.Structure):
@@ -42,7 +42,7 @@ class Adapters(ctypes.Structure):
 
 
 class Grads(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd", "dw")]
 
 
 class CtxLayout(ctypes.Structure):
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
         "lora_rmsnorm_fwd": [i64, i32, f32, vp, vp, vp, vp, vp],
         "lora_rmsnorm_bwd": [i64, i32, vp, vp, vp, vp, vp, vp],
         "lora_quantize_4bit": [vp, i64, i32, vp, vp, vp, vp],
+        "lora_merge_weights": [i64, i64, i32, f32, vp, vp, vp, vp, vp],
         "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, i32, vp],
         "lora_lowrank_proj_noalloc": [i64, i32, i32, f32, vp, vp, vp, vp],
         "lora_mlp_timing_enable": [i32],
@@ -113,8 +114,8 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_dims(T, d, f, r, eps=1e-6, scale=1.0, wfmt=WFMT_BF16, qblock=64) -> Dims:
-    return Dims(T, d, f, r, eps, scale, wfmt, qblock)
+def make_dims(T, d, f, r, eps=1e-6, scale=1.0, wfmt=WFMT_BF16, qblock=64, residual=False) -> Dims:
+    return Dims(T, d, f, r, eps, scale, wfmt, qblock, int(bool(residual)))
 
 
 def ctx_layout(dims: Dims) -> CtxLayout:
@@ -163,8 +164,20 @@ def make_adapters(Ag, Bg, Au, Bu, Ad, Bd) -> Adapters:
     return Adapters(*[_p(t) for t in (Ag, Bg, Au, Bu, Ad, Bd)])
 
 
-def make_grads(dAg, dBg, dAu, dBu, dAd, dBd) -> Grads:
-    return Grads(*[_p(t) for t in (dAg, dBg, dAu, dBu, dAd, dBd)])
+def make_grads(dAg, dBg, dAu, dBu, dAd, dBd, dw=None) -> Grads:
+    """dw (fp32 [d]) only for a trainable norm weight; None leaves it uncomputed."""
+    return Grads(*[_p(t) for t in (dAg, dBg, dAu, dBu, dAd, dBd, dw)])
+
+
+def merge_weights(W, A, B, scale, out=None, stream=None):
+    """Wm = bf16(W + scale * B A) (W [rows x cols], A [r x cols], B [rows x r], bf16 on the
+    device); `out` may be W itself (in place)."""
+    import torch
+    rows, cols = W.shape
+    r = A.shape[0]
+    out = torch.empty_like(W) if out is None else out
+    _check(lib().lora_merge_weights(rows, cols, r, float(scale), _p(W), _p(A), _p(B), _p(out), _stream(stream)))
+    return out
 
 
 def lora_mlp_fwd(dims: Dims, X, rms_w, weights: Weights, adapters: Adapters, Y, ctx, workspace, stream=None):

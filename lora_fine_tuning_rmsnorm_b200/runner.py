@@ -33,12 +33,12 @@ class Problem:
     """All device buffers of one fwd+bwd step for a Shape."""
 
     def __init__(self, shape: synth.Shape, bits: dict | None = None, seed: int = synth.BASE_SEED,
-                 device="cuda"):
+                 device="cuda", residual: bool = False, norm_grad: bool = False):
         self.shape = s = shape
         self.device = device
         bits = bits if bits is not None else synth.make_inputs_bits(s, seed)
         self.t = {k: bf16_tensor(v, device) for k, v in bits.items()}
-        self.dims = ops.make_dims(s.T, s.d, s.f, s.r, eps=s.eps, scale=s.scale)
+        self.dims = ops.make_dims(s.T, s.d, s.f, s.r, eps=s.eps, scale=s.scale, residual=residual)
         self.weights = ops.make_weights(Wg=self.t["Wg"], Wu=self.t["Wu"], Wd=self.t["Wd"])
         self.adapters = ops.make_adapters(*(self.t[k] for k in ADAPTERS))
         self.Y = torch.empty(s.T, s.d, dtype=torch.bfloat16, device=device)
@@ -46,7 +46,8 @@ class Problem:
         shapes = {"dAg": (s.r, s.d), "dBg": (s.f, s.r), "dAu": (s.r, s.d), "dBu": (s.f, s.r),
                   "dAd": (s.r, s.f), "dBd": (s.d, s.r)}
         self.g = {k: torch.empty(*shapes[k], dtype=torch.float32, device=device) for k in GRADS}
-        self.grads = ops.make_grads(*(self.g[k] for k in GRADS))
+        self.dw = torch.empty(s.d, dtype=torch.float32, device=device) if norm_grad else None
+        self.grads = ops.make_grads(*(self.g[k] for k in GRADS), dw=self.dw)
         self.ctx = ops.alloc_ctx(self.dims, device)
         self.ws = ops.alloc_workspace(self.dims, device)
 
