@@ -118,3 +118,52 @@ def row_slice_bits(bits: dict, rows) -> dict:
         if k in out:
             out[k] = np.ascontiguousarray(out[k][rows])
     return out
+
+
+# ---------------------------------------------------------------- attention Q/K/V projections
+QKV_TENSOR_ORDER = ("X", "w", "Wq", "Wk", "Wv", "Aq", "Bq", "Ak", "Bk", "Av", "Bv", "dQ", "dK", "dV")
+# streams of their own (k offset), so the MLP inputs of the same seed are not reused
+_QKV_STREAM0 = 100
+
+
+@dataclasses.dataclass(frozen=True)
+class QkvShape:
+    """T tokens, hidden d, nq query features, nkv key/value features (grouped-query
+    attention when nkv < nq), LoRA rank r."""
+    T: int
+    d: int
+    nq: int
+    nkv: int
+    r: int
+    alpha: float = 16.0
+    eps: float = 1e-6
+
+    @property
+    def scale(self) -> float:
+        return self.alpha / self.r
+
+
+def qkv_tensor_f64(name: str, s: QkvShape, seed: int = BASE_SEED) -> np.ndarray:
+    """One Q/K/V-projection input in fp64, before bf16 rounding (the same distributions
+    as the MLP's: activations N(0,1), norm weight 1 + N(0,0.1), W N(0,0.02),
+    A U(+-1/sqrt(in)), B N(0,0.01))."""
+    k = _QKV_STREAM0 + QKV_TENSOR_ORDER.index(name)
+    T, d, nq, nkv, r = s.T, s.d, s.nq, s.nkv, s.r
+    n_out = {"q": nq, "k": nkv, "v": nkv}
+    if name == "X":
+        return _normal(k, seed, (T, d), 0.0, 1.0)
+    if name == "w":
+        return _normal(k, seed, (d,), 1.0, 0.1)
+    if name[0] == "W":
+        return _normal(k, seed, (n_out[name[1]], d), 0.0, 0.02)
+    if name[0] == "A":
+        return _uniform(k, seed, (r, d), 1.0 / np.sqrt(d))
+    if name[0] == "B":
+        return _normal(k, seed, (n_out[name[1]], r), 0.0, 0.01)
+    if name[0] == "d":
+        return _normal(k, seed, (T, n_out[name[1].lower()]), 0.0, 1.0)
+    raise KeyError(name)
+
+
+def make_qkv_inputs_bits(s: QkvShape, seed: int = BASE_SEED, names=QKV_TENSOR_ORDER) -> dict:
+    return {n: f32_to_bf16_bits(qkv_tensor_f64(n, s, seed).astype(np.float32)) for n in names}
