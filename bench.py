@@ -398,6 +398,34 @@ def extras(args):
     print(json.dumps(out), flush=True)
 
 
+def qkv(args):
+    """LoRA Q/K/V projections fwd+bwd at the 8B attention shape: one JSON line with
+    tokens/s, algorithmic TFLOP/s and the fraction of the sustained bf16 peak."""
+    import torch
+    from lora_fine_tuning_rmsnorm_b200 import configs
+    from lora_fine_tuning_rmsnorm_b200.runner import QkvProblem
+    torch.cuda.set_device(0)
+    s = configs.QKV_8B if not args.T else configs.QkvShape(T=args.T, d=4096, nq=4096, nkv=1024, r=16)
+    pb = QkvProblem(s)
+    for _ in range(args.warmup):
+        pb.step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        pb.step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = configs.qkv_algorithmic_flops(s)
+    sust = peaks()[2]
+    print(json.dumps({"qkv": True, "workload": f"LoRA Q/K/V projections fwd+bwd, Llama-3-8B attention shape: T={s.T} "
+                                               f"d={s.d} nq={s.nq} nkv={s.nkv} r={s.r} alpha={s.alpha:g}",
+                      "tokens_per_s": s.T / (ms / 1e3), "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                      "frac_of_bf16_sustained": flops / (ms / 1e3) / 1e12 / sust, "steps": args.steps,
+                      "warmup": args.warmup}), flush=True)
+
+
 def sweep(args):
     """Rank / length sweep at d = 4096, f = 14336 (alpha = 16): one JSON line per
     point with tokens/s and the dense-GEMM vs memory-bound phase split."""
@@ -443,6 +471,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (profiling runs)")
     ap.add_argument("--T", type=int, default=None, help="override the token count (profiling on small cases)")
     ap.add_argument("--sweep", action="store_true", help="rank/length sweep, one JSON line per point")
+    ap.add_argument("--qkv", action="store_true", help="LoRA Q/K/V projections fwd+bwd, one JSON line")
     ap.add_argument("--extras", action="store_true",
                     help="residual / norm-weight-gradient step and weight merge, one JSON line")
     args = ap.parse_args()
@@ -458,6 +487,9 @@ def main():
         return
     if args.extras:
         extras(args)
+        return
+    if args.qkv:
+        qkv(args)
         return
     if world > 1:
         import datetime

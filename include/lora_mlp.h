@@ -175,6 +175,75 @@ int lora_rmsnorm_fwd(int64_t T, int32_t d, float eps, const void* X, const void*
 int lora_rmsnorm_bwd(int64_t T, int32_t d, const float* dH, const void* X, const void* w,
                      const float* rstd, void* dX, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * LoRA on the attention Q/K/V projections (the layer's attention half up to
+ * RoPE: "Unsloth — 用手写 Triton kernel 给 HF 微调换心脏", §2.3, RMSNorm kernel then
+ * the Q/K/V projection with the LoRA forward written by hand; §7, LoRA_QKV /
+ * apply_lora_qkv):
+ *   H = RMSNorm(X) (cached rstd);  Q = H Wq^T + s (H Aq^T) Bq^T;  K, V likewise.
+ * Backward from dQ, dK, dV: dX and the six adapter gradients (frozen W and norm
+ * weight).  Same conventions as the MLP calls (asynchronous, caller-owned buffers,
+ * 16-byte aligned pointers, status codes). */
+typedef struct lora_qkv_dims {
+  int64_t T;            /* tokens, 1 <= T < 2^31                                    */
+  int32_t d;            /* hidden size, multiple of 8, 8 <= d <= 65536              */
+  int32_t nq, nkv;      /* Q and K/V output features (grouped-query: nkv < nq),    */
+                        /* multiples of 8                                          */
+  int32_t r;            /* rank, multiple of 8, 8 <= r <= 128                       */
+  float eps;
+  float scale;          /* s = alpha / r                                            */
+} lora_qkv_dims;
+
+/* Wq [nq x d], Wk, Wv [nkv x d] bf16 row-major. */
+typedef struct lora_qkv_weights {
+  const void* Wq;
+  const void* Wk;
+  const void* Wv;
+} lora_qkv_weights;
+
+/* Aq, Ak, Av [r x d]; Bq [nq x r]; Bk, Bv [nkv x r]; bf16 row-major. */
+typedef struct lora_qkv_adapters {
+  const void* Aq;
+  const void* Bq;
+  const void* Ak;
+  const void* Bk;
+  const void* Av;
+  const void* Bv;
+} lora_qkv_adapters;
+
+/* fp32, shapes of the adapters, OVERWRITTEN (fp32 atomics over T). */
+typedef struct lora_qkv_grads {
+  float* dAq;
+  float* dBq;
+  float* dAk;
+  float* dBk;
+  float* dAv;
+  float* dBv;
+} lora_qkv_grads;
+
+/* Saved context: rstd [T] fp32; H [T x d] bf16; P [T x 3rp] bf16 =
+ * s (H Aq^T | H Ak^T | H Av^T), each block rp = r rounded up to 16 wide (zero padded).
+ * Offsets are multiples of 256. */
+typedef struct lora_qkv_ctx_layout {
+  size_t rstd, H, P;
+  size_t total;
+  int32_t rp;
+} lora_qkv_ctx_layout;
+
+int lora_qkv_ctx_layout_get(const lora_qkv_dims* dims, lora_qkv_ctx_layout* out);
+int lora_qkv_workspace_bytes(const lora_qkv_dims* dims, size_t* bytes);
+
+/* Forward: Q [T x nq], K, V [T x nkv] bf16; writes the context. */
+int lora_qkv_fwd(const lora_qkv_dims* dims, const void* X, const void* rms_w, const lora_qkv_weights* W,
+                 const lora_qkv_adapters* A, void* Q, void* K, void* V, void* ctx, void* workspace,
+                 void* stream);
+
+/* Backward: dQ [T x nq], dK, dV [T x nkv] bf16 in; dX [T x d] bf16 and the grads out.
+ * Needs the context of the forward of the same X. */
+int lora_qkv_bwd(const lora_qkv_dims* dims, const void* dQ, const void* dK, const void* dV, const void* X,
+                 const void* rms_w, const lora_qkv_weights* W, const lora_qkv_adapters* A, const void* ctx,
+                 void* dX, const lora_qkv_grads* grads, void* workspace, void* stream);
+
 /* Adapter folded into its frozen weight for export ("Unsloth提速秘诀…", §3.1, "LoRA
  * Update + Weight Merge"; "Unsloth 深度实战", §5.1, the merged 16-bit save):
  *   Wm[o][i] = bf16( W[o][i] + scale * sum_{k<r} B[o][k] A[k][i] )

@@ -4,7 +4,7 @@ The shapes stand in for the pages' fine-tuning workloads: Llama-3-8B / Llama-3.2
 LoRA/QLoRA SFT at sequence 2048 and batch 4 ("Unsloth提速秘诀：Triton内核如何加速反向传播",
 §4.1; "Unsloth 深度实战", §3.2), with alpha = 16 and eps = 1e-6.
 """
-from .synth import Shape
+from .synth import QkvShape, Shape
 
 TINY = Shape(T=64, d=128, f=344, r=8, alpha=16.0)            # batch 2 x seq 32
 LLAMA32_1B = Shape(T=8192, d=2048, f=8192, r=16, alpha=16.0)  # batch 4 x seq 2048
@@ -20,3 +20,15 @@ QBLOCK = 64  # 4-bit blockwise quantisation block size
 def algorithmic_flops(s: Shape) -> float:
     """Dense 12*T*d*f (6 fwd + 6 bwd, frozen W gets no gradient) + LoRA 18*T*r*(d+f)."""
     return 12.0 * s.T * s.d * s.f + 18.0 * s.T * s.r * (s.d + s.f)
+
+
+# attention Q/K/V projections of the same 8B model: 32 query heads and 8 key/value heads
+# of 128 (grouped-query attention), batch 4 x seq 2048
+QKV_8B = QkvShape(T=8192, d=4096, nq=4096, nkv=1024, r=16, alpha=16.0)
+
+
+def qkv_algorithmic_flops(s: QkvShape) -> float:
+    """Dense 4*T*d*N with N = nq + 2 nkv (forward and input gradient; frozen W gets no
+    gradient) + LoRA 2*T*r*(9 d + 3 N) (P, P B^T; Q, the dH term, dA, dB)."""
+    N = s.nq + 2 * s.nkv
+    return 4.0 * s.T * s.d * N + 2.0 * s.T * s.r * (9 * s.d + 3 * N)

@@ -33,7 +33,7 @@ namespace lm {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kMaxStages = 8;
-constexpr int kMaxSegs = 4;
+constexpr int kMaxSegs = 6;
 constexpr int kMaxMaps = 10;
 constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16-column chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;

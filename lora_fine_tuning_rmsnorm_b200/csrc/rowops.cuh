@@ -180,6 +180,25 @@ __global__ void splitk_finalize_kernel(const float* __restrict__ part, int split
   *reinterpret_cast<uint2*>(out + i4) = o;
 }
 
+// The same sum of K-split partials, written into columns [0, cols) of an output with
+// row stride ld_out (a column block of a wider matrix).  cols is a multiple of 4.
+__global__ void splitk_finalize_strided_kernel(const float* __restrict__ part, int splits, long long stride,
+                                               long long rows, int cols, long long ld_out, float scale,
+                                               uint16_t* __restrict__ out) {
+  const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i4 >= rows * cols) return;
+  float4 acc = *reinterpret_cast<const float4*>(part + i4);
+  for (int s = 1; s < splits; ++s) {
+    const float4 v = *reinterpret_cast<const float4*>(part + s * stride + i4);
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  const long long row = i4 / cols, col = i4 - row * cols;
+  uint2 o;
+  o.x = pack_bf16x2(acc.x * scale, acc.y * scale);
+  o.y = pack_bf16x2(acc.z * scale, acc.w * scale);
+  *reinterpret_cast<uint2*>(out + row * ld_out + col) = o;
+}
+
 constexpr int kZeroMax = 7;
 struct ZeroList {
   float* p[kZeroMax];  // NULL entries (n = 0) are skipped

@@ -50,6 +50,27 @@ class CtxLayout(ctypes.Structure):
                [("rp", ctypes.c_int32)]
 
 
+class QkvDims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("nq", ctypes.c_int32), ("nkv", ctypes.c_int32),
+                ("r", ctypes.c_int32), ("eps", ctypes.c_float), ("scale", ctypes.c_float)]
+
+
+class QkvWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Wq", "Wk", "Wv")]
+
+
+class QkvAdapters(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Aq", "Bq", "Ak", "Bk", "Av", "Bv")]
+
+
+class QkvGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dAq", "dBq", "dAk", "dBk", "dAv", "dBv")]
+
+
+class QkvCtxLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("rstd", "H", "P", "total")] + [("rp", ctypes.c_int32)]
+
+
 def header_functions() -> list[str]:
     """Names of the functions include/lora_mlp.h declares."""
     txt = open(HEADER).read()
@@ -80,6 +101,12 @@ def lib() -> ctypes.CDLL:
         "lora_rmsnorm_bwd": [i64, i32, vp, vp, vp, vp, vp, vp],
         "lora_quantize_4bit": [vp, i64, i32, vp, vp, vp, vp],
         "lora_merge_weights": [i64, i64, i32, f32, vp, vp, vp, vp, vp],
+        "lora_qkv_ctx_layout_get": [ctypes.POINTER(QkvDims), ctypes.POINTER(QkvCtxLayout)],
+        "lora_qkv_workspace_bytes": [ctypes.POINTER(QkvDims), ctypes.POINTER(ctypes.c_size_t)],
+        "lora_qkv_fwd": [ctypes.POINTER(QkvDims), vp, vp, ctypes.POINTER(QkvWeights), ctypes.POINTER(QkvAdapters),
+                         vp, vp, vp, vp, vp, vp],
+        "lora_qkv_bwd": [ctypes.POINTER(QkvDims), vp, vp, vp, vp, vp, ctypes.POINTER(QkvWeights),
+                         ctypes.POINTER(QkvAdapters), vp, vp, ctypes.POINTER(QkvGrads), vp, vp],
         "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, i32, vp],
         "lora_lowrank_proj_noalloc": [i64, i32, i32, f32, vp, vp, vp, vp],
         "lora_mlp_timing_enable": [i32],
@@ -237,3 +264,33 @@ def timing_collect() -> dict:
         if n[i]:
             out[lib().lora_mlp_phase_name(i).decode()] = (ms[i], n[i])
     return out
+
+
+# ------------------------------------------------------------------ Q/K/V projections
+def qkv_dims(T, d, nq, nkv, r, eps=1e-6, scale=1.0) -> QkvDims:
+    return QkvDims(T, d, nq, nkv, r, eps, scale)
+
+
+def qkv_ctx_layout(dims: QkvDims) -> QkvCtxLayout:
+    out = QkvCtxLayout()
+    _check(lib().lora_qkv_ctx_layout_get(ctypes.byref(dims), ctypes.byref(out)))
+    return out
+
+
+def qkv_workspace_bytes(dims: QkvDims) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().lora_qkv_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)))
+    return out.value
+
+
+def lora_qkv_fwd(dims: QkvDims, X, rms_w, weights: QkvWeights, adapters: QkvAdapters, Q, K, V, ctx, workspace,
+                 stream=None):
+    _check(lib().lora_qkv_fwd(ctypes.byref(dims), _p(X), _p(rms_w), ctypes.byref(weights), ctypes.byref(adapters),
+                              _p(Q), _p(K), _p(V), _p(ctx), _p(workspace), _stream(stream)))
+
+
+def lora_qkv_bwd(dims: QkvDims, dQ, dK, dV, X, rms_w, weights: QkvWeights, adapters: QkvAdapters, ctx, dX,
+                 grads: QkvGrads, workspace, stream=None):
+    _check(lib().lora_qkv_bwd(ctypes.byref(dims), _p(dQ), _p(dK), _p(dV), _p(X), _p(rms_w), ctypes.byref(weights),
+                              ctypes.byref(adapters), _p(ctx), _p(dX), ctypes.byref(grads), _p(workspace),
+                              _stream(stream)))

@@ -146,3 +146,41 @@ class HostPipeline:
             self.hflat.copy_(b["flat"], non_blocking=True)
         if n_steps is None or i + 2 < n_steps:
             self._load(b)  # inputs of step i + 2 (after this step's compute has read them)
+
+
+QKV_GRADS = ("dAq", "dBq", "dAk", "dBk", "dAv", "dBv")
+
+
+class QkvProblem:
+    """All device buffers of one Q/K/V-projection fwd+bwd step for a QkvShape."""
+
+    def __init__(self, shape: synth.QkvShape, bits: dict | None = None, seed: int = synth.BASE_SEED,
+                 device="cuda"):
+        self.shape = s = shape
+        bits = bits if bits is not None else synth.make_qkv_inputs_bits(s, seed)
+        self.t = {k: bf16_tensor(v, device) for k, v in bits.items()}
+        self.dims = ops.qkv_dims(s.T, s.d, s.nq, s.nkv, s.r, eps=s.eps, scale=s.scale)
+        self.weights = ops.QkvWeights(*(ops._p(self.t[k]) for k in ("Wq", "Wk", "Wv")))
+        self.adapters = ops.QkvAdapters(*(ops._p(self.t[k]) for k in ("Aq", "Bq", "Ak", "Bk", "Av", "Bv")))
+        n = {"q": s.nq, "k": s.nkv, "v": s.nkv}
+        self.out = {k: torch.empty(s.T, n[k.lower()], dtype=torch.bfloat16, device=device) for k in ("Q", "K", "V")}
+        self.dX = torch.empty(s.T, s.d, dtype=torch.bfloat16, device=device)
+        shapes = {"dAq": (s.r, s.d), "dBq": (s.nq, s.r), "dAk": (s.r, s.d), "dBk": (s.nkv, s.r),
+                  "dAv": (s.r, s.d), "dBv": (s.nkv, s.r)}
+        self.g = {k: torch.empty(*shapes[k], dtype=torch.float32, device=device) for k in QKV_GRADS}
+        self.grads = ops.QkvGrads(*(ops._p(self.g[k]) for k in QKV_GRADS))
+        L = ops.qkv_ctx_layout(self.dims)
+        self.ctx = torch.empty(L.total, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(ops.qkv_workspace_bytes(self.dims), dtype=torch.uint8, device=device)
+
+    def forward(self, stream=None):
+        ops.lora_qkv_fwd(self.dims, self.t["X"], self.t["w"], self.weights, self.adapters, self.out["Q"],
+                         self.out["K"], self.out["V"], self.ctx, self.ws, stream)
+
+    def backward(self, stream=None):
+        ops.lora_qkv_bwd(self.dims, self.t["dQ"], self.t["dK"], self.t["dV"], self.t["X"], self.t["w"],
+                         self.weights, self.adapters, self.ctx, self.dX, self.grads, self.ws, stream)
+
+    def step(self, stream=None):
+        self.forward(stream)
+        self.backward(stream)
