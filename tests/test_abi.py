@@ -95,3 +95,51 @@ def test_phase_names(L):
     names = [L.lora_mlp_phase_name(i).decode() for i in range(ops.NUM_PHASES)]
     assert "gemm_gate_up_swiglu" in names and "rmsnorm_fwd" in names
     assert L.lora_mlp_phase_name(99) == b"invalid"
+
+
+def test_residual_flag_and_dw_pointer_checked(L):
+    dims = ops.make_dims(64, 128, 344, 8)
+    dims.residual = 2
+    out = ctypes.c_size_t()
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -1
+    dims.residual = 1
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == 0
+    good = ctypes.c_void_p(0x1000)
+    w = ops.Weights(*([0x1000] * 3))
+    a = ops.Adapters(*([0x1000] * 6))
+    g = ops.Grads(*([0x1000] * 6 + [0x1004]))   # dw given but not 16-byte aligned
+    rc = L.lora_mlp_bwd(ctypes.byref(dims), good, good, good, ctypes.byref(w), ctypes.byref(a), good, good,
+                        ctypes.byref(g), good, None)
+    assert rc == -2
+
+
+def test_merge_weights_argument_checks(L):
+    good = ctypes.c_void_p(0x1000)
+    assert L.lora_merge_weights(0, 64, 8, 1.0, good, good, good, good, None) == -1          # rows
+    assert L.lora_merge_weights(16, 60, 8, 1.0, good, good, good, good, None) == -1         # cols % 8
+    assert L.lora_merge_weights(16, 64, 300, 1.0, good, good, good, good, None) == -3       # r > 256
+    assert L.lora_merge_weights(16, 64, 8, float("inf"), good, good, good, good, None) == -1
+    assert L.lora_merge_weights(16, 64, 8, 1.0, ctypes.c_void_p(0x1008), good, good, good, None) == -2
+    assert L.lora_merge_weights(16, 64, 8, 1.0, good, good, ctypes.c_void_p(0x1001), good, None) == -2
+
+
+def test_qkv_layout_and_argument_checks(L):
+    dims = ops.qkv_dims(8192, 4096, 4096, 1024, 16)
+    lay = ops.qkv_ctx_layout(dims)
+    assert lay.rp == 16
+    for off in (lay.rstd, lay.H, lay.P):
+        assert off % 256 == 0
+    assert lay.total >= 8192 * 4 + 8192 * 4096 * 2 + 8192 * 48 * 2
+    assert ops.qkv_workspace_bytes(dims) >= 8192 * 4096 * 4 + 8192 * 48 * 2
+    out = ctypes.c_size_t()
+    for bad, code in (((64, 128, 128, 60, 8), -2), ((64, 128, 0, 64, 8), -1), ((64, 128, 128, 64, 136), -3),
+                      ((0, 128, 128, 64, 8), -1)):
+        assert L.lora_qkv_workspace_bytes(ctypes.byref(ops.qkv_dims(*bad)), ctypes.byref(out)) == code, bad
+    w, a, g = ops.QkvWeights(), ops.QkvAdapters(), ops.QkvGrads()
+    good = ctypes.c_void_p(0x1000)
+    rc = L.lora_qkv_fwd(ctypes.byref(ops.qkv_dims(64, 128, 128, 64, 8)), good, good, ctypes.byref(w), ctypes.byref(a),
+                        good, good, good, good, good, None)
+    assert rc == -1 and b"NULL" in L.lora_mlp_last_error()
+    rc = L.lora_qkv_bwd(ctypes.byref(ops.qkv_dims(64, 128, 128, 64, 8)), good, good, good, good, good,
+                        ctypes.byref(w), ctypes.byref(a), good, good, ctypes.byref(g), good, None)
+    assert rc == -1
