@@ -47,3 +47,19 @@ def test_distributions():
 def test_flops_formula():
     assert abs(configs.algorithmic_flops(configs.LLAMA3_8B) - 5.8159e12) / 5.8159e12 < 1e-4
     assert abs(configs.algorithmic_flops(configs.LLAMA32_1B) - 1.6734e12) / 1.6734e12 < 1e-4
+
+
+def test_qkv_inputs_shapes_streams_and_determinism():
+    s = synth.QkvShape(T=33, d=64, nq=64, nkv=16, r=8)
+    a = synth.make_qkv_inputs_bits(s)
+    b = synth.make_qkv_inputs_bits(s)
+    shapes = {"X": (33, 64), "w": (64,), "Wq": (64, 64), "Wk": (16, 64), "Wv": (16, 64), "Aq": (8, 64),
+              "Bq": (64, 8), "Ak": (8, 64), "Bk": (16, 8), "Av": (8, 64), "Bv": (16, 8), "dQ": (33, 64),
+              "dK": (33, 16), "dV": (33, 16)}
+    for k, sh in shapes.items():
+        assert a[k].shape == sh and a[k].dtype == np.uint16, k
+        assert np.array_equal(a[k], b[k]), k
+    # streams of their own: not the MLP's X for the same seed and size
+    mlp = synth.make_inputs_bits(synth.Shape(T=33, d=64, f=128, r=8), names=("X",))
+    assert not np.array_equal(mlp["X"], a["X"])
+    assert abs(s.scale - 2.0) < 1e-12
