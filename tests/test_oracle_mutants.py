@@ -76,3 +76,61 @@ def test_finite_difference_pin_catches_mutant(monkeypatch, name):
 def test_unmutated_oracle_passes_same_check():
     s, inp = tiny_inputs(seed=31)
     assert max(fd_errors(inp, s, eps=0.1).values()) < 1e-7
+
+
+# ---------------------------------------------------------------- Q/K/V projections
+from oracle import lora_qkv_ref as qref  # noqa: E402
+from tests.test_oracle_qkv_pins import loss as qkv_loss, run as qkv_run, tiny as qkv_tiny  # noqa: E402
+
+QKV_ORIG_BWD = qref.backward
+
+
+def _qkv_bwd_drop_lora_k(fw, dQ, dK, dV, X, w, Wq, Wk, Wv, Aq, Bq, Ak, Bk, Av, Bv, s):
+    out = QKV_ORIG_BWD(fw, dQ, dK, dV, X, w, Wq, Wk, Wv, Aq, Bq, Ak, Bk, Av, Bv, s)
+    dH = out["dH"] - s * ((dK @ Bk) @ Ak)          # the K adapter's term missing from dH
+    out["dX"] = qref.rmsnorm_bwd(dH, X, w, fw["rstd"])
+    return out
+
+
+def _qkv_bwd_dBv_no_scale(fw, dQ, dK, dV, X, w, Wq, Wk, Wv, Aq, Bq, Ak, Bk, Av, Bv, s):
+    out = QKV_ORIG_BWD(fw, dQ, dK, dV, X, w, Wq, Wk, Wv, Aq, Bq, Ak, Bk, Av, Bv, s)
+    out["dBv"] = dV.T @ fw["Pv"]                    # dropped scaling
+    return out
+
+
+def _qkv_bwd_dAq_wrong_operand(fw, dQ, dK, dV, X, w, Wq, Wk, Wv, Aq, Bq, Ak, Bk, Av, Bv, s):
+    out = QKV_ORIG_BWD(fw, dQ, dK, dV, X, w, Wq, Wk, Wv, Aq, Bq, Ak, Bk, Av, Bv, s)
+    out["dAq"] = s * ((dQ @ Bq).T @ X)              # raw X instead of the normalised H
+    return out
+
+
+QKV_MUTANTS = {"drop_lora_k_in_dH": _qkv_bwd_drop_lora_k, "dBv_missing_scale": _qkv_bwd_dBv_no_scale,
+               "dAq_uses_X_not_H": _qkv_bwd_dAq_wrong_operand}
+
+
+def _qkv_fd_max_err(inp, s):
+    _, bw = qkv_run(inp, s)
+    rng = np.random.default_rng(3)
+    h = 1e-5
+    worst = 0.0
+    for name, g in (("X", "dX"), ("Aq", "dAq"), ("Bq", "dBq"), ("Ak", "dAk"), ("Bk", "dBk"), ("Av", "dAv"),
+                    ("Bv", "dBv")):
+        V = rng.standard_normal(inp[name].shape)
+        p = dict(inp); p[name] = inp[name] + h * V
+        m = dict(inp); m[name] = inp[name] - h * V
+        fd = (qkv_loss(p, s) - qkv_loss(m, s)) / (2 * h)
+        an = float(np.sum(bw[g] * V))
+        worst = max(worst, abs(fd - an) / max(abs(fd), 1e-300))
+    return worst
+
+
+@pytest.mark.parametrize("name", sorted(QKV_MUTANTS))
+def test_qkv_finite_difference_pin_catches_mutant(monkeypatch, name):
+    monkeypatch.setattr(qref, "backward", QKV_MUTANTS[name])
+    s, inp = qkv_tiny(seed=44)
+    assert _qkv_fd_max_err(inp, s) > 1e-4, name
+
+
+def test_qkv_unmutated_oracle_passes_same_check():
+    s, inp = qkv_tiny(seed=44)
+    assert _qkv_fd_max_err(inp, s) < 1e-7
