@@ -51,7 +51,8 @@ enum lora_status {
   LORA_ERR_ALIGNMENT = -2,   /* pointer not 16-B aligned; d, f, r not multiples of 8 */
   LORA_ERR_UNSUPPORTED = -3, /* size outside the supported range (see each call)     */
   LORA_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (message has text)  */
-  LORA_ERR_TIMEOUT = -5      /* a bounded device-side wait gave up (debug mode only) */
+  LORA_ERR_TIMEOUT = -5      /* a bounded device-side wait gave up (reported by the   */
+                             /* call itself in debug mode, else by lora_mlp_status)   */
 };
 
 enum lora_wfmt {
@@ -144,7 +145,8 @@ int lora_mlp_ctx_layout_get(const lora_mlp_dims* dims, lora_mlp_ctx_layout* out)
 
 /* Workspace bytes needed by lora_mlp_fwd / lora_mlp_bwd (one buffer serves both;
  * it holds the backward's dH fp32 [T x d], dG, dU bf16 [T x f], the rank-r
- * projections and a device status word).  Contents need not be initialised. */
+ * projections and, at offset 0, a device status word).  Contents need not be
+ * initialised. */
 int lora_mlp_workspace_bytes(const lora_mlp_dims* dims, size_t* bytes);
 
 /* Forward.  X [T x d] bf16, rms_w [d] bf16 -> Y [T x d] bf16, and the saved context
@@ -271,8 +273,27 @@ int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float*
  * flags: LORA_GEMM_CTA_PAIR runs 256-row tiles on pairs of SMs (tcgen05
  * cta_group::2; needs a_mn = 0), otherwise one 128-row tile per SM. */
 #define LORA_GEMM_CTA_PAIR 1
+/* Test of the failure path only: the kernel's copy warp issues no loads and arms no
+ * barrier, so the MMA's first bounded wait runs out after LORA_MLP_WAIT_LIMIT_MS; the
+ * kernel then records the timeout, frees its tensor memory and returns (C is left
+ * unwritten).  Not combinable with LORA_GEMM_CTA_PAIR. */
+#define LORA_GEMM_TEST_NO_LOADS 2
 int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B,
                    int32_t b_mn, float* C, int32_t flags, void* stream);
+
+/* Bounded-wait status of the most recent call that used `workspace` (any workspace
+ * of this library: its status word sits at offset 0), or, with workspace = NULL, of
+ * the most recent lora_gemm_bf16 / lora_lowrank_proj_noalloc call in the current
+ * CUDA context.  Every device wait in the kernels has a time limit
+ * (LORA_MLP_WAIT_LIMIT_MS in the environment, default 5000 ms); a wait that runs out
+ * makes its kernel record a code in the status word, stop its other roles, wait for
+ * its own copies and tensor-core operations in flight, free its tensor memory and
+ * return, leaving the outputs incomplete.  Each call clears its status word when it
+ * is enqueued, so check after every call whose result matters.
+ * Synchronises `stream`, then returns LORA_OK, or LORA_ERR_TIMEOUT with the code in
+ * *code (may be NULL) and in lora_mlp_last_error().  With LORA_MLP_DEBUG=1 every call
+ * does this check itself before it returns. */
+int lora_mlp_status(const void* workspace, int32_t* code, void* stream);
 
 /* Allocation-free rank-r projection.  The pages have no counterpart to this entry
  * point; it exists for callers that cannot allocate device memory themselves, such
@@ -285,9 +306,13 @@ int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn,
  * The K-split fp32 partial sums go to a fixed 16 MiB array inside the library
  * (4 Mi floats, held on every GPU that loads the library until the process exits);
  * sizes with splits * T * rp above that are rejected with LORA_ERR_UNSUPPORTED.
- * No cudaMalloc/cudaFree or other allocation is made.  The first call on each
- * device looks up that array's device address (cudaGetSymbolAddress, with the
- * device current) and caches it; make that first call before any stream capture.
+ * No cudaMalloc/cudaFree or other allocation is made.  The array's device address
+ * belongs to one CUDA context, so the first call in each context (the one current
+ * on the calling thread: the device's primary context, or a context the caller
+ * created) looks it up with cudaGetSymbolAddress and caches it under that context's
+ * unique id; make that first call before any stream capture.  The bounded-wait
+ * status of the call is kept in a library word of the same context (read it with
+ * lora_mlp_status(NULL, ...); debug mode reports it from the call itself).
  * All calls share the array: calls that can overlap on the GPU (different streams,
  * or several host threads) race on it and must be serialised by the caller.  Every
  * partial-sum element is rewritten by each call, so nothing has to be cleared. */
@@ -298,7 +323,7 @@ int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, cons
  * is bracketed by CUDA events on the caller's stream.  lora_mlp_timing_collect()
  * synchronises those events and returns, per phase id, the summed milliseconds and
  * the number of launches since the previous collect (arrays of LORA_NUM_PHASES). */
-#define LORA_NUM_PHASES 17
+#define LORA_NUM_PHASES 20
 int lora_mlp_timing_enable(int32_t on);
 int lora_mlp_timing_collect(double* ms, int64_t* launches);
 const char* lora_mlp_phase_name(int32_t phase);

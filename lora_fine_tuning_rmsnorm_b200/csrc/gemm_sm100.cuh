@@ -118,6 +118,8 @@ struct GemmArgs {
   unsigned long long limit_ns;
   const float* codebook;  // 4-bit code values (16 fp32)
   uint32_t cr_bytes;      // 4-bit: bytes of one code-ring entry
+  int test_no_loads;      // test of the bounded waits: the producer copies nothing and arms no
+                          // barrier, so the MMA's first wait runs out (single-CTA tiles only)
 };
 
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
@@ -225,6 +227,13 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         if (!mbar_wait(empty, phase ^ 1, wc, kDevTimeoutProducer)) {
           ok = false;
           break;
+        }
+        if (p.test_no_loads) {  // nothing issued, nothing armed: no copy can be in flight
+          if (++stage == p.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          continue;
         }
         if (stage_tx) mbar_expect_tx(full, stage_tx);
         const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);

@@ -158,10 +158,11 @@ const char* kPhaseNames[LORA_NUM_PHASES] = {
     "rmsnorm_fwd", "proj_P_gate_up", "gemm_gate_up_swiglu", "proj_P_down", "gemm_down",
     "proj_Q_down", "gemm_dact_swiglu_bwd", "proj_Q_gate_up", "gemm_dH", "rmsnorm_bwd",
     "zero_grads", "reduce_dA_gate_up", "reduce_dB_gate_up", "reduce_dB_down", "reduce_dA_down",
-    "norm_weight_grad", "other"};
+    "norm_weight_grad", "other", "qkv_gemm", "qkv_gemm_dH", "qkv_lowrank"};
 enum Phase {
   PH_RMS_FWD = 0, PH_P_GU, PH_GATEUP, PH_P_D, PH_DOWN, PH_Q_D, PH_DACT, PH_Q_GU, PH_DH,
-  PH_RMS_BWD, PH_ZERO, PH_RED_DA_GU, PH_RED_DB_GU, PH_RED_DB_D, PH_RED_DA_D, PH_DW, PH_OTHER
+  PH_RMS_BWD, PH_ZERO, PH_RED_DA_GU, PH_RED_DB_GU, PH_RED_DB_D, PH_RED_DA_D, PH_DW, PH_OTHER,
+  PH_QKV_GEMM, PH_QKV_DH, PH_QKV_LOWRANK
 };
 
 struct Timing {
@@ -427,8 +428,10 @@ int check_ptrs(std::initializer_list<const void*> ps) {
   return LORA_OK;
 }
 
+// Every call clears its status word first (in every mode), so the word reports the
+// bounded waits of the most recent call that used it (lora_mlp_status reads it).
 int begin_call(int* status, cudaStream_t st) {
-  if (debug_mode() && status) CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  if (status) CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
   return LORA_OK;
 }
 
@@ -613,33 +616,79 @@ int launch_proj_into(GemmArgs& a, long long T, long long K, int rp, float* part,
 
 }  // namespace
 
-// ---------------------------------------------------- allocation-free variant
+// ------------------------------------------------- library-owned device memory
 // Scratch for lora_lowrank_proj_noalloc: the K-split fp32 partial sums live in a
 // file-scope device array instead of caller memory.  Every GPU that loads this
 // library holds it until the process exits.
 constexpr size_t kNoAllocScratchFloats = size_t(4) << 20;  // 16 MiB
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+// Bounded-wait status word of the calls that take no workspace (lora_gemm_bf16,
+// lora_lowrank_proj_noalloc); the calls with a workspace keep theirs at its offset 0.
+static __device__ __align__(256) int g_lib_status;
 
-// Host code may not use &g_noalloc_scratch as a device address (in host code the
-// name denotes a host-side stand-in), so the device address is looked up once per
-// device, with that device current, and cached.
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kMaxDevices] = {};
+// In host code the names above denote host-side stand-ins, not device addresses.
+// Their device addresses belong to one CUDA context (the module is loaded per
+// context), so they are looked up with cudaGetSymbolAddress, with the caller's context
+// current, and cached under that context's unique id (cuCtxGetId: unlike the CUcontext
+// handle, an id is never reused within the process, so a context destroyed by
+// cudaDeviceReset and its successor get different entries).
+struct LibSyms {
+  unsigned long long ctx_id;
+  float* scratch;
+  int* status;
+};
+std::mutex g_syms_mu;
+std::vector<LibSyms> g_syms;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
 
-int noalloc_scratch(float** out) {
-  int dev = 0;
-  CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(LORA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || !ptr)
-      return fail(LORA_ERR_CUDA, "cudaGetSymbolAddress(no-alloc scratch) failed: %s", cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+int resolve_ctx_fns() {
+  if (g_ctx_current && g_ctx_id) return LORA_OK;
+  void* f1 = nullptr;
+  void* f2 = nullptr;
+  cudaDriverEntryPointQueryResult q1, q2;
+  cudaError_t e1 = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1);
+  cudaError_t e2 = cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2);
+  if (e1 != cudaSuccess || e2 != cudaSuccess || q1 != cudaDriverEntryPointSuccess ||
+      q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+    return fail(LORA_ERR_CUDA, "cannot resolve cuCtxGetCurrent / cuCtxGetId");
+  g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+  g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+  return LORA_OK;
+}
+
+int lib_syms(LibSyms* out) {
+  std::lock_guard<std::mutex> lk(g_syms_mu);
+  TRY(resolve_ctx_fns());
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return fail(LORA_ERR_CUDA, "cuCtxGetCurrent failed");
+  if (!ctx) {
+    // no context current yet: the runtime makes the device's primary context current
+    // on its first use, which this lookup is
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_lib_status));
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return fail(LORA_ERR_CUDA, "no current CUDA context");
   }
-  *out = g_noalloc_ptr[dev];
+  unsigned long long id = 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return fail(LORA_ERR_CUDA, "cuCtxGetId failed");
+  for (const LibSyms& e : g_syms)
+    if (e.ctx_id == id) {
+      *out = e;
+      return LORA_OK;
+    }
+  LibSyms e{id, nullptr, nullptr};
+  void* p = nullptr;
+  cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (err != cudaSuccess || !p)
+    return fail(LORA_ERR_CUDA, "cudaGetSymbolAddress(no-alloc scratch) failed: %s", cudaGetErrorString(err));
+  e.scratch = static_cast<float*>(p);
+  err = cudaGetSymbolAddress(&p, g_lib_status);
+  if (err != cudaSuccess || !p)
+    return fail(LORA_ERR_CUDA, "cudaGetSymbolAddress(status word) failed: %s", cudaGetErrorString(err));
+  e.status = static_cast<int*>(p);
+  if (g_syms.size() >= 64) g_syms.erase(g_syms.begin());  // contexts long gone
+  g_syms.push_back(e);
+  *out = e;
   return LORA_OK;
 }
 
@@ -755,8 +804,14 @@ int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn,
     return fail(LORA_ERR_INVALID_ARG, "bad M/N/K");
   if (M % 8 || N % 8 || K % 8) return fail(LORA_ERR_ALIGNMENT, "M, N, K must be multiples of 8");
   TRY(check_ptrs({A, B, C}));
+  if (flags & ~(LORA_GEMM_CTA_PAIR | LORA_GEMM_TEST_NO_LOADS)) return fail(LORA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if ((flags & LORA_GEMM_TEST_NO_LOADS) && (flags & LORA_GEMM_CTA_PAIR))
+    return fail(LORA_ERR_INVALID_ARG, "LORA_GEMM_TEST_NO_LOADS is for single-CTA tiles only");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  GemmArgs a = new_args(nullptr);
+  LibSyms ls;
+  TRY(lib_syms(&ls));
+  GemmArgs a = new_args(ls.status);
+  a.test_no_loads = (flags & LORA_GEMM_TEST_NO_LOADS) ? 1 : 0;
   const int pair = (flags & LORA_GEMM_CTA_PAIR) && !a_mn ? 2 : 1;
   int bn = b_mn ? (N >= 256 ? 256 : round_up(static_cast<int>(N), 64))
                 : (N >= 256 ? 256 : round_up(static_cast<int>(N), 16));
@@ -778,14 +833,38 @@ int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn,
   a.tiles_n = static_cast<int>((N + bn - 1) / bn);
   a.out[0] = C;
   a.ld_out = N;
+  TRY(begin_call(a.status, st));
   if (pair == 2) {
-    if (b_mn) return launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_OTHER);
-    return launch_gemm<0, 0, 1, EPI_F32, 2>(a, st, PH_OTHER);
+    if (b_mn) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_OTHER)));
+    else TRY((launch_gemm<0, 0, 1, EPI_F32, 2>(a, st, PH_OTHER)));
+  } else if (!a_mn && !b_mn) {
+    TRY((launch_gemm<0, 0, 1, EPI_F32>(a, st, PH_OTHER)));
+  } else if (!a_mn && b_mn) {
+    TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_OTHER)));
+  } else if (a_mn && !b_mn) {
+    TRY((launch_gemm<1, 0, 1, EPI_F32>(a, st, PH_OTHER)));
+  } else {
+    TRY((launch_gemm<1, 1, 1, EPI_F32>(a, st, PH_OTHER)));
   }
-  if (!a_mn && !b_mn) return launch_gemm<0, 0, 1, EPI_F32>(a, st, PH_OTHER);
-  if (!a_mn && b_mn) return launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_OTHER);
-  if (a_mn && !b_mn) return launch_gemm<1, 0, 1, EPI_F32>(a, st, PH_OTHER);
-  return launch_gemm<1, 1, 1, EPI_F32>(a, st, PH_OTHER);
+  return end_call(a.status, st);
+}
+
+int lora_mlp_status(const void* workspace, int32_t* code, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int* word = static_cast<const int*>(workspace);
+  if (!word) {
+    LibSyms ls;
+    TRY(lib_syms(&ls));
+    word = ls.status;
+  } else if (!aligned16(workspace)) {
+    return fail(LORA_ERR_ALIGNMENT, "workspace %p is not 16-byte aligned", workspace);
+  }
+  CUDA_TRY(cudaStreamSynchronize(st));
+  int v = 0;
+  CUDA_TRY(cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code) *code = v;
+  if (v) return fail(LORA_ERR_TIMEOUT, "device-side bounded wait gave up (code 0x%x)", v);
+  return LORA_OK;
 }
 
 int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const lora_mlp_weights* W,
@@ -1198,18 +1277,21 @@ int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, cons
     return fail(LORA_ERR_UNSUPPORTED,
                 "T x rp x splits = %lld x %d x %d fp32 partial sums exceed the %zu-float no-alloc scratch",
                 (long long)T, rp, splits, kNoAllocScratchFloats);
-  float* part = nullptr;
-  TRY(noalloc_scratch(&part));
+  LibSyms ls;
+  TRY(lib_syms(&ls));
+  float* part = ls.scratch;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Every partial-sum element is overwritten by the split GEMM (all T rows and rp
   // columns of each split), so the scratch needs no clearing between calls.
-  GemmArgs a = new_args(nullptr);
+  GemmArgs a = new_args(ls.status);
   TRY(map_k(&a.maps[0], X, T, K, K, 128));
   TRY(map_k(&a.maps[1], A, r, K, K, rp));
   set_seg(a, 0, 0, 0, 1, 0, -1, 0, K);
   a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
   a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
-  return launch_proj<0, 1>(a, T, K, rp, part, P, scale, st, PH_OTHER);
+  TRY(begin_call(a.status, st));
+  TRY((launch_proj<0, 1>(a, T, K, rp, part, P, scale, st, PH_OTHER)));
+  return end_call(a.status, st);
 }
 
 
@@ -1260,7 +1342,7 @@ int lora_qkv_fwd(const lora_qkv_dims* D, const void* X, const void* rms_w, const
     a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
     a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
     TRY((launch_proj_into<0>(a, T, d, rp, part, P + static_cast<size_t>(x) * rp * 2, 3LL * rp, D->scale, st,
-                             PH_OTHER)));
+                             PH_QKV_LOWRANK)));
   }
   // Out_x = H W_x^T + P_x B_x^T: the LoRA term as a K = rp extension of the dense GEMM
   for (int x = 0; x < 3; ++x) {
@@ -1279,8 +1361,8 @@ int lora_qkv_fwd(const lora_qkv_dims* D, const void* X, const void* rms_w, const
     a.out[0] = Ox[x]; a.ld_out = nx[x];
     a.stream_out = 1;
     set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_OTHER)));
-    else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_OTHER)));
+    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_QKV_GEMM)));
+    else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_QKV_GEMM)));
   }
   return end_call(status, st);
 }
@@ -1322,7 +1404,7 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     a.M = static_cast<int>(T); a.N = rp; a.bn = qbn;
     a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
     TRY((launch_proj_into<1>(a, T, nx[x], rp, part, Q + static_cast<size_t>(x) * rp * 2, 3LL * rp, D->scale, st,
-                             PH_OTHER)));
+                             PH_QKV_LOWRANK)));
   }
   // dH = dQ Wq + dK Wk + dV Wv + [Q_q | Q_k | Q_v] [Aq; Ak; Av]   (fp32; six K segments)
   {
@@ -1348,8 +1430,8 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
     set_band(a, 4);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_OTHER)));
-    else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_OTHER)));
+    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_QKV_DH)));
+    else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_QKV_DH)));
   }
   TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));
   {
@@ -1375,7 +1457,7 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     a.rng[0] = OutRange{dAx[x], 0, 1, d};
     a.nrng = 1;
     choose_splits(a, T);
-    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_OTHER)));
+    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_QKV_LOWRANK)));
   }
   // dB_x = dZ_x^T P_x  ([n_x x r])
   for (int x = 0; x < 3; ++x) {
@@ -1389,7 +1471,7 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     a.rng[0] = OutRange{dBx[x], 0, 0, r};
     a.nrng = 1;
     choose_splits(a, T);
-    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_OTHER)));
+    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_QKV_LOWRANK)));
   }
   return end_call(status, st);
 }

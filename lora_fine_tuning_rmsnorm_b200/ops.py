@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "lora_mlp.h")
 LORA_OK = 0
 ERRORS = {-1: "INVALID_ARG", -2: "ALIGNMENT", -3: "UNSUPPORTED", -4: "CUDA", -5: "TIMEOUT"}
 WFMT_BF16, WFMT_4BIT = 0, 1
-NUM_PHASES = 17
+NUM_PHASES = 20
 
 
 class LoraError(RuntimeError):
@@ -109,6 +109,7 @@ def lib() -> ctypes.CDLL:
                          ctypes.POINTER(QkvAdapters), vp, vp, ctypes.POINTER(QkvGrads), vp, vp],
         "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, i32, vp],
         "lora_lowrank_proj_noalloc": [i64, i32, i32, f32, vp, vp, vp, vp],
+        "lora_mlp_status": [vp, ctypes.POINTER(ctypes.c_int32), vp],
         "lora_mlp_timing_enable": [i32],
         "lora_mlp_timing_collect": [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
     }
@@ -235,13 +236,26 @@ def lora_quantize_4bit(W, codebook, codes, absmax, block=64, stream=None):
 
 
 GEMM_CTA_PAIR = 1
+GEMM_TEST_NO_LOADS = 2
 
 
-def lora_gemm_bf16(A, a_mn, B, b_mn, C, pair=False, stream=None):
+def lora_gemm_bf16(A, a_mn, B, b_mn, C, pair=False, stream=None, test_no_loads=False):
+    """C = A' B'^T (see lora_gemm_bf16 in the header).  test_no_loads exercises the
+    bounded-wait failure path: nothing is copied, the kernel's waits run out."""
     M, N = C.shape
     K = A.shape[0] if a_mn else A.shape[1]
-    _check(lib().lora_gemm_bf16(M, N, K, _p(A), int(a_mn), _p(B), int(b_mn), _p(C),
-                                GEMM_CTA_PAIR if pair else 0, _stream(stream)))
+    flags = (GEMM_CTA_PAIR if pair else 0) | (GEMM_TEST_NO_LOADS if test_no_loads else 0)
+    _check(lib().lora_gemm_bf16(M, N, K, _p(A), int(a_mn), _p(B), int(b_mn), _p(C), flags, _stream(stream)))
+
+
+def status(workspace=None, stream=None) -> int:
+    """Bounded-wait status code of the last call that used `workspace` (None: the last
+    workspace-less call in this context); 0 = every wait completed.  Synchronises."""
+    code = ctypes.c_int32(0)
+    rc = lib().lora_mlp_status(_p(workspace), ctypes.byref(code), _stream(stream))
+    if rc not in (LORA_OK, -5):
+        _check(rc)
+    return code.value
 
 
 def lora_lowrank_proj_noalloc(X, A, P, scale, stream=None):

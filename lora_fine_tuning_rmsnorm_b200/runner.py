@@ -12,16 +12,6 @@ ADAPTERS = ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")
 GRADS = ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")
 
 
-def load_codebook() -> list:
-    """The 16-entry 4-bit codebook written by tests/golden/make_codebook.py."""
-    import json
-    import os
-    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "tests", "golden",
-                        "codebook16.json")
-    with open(path) as fh:
-        return [float.fromhex(h) for h in json.load(fh)["codebook_f32_hex"]]
-
-
 def bf16_tensor(bits: np.ndarray, device="cuda", pin=False) -> torch.Tensor:
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
     if device == "cpu":

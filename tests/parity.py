@@ -33,3 +33,12 @@ def assert_close(name, out, ref, rel_fro=REL_FRO, max_rel=MAX_REL):
 def to_np(t):
     import torch
     return t.detach().float().cpu().numpy().astype(np.float64) if t.dtype != torch.float64 else t.cpu().numpy()
+
+
+def load_codebook() -> list:
+    """The 16-entry 4-bit codebook written by tests/golden/make_codebook.py (an input of
+    the 4-bit kernels, computed once by the oracle)."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "codebook16.json")) as fh:
+        return [float.fromhex(h) for h in json.load(fh)["codebook_f32_hex"]]

@@ -143,3 +143,12 @@ def test_qkv_layout_and_argument_checks(L):
     rc = L.lora_qkv_bwd(ctypes.byref(ops.qkv_dims(64, 128, 128, 64, 8)), good, good, good, good, good,
                         ctypes.byref(w), ctypes.byref(a), good, good, ctypes.byref(g), good, None)
     assert rc == -1
+
+
+def test_gemm_flags_and_status_argument_checks(L):
+    good = ctypes.c_void_p(0x1000)
+    assert L.lora_gemm_bf16(64, 64, 64, good, 0, good, 0, good, 4, None) == -1        # unknown flag
+    assert L.lora_gemm_bf16(64, 64, 64, good, 0, good, 0, good, 3, None) == -1        # test flag + pair
+    assert b"single-CTA" in L.lora_mlp_last_error()
+    code = ctypes.c_int32(0)
+    assert L.lora_mlp_status(ctypes.c_void_p(0x1004), ctypes.byref(code), None) == -2  # misaligned workspace

@@ -6,10 +6,10 @@ import pytest
 import torch
 
 from lora_fine_tuning_rmsnorm_b200 import configs, ops, synth
-from lora_fine_tuning_rmsnorm_b200.runner import GRADS, Problem, load_codebook
+from lora_fine_tuning_rmsnorm_b200.runner import GRADS, Problem
 from oracle import lora_mlp_ref as ref
 from oracle import quant4_ref as q4
-from tests.parity import assert_close, to_np
+from tests.parity import assert_close, load_codebook, to_np
 
 pytestmark = pytest.mark.gpu
 

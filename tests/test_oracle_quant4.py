@@ -112,3 +112,11 @@ def test_golden_codebook_file_matches_oracle():
         j = json.load(fh)
     got = np.array([float.fromhex(h) for h in j["codebook_f32_hex"]], dtype=np.float64)
     np.testing.assert_array_equal(got, q4.codebook16().astype(np.float64))
+
+
+def test_stored_codebook_is_the_oracles():
+    """tests/golden/codebook16.json (the 4-bit kernels' codebook input) holds exactly the
+    oracle's fp32 codebook, as written by tests/golden/make_codebook.py."""
+    from tests.parity import load_codebook
+    np.testing.assert_array_equal(np.asarray(load_codebook(), dtype=np.float64),
+                                  q4.codebook16().astype(np.float64))
