@@ -167,3 +167,107 @@ def qkv_tensor_f64(name: str, s: QkvShape, seed: int = BASE_SEED) -> np.ndarray:
 
 def make_qkv_inputs_bits(s: QkvShape, seed: int = BASE_SEED, names=QKV_TENSOR_ORDER) -> dict:
     return {n: f32_to_bf16_bits(qkv_tensor_f64(n, s, seed).astype(np.float32)) for n in names}
+
+
+# ---------------------------------------------------------------- attention output projection o_proj
+O_TENSOR_ORDER = ("X", "Wo", "Ao", "Bo", "dY")
+_O_STREAM0 = 200
+
+
+@dataclasses.dataclass(frozen=True)
+class OShape:
+    """T tokens, n_in input features (the attention output, heads x head dim), n_out
+    output features (the hidden size), LoRA rank r."""
+    T: int
+    n_in: int
+    n_out: int
+    r: int
+    alpha: float = 16.0
+
+    @property
+    def scale(self) -> float:
+        return self.alpha / self.r
+
+
+def o_tensor_f64(name: str, s: OShape, seed: int = BASE_SEED) -> np.ndarray:
+    """One o_proj input in fp64 (the MLP's distributions: activations and upstream
+    gradients N(0,1), W N(0,0.02), A U(+-1/sqrt(in)), B N(0,0.01))."""
+    k = _O_STREAM0 + O_TENSOR_ORDER.index(name)
+    if name == "X":
+        return _normal(k, seed, (s.T, s.n_in), 0.0, 1.0)
+    if name == "Wo":
+        return _normal(k, seed, (s.n_out, s.n_in), 0.0, 0.02)
+    if name == "Ao":
+        return _uniform(k, seed, (s.r, s.n_in), 1.0 / np.sqrt(s.n_in))
+    if name == "Bo":
+        return _normal(k, seed, (s.n_out, s.r), 0.0, 0.01)
+    if name == "dY":
+        return _normal(k, seed, (s.T, s.n_out), 0.0, 1.0)
+    raise KeyError(name)
+
+
+def make_o_inputs_bits(s: OShape, seed: int = BASE_SEED) -> dict:
+    return {n: f32_to_bf16_bits(o_tensor_f64(n, s, seed).astype(np.float32)) for n in O_TENSOR_ORDER}
+
+
+# ---------------------------------------------------------------- RoPE on the query / key heads
+_ROPE_STREAM0 = 300
+
+
+@dataclasses.dataclass(frozen=True)
+class RopeShape:
+    """T tokens in sequences of seq_len (position ids t mod seq_len), hq query heads and
+    hk key heads of hd features, rotary base."""
+    T: int
+    hq: int
+    hk: int
+    hd: int
+    seq_len: int
+    base: float = 500000.0
+
+
+def rope_tables(n_pos: int, hd: int, base: float):
+    """The cos / sin caches the RoPE kernel looks up by position: [n_pos x hd/2] fp32,
+    angle(p, i) = p * base^(-2 i / hd), computed in fp64 and rounded once (how a model
+    builds its rotary caches; they are inputs of the kernel)."""
+    theta = base ** (-2.0 * np.arange(hd // 2, dtype=np.float64) / hd)
+    ang = np.outer(np.arange(n_pos, dtype=np.float64), theta)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def make_rope_inputs(s: RopeShape, seed: int = BASE_SEED) -> dict:
+    """Q [T x hq hd], K [T x hk hd] and their upstream gradients dQ, dK as bf16 bits
+    (N(0,1)), position ids int32 [T] = t mod seq_len, cos / sin tables fp32."""
+    out = {}
+    for i, (name, h) in enumerate((("Q", s.hq), ("K", s.hk), ("dQ", s.hq), ("dK", s.hk))):
+        out[name] = f32_to_bf16_bits(_normal(_ROPE_STREAM0 + i, seed, (s.T, h * s.hd), 0.0, 1.0).astype(np.float32))
+    out["pos"] = (np.arange(s.T) % s.seq_len).astype(np.int32)
+    out["cos"], out["sin"] = rope_tables(s.seq_len, s.hd, s.base)
+    return out
+
+
+# ---------------------------------------------------------------- LM-head cross-entropy
+_CE_STREAM0 = 400
+IGNORE_INDEX = -100
+
+
+@dataclasses.dataclass(frozen=True)
+class CeShape:
+    """T tokens, hidden d, vocabulary V; a fraction of the labels is the ignore index
+    (prompt tokens left out of the loss)."""
+    T: int
+    d: int
+    V: int
+    ignored: float = 0.05
+
+
+def make_ce_inputs(s: CeShape, seed: int = BASE_SEED) -> dict:
+    """H [T x d] (final normalised hidden states) N(0,1) and the frozen LM head W [V x d]
+    N(0,0.02) as bf16 bits; labels int32 [T] uniform over the vocabulary with the given
+    fraction set to the ignore index."""
+    H = f32_to_bf16_bits(_normal(_CE_STREAM0, seed, (s.T, s.d), 0.0, 1.0).astype(np.float32))
+    W = f32_to_bf16_bits(_normal(_CE_STREAM0 + 1, seed, (s.V, s.d), 0.0, 0.02).astype(np.float32))
+    g = _rng(_CE_STREAM0 + 2, seed)
+    labels = g.integers(0, s.V, s.T).astype(np.int32)
+    labels[g.random(s.T) < s.ignored] = IGNORE_INDEX
+    return {"H": H, "W": W, "labels": labels}
