@@ -11,8 +11,9 @@ batch (weak scaling) and the adapter gradients are summed across ranks with one 
 all-reduce per step, as data-parallel LoRA training does.  Rank 0 prints one JSON line.
 
 The default line also carries sub-records measured in the same run on the same GPU:
-the Llama-3.2-1B MLP shape, the 8B shape with 4-bit frozen weights, and the 8B
-attention Q/K/V projections, each with its dominant kernel's fraction of the bf16 peak.
+the Llama-3.2-1B MLP shape, the 8B shape with 4-bit frozen weights, and the 8B model's
+attention Q/K/V projections, o_proj, RoPE and LM-head cross-entropy, each with its
+dominant kernel's fraction of its roofline.
 
 --impl reference times the fp64 CPU oracle on this host's cores instead (a bounded
 sample of rows per step), on the same metric and unit.
@@ -251,12 +252,15 @@ def timed(step, steps, stream, clk=None, label=None):
     return e0.elapsed_time(e1), ph
 
 
-def dominant(phases, name, flops_per_launch, peak):
+def dominant(phases, name, flops_per_step, steps, peak):
+    """Achieved rate of the launches of phase `name`: their algorithmic FLOPs per step
+    (all launches of the phase in one step) over their summed time per step."""
     ms, n = phases.get(name, (0.0, 0))
     if not n:
         return None
-    ach = flops_per_launch / (ms / n / 1e3) / 1e12
-    return {"kernel": name, "achieved_tflops": ach, "frac_of_burst": ach / peak, "us_per_launch": 1e3 * ms / n}
+    ach = flops_per_step / (ms / steps / 1e3) / 1e12
+    return {"kernel": name, "achieved_tflops": ach, "frac_of_burst": ach / peak, "launches_per_step": n / steps,
+            "us_per_step": 1e3 * ms / steps}
 
 
 def sub_records(args, pb8, bits8, clk, pk):
@@ -264,7 +268,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     the 4-bit record re-quantises the 8B problem's frozen weights in place)."""
     import torch
     from lora_fine_tuning_rmsnorm_b200 import configs, ops, synth
-    from lora_fine_tuning_rmsnorm_b200.runner import Problem, QkvProblem
+    from lora_fine_tuning_rmsnorm_b200.runner import CeProblem, OProblem, Problem, QkvProblem, RopeProblem
     out = {}
     steps = max(5, min(args.steps, 20))
     stream = torch.cuda.current_stream()
@@ -272,7 +276,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     def rec(label, workload, shape_T, flops, ms, ph, dom_name, dom_flops, dtype="bf16"):
         out[label] = {"workload": workload, "dtype": dtype, "steps": steps, "warmup": 3, "ms_per_step": ms / steps,
                       "tokens_per_s": shape_T * steps / (ms / 1e3), "tflops": flops * steps / (ms / 1e3) / 1e12,
-                      "dominant": dominant(ph, dom_name, dom_flops, pk["burst"]),
+                      "dominant": dominant(ph, dom_name, dom_flops, steps, pk["burst"]),
                       "gpu_launches": sum(n for _, n in ph.values()), "clocks": clk.stats(label) if clk else None}
 
     # Llama-3.2-1B MLP shape
@@ -304,6 +308,43 @@ def sub_records(args, pb8, bits8, clk, pk):
         f"nkv={sq.nkv} r={sq.r} alpha=16", sq.T, configs.qkv_algorithmic_flops(sq), ms, ph, "qkv_gemm",
         2.0 * sq.T * sq.d * (sq.nq + 2 * sq.nkv))
     del qp
+    # attention output projection o_proj of the 8B model
+    so = configs.O_8B
+    op = OProblem(so)
+    for _ in range(3):
+        op.step()
+    ms, ph = timed(op.step, steps, stream, clk, "o_proj")
+    rec("o_proj", f"LoRA o_proj fwd+bwd, Llama-3-8B shape: T={so.T} n_in={so.n_in} n_out={so.n_out} r={so.r} "
+        "alpha=16", so.T, configs.o_algorithmic_flops(so), ms, ph, "o_gemm", 2.0 * so.T * so.n_in * so.n_out)
+    del op
+    # RoPE on the 8B model's query / key heads (forward + backward, in place)
+    sr = configs.ROPE_8B
+    rp = RopeProblem(sr)
+    for _ in range(3):
+        rp.step()
+    ms, ph = timed(rp.step, steps, stream, clk, "rope")
+    rb = configs.rope_bytes(sr)
+    rms, rn = ph.get("rope", (0.0, 0))
+    gbs = rb / (rms / rn / 1e3) / 1e9 if rn else None
+    out["rope"] = {"workload": f"RoPE fwd+bwd on Q/K in place, Llama-3-8B heads: T={sr.T} hq={sr.hq} hk={sr.hk} "
+                               f"hd={sr.hd} seq={sr.seq_len} base={sr.base:g}",
+                   "dtype": "bf16 (fp32 tables)", "steps": steps, "warmup": 3, "ms_per_step": ms / steps,
+                   "tokens_per_s": sr.T * steps / (ms / 1e3),
+                   "dominant": {"kernel": "rope", "bytes_per_launch": rb, "GB/s": gbs,
+                                "frac_of_hbm": gbs / pk["hbm"] if gbs else None,
+                                "us_per_launch": 1e3 * rms / rn if rn else None},
+                   "gpu_launches": sum(n for _, n in ph.values()), "clocks": clk.stats("rope") if clk else None}
+    del rp
+    # fused LM-head cross-entropy of the 8B model (vocabulary 128256)
+    sc = configs.CE_8B
+    cp = CeProblem(sc)
+    for _ in range(3):
+        cp.step()
+    ms, ph = timed(cp.step, steps, stream, clk, "ce")
+    rec("ce", f"fused LM-head cross-entropy fwd+bwd, Llama-3-8B head: T={sc.T} d={sc.d} V={sc.V} "
+        f"(vocabulary chunk 32768 in the backward)", sc.T, configs.ce_algorithmic_flops(sc), ms, ph,
+        "ce_gemm_lse", 2.0 * sc.T * sc.d * sc.V)
+    del cp
     torch.cuda.empty_cache()
     return out
 

@@ -246,6 +246,86 @@ int lora_qkv_bwd(const lora_qkv_dims* dims, const void* dQ, const void* dK, cons
                  const void* rms_w, const lora_qkv_weights* W, const lora_qkv_adapters* A, const void* ctx,
                  void* dX, const lora_qkv_grads* grads, void* workspace, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * LoRA on the attention output projection o_proj: a LoRA linear with no norm in front
+ * (o_proj is adapted in every LoRA configuration of the pages: target_modules q_proj,
+ * k_proj, v_proj, o_proj, gate_proj, up_proj, down_proj — "【编译】结合 Unsloth 与 🤗 TRL",
+ * §三.2; the adapter is the LoRALayer linear of "Unsloth 深度实战…", §1.3):
+ *   P = s X Ao^T;  Y = X Wo^T + P Bo^T
+ * X [T x n_in] (the attention output, heads x head dim), Wo [n_out x n_in], Ao [r x n_in],
+ * Bo [n_out x r], Y [T x n_out], all bf16 row-major; the context holds P [T x rp] bf16
+ * (rp = r rounded up to 16, zero padded).  Backward from dY [T x n_out] (frozen Wo):
+ *   Q = s dY Bo;  dX = dY Wo + Q Ao (bf16);  dAo = Q^T X, dBo = dY^T P (fp32 [r x n_in],
+ *   [n_out x r], OVERWRITTEN, fp32 atomics over T).
+ * Limits: 1 <= T < 2^31; n_in, n_out >= 8 and r multiples of 8, r <= 128.  Same conventions
+ * as the MLP calls (asynchronous, caller-owned 16-byte aligned device buffers). */
+typedef struct lora_o_dims {
+  int64_t T;
+  int32_t n_in, n_out, r;
+  float scale;          /* s = alpha / r */
+} lora_o_dims;
+
+int lora_o_ctx_bytes(const lora_o_dims* dims, size_t* bytes);
+int lora_o_workspace_bytes(const lora_o_dims* dims, size_t* bytes);
+int lora_o_fwd(const lora_o_dims* dims, const void* X, const void* Wo, const void* Ao, const void* Bo, void* Y,
+               void* ctx, void* workspace, void* stream);
+int lora_o_bwd(const lora_o_dims* dims, const void* dY, const void* X, const void* Wo, const void* Ao,
+               const void* Bo, const void* ctx, void* dX, float* dAo, float* dBo, void* workspace, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Rotary position embedding of the query and key heads, in place ("Unsloth — 用手写
+ * Triton kernel 给 HF 微调换心脏", §2.3: the RoPE kernel after the Q/K/V projections,
+ * writing in place; §4: the backward is the same kernel with the sine negated;
+ * "Unsloth加速原理揭秘", §2.2: q and k rotated at their positions by one kernel).
+ * Q [T x hq*hd], K [T x hk*hd] bf16 row-major (heads of hd contiguous features, as the
+ * Q/K/V projections write them).  Dimension i of a head is paired with i + hd/2:
+ *   q_i <- q_i c - q_{i+hd/2} s,   q_{i+hd/2} <- q_{i+hd/2} c + q_i s,
+ *   c = cos[pos[t]][i], s = sin[pos[t]][i] (fp32 tables [n_pos x hd/2], row-major),
+ * computed in fp32 and rounded once to bf16.  backward = 1 applies the inverse rotation
+ * (s negated): the gradient of the forward, in place on dQ, dK.  pos [T] int32 position
+ * ids (packed sequences restart them).  hd a multiple of 16; hq or hk may be 0 (that
+ * pointer may then be NULL).  A position outside [0, n_pos) leaves its row unchanged and
+ * is reported as LORA_ERR_INVALID_ARG (by the call in debug mode, else by
+ * lora_mlp_status(NULL, ...)). */
+int lora_rope(int64_t T, int32_t hq, int32_t hk, int32_t hd, const int32_t* pos, int64_t n_pos, const float* cos_t,
+              const float* sin_t, void* Q, void* K, int32_t backward, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Fused cross-entropy of the language-model head ("Unsloth — 用手写 Triton kernel 给 HF
+ * 微调换心脏", §2.3 step 6 and §4: the loss is computed from the final hidden states in
+ * chunks and the logits tensor never exists in full; §7, Fast_CrossEntropyLoss):
+ *   z = H W^T (never stored), lse_t = log sum_v exp(z_tv),
+ *   loss_t = lse_t - z_{t, labels[t]}, or 0 when labels[t] is outside [0, V) (the ignore
+ *   index -100 included: the token is left out);
+ *   loss = mean of loss_t over the kept tokens (LORA_CE_MEAN; 0 if none) or their sum.
+ * Backward for the upstream gradient dloss of the reduced loss (W frozen):
+ *   dH_t = dloss' sum_v (softmax(z_t)_v - [v = labels[t]]) W_v,  dloss' = dloss / n_valid
+ *   (mean) or dloss (sum); dH_t = 0 for tokens left out.
+ * H [T x d] bf16 (final normalised hidden states), W [V x d] bf16 (the LM head), labels
+ * [T] int32 (already shifted by the caller), all row-major device memory.  Forward writes
+ * loss_rows [T] fp32, lse [T] fp32 (saved for the backward), *loss (fp32) and *n_valid
+ * (int32, the kept count); the backward reads lse and n_valid from the forward and writes
+ * dH [T x d] fp32 (OVERWRITTEN).  The backward recomputes the logits of vocab_chunk
+ * columns at a time and keeps only that chunk's dZ = dloss' (softmax - onehot) in the
+ * workspace (bf16 [T x vocab_chunk]).  d, V multiples of 8; vocab_chunk a multiple of
+ * 256, 0 = 32768.  loss and n_valid need 4-byte alignment, the rest 16.  The per-token
+ * sums are reduced in a fixed order (the loss is deterministic). */
+#define LORA_CE_MEAN 0
+#define LORA_CE_SUM 1
+typedef struct lora_ce_dims {
+  int64_t T;
+  int32_t d;
+  int32_t V;
+  int32_t vocab_chunk;
+  int32_t reduction;  /* LORA_CE_MEAN or LORA_CE_SUM */
+} lora_ce_dims;
+
+int lora_ce_workspace_bytes(const lora_ce_dims* dims, size_t* bytes);
+int lora_ce_fwd(const lora_ce_dims* dims, const void* H, const void* W, const int32_t* labels, float* loss_rows,
+                float* lse, float* loss, int32_t* n_valid, void* workspace, void* stream);
+int lora_ce_bwd(const lora_ce_dims* dims, const void* H, const void* W, const int32_t* labels, const float* lse,
+                const int32_t* n_valid, float dloss, float* dH, void* workspace, void* stream);
+
 /* Adapter folded into its frozen weight for export ("Unsloth提速秘诀…", §3.1, "LoRA
  * Update + Weight Merge"; "Unsloth 深度实战", §5.1, the merged 16-bit save):
  *   Wm[o][i] = bf16( W[o][i] + scale * sum_{k<r} B[o][k] A[k][i] )
@@ -283,15 +363,16 @@ int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn,
 
 /* Bounded-wait status of the most recent call that used `workspace` (any workspace
  * of this library: its status word sits at offset 0), or, with workspace = NULL, of
- * the most recent lora_gemm_bf16 / lora_lowrank_proj_noalloc call in the current
- * CUDA context.  Every device wait in the kernels has a time limit
+ * the most recent lora_gemm_bf16 / lora_lowrank_proj_noalloc / lora_rope call in the
+ * current CUDA context.  Every device wait in the kernels has a time limit
  * (LORA_MLP_WAIT_LIMIT_MS in the environment, default 5000 ms); a wait that runs out
  * makes its kernel record a code in the status word, stop its other roles, wait for
  * its own copies and tensor-core operations in flight, free its tensor memory and
  * return, leaving the outputs incomplete.  Each call clears its status word when it
  * is enqueued, so check after every call whose result matters.
  * Synchronises `stream`, then returns LORA_OK, or LORA_ERR_TIMEOUT with the code in
- * *code (may be NULL) and in lora_mlp_last_error().  With LORA_MLP_DEBUG=1 every call
+ * *code (may be NULL) and in lora_mlp_last_error() (LORA_ERR_INVALID_ARG for a device-side
+ * index input out of range, such as a RoPE position).  With LORA_MLP_DEBUG=1 every call
  * does this check itself before it returns. */
 int lora_mlp_status(const void* workspace, int32_t* code, void* stream);
 
@@ -323,7 +404,7 @@ int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, cons
  * is bracketed by CUDA events on the caller's stream.  lora_mlp_timing_collect()
  * synchronises those events and returns, per phase id, the summed milliseconds and
  * the number of launches since the previous collect (arrays of LORA_NUM_PHASES). */
-#define LORA_NUM_PHASES 20
+#define LORA_NUM_PHASES 28
 int lora_mlp_timing_enable(int32_t on);
 int lora_mlp_timing_collect(double* ms, int64_t* launches);
 const char* lora_mlp_phase_name(int32_t phase);

@@ -67,7 +67,10 @@ enum Epi : int {
   EPI_BF16 = 1,        // out[0] bf16 = acc_a * alpha (+ in[0] when set), accumulator a at column a * out_acc_col
   EPI_SWIGLU_FWD = 2,  // acc0 = G, acc1 = U -> out[0] G, out[1] U, out[2] silu(G) * U (bf16)
   EPI_SWIGLU_BWD = 3,  // acc0 = dAct; in[0] G, in[1] U -> out[0] dG, out[1] dU (bf16)
-  EPI_ATOMIC = 4       // accumulator a atomically added into fp32 output rng[a] (split-K reductions)
+  EPI_ATOMIC = 4,      // accumulator a atomically added into fp32 output rng[a] (split-K reductions)
+  EPI_CE_LSE = 5,      // logits tile -> per row and tile half: (max, sum exp(z - max)) into out[0] (float2
+                       // [2 tiles_n][M]) and the label's logit into out[1] (float [M]); logits never stored
+  EPI_CE_DZ = 6        // logits tile -> dZ = g' (softmax - onehot(label)) as bf16 into out[0] (ld_out)
 };
 
 enum Hint : int { HINT_NONE = 0, HINT_EVICT_FIRST = 1, HINT_EVICT_LAST = 2 };
@@ -120,6 +123,14 @@ struct GemmArgs {
   uint32_t cr_bytes;      // 4-bit: bytes of one code-ring entry
   int test_no_loads;      // test of the bounded waits: the producer copies nothing and arms no
                           // barrier, so the MMA's first wait runs out (single-CTA tiles only)
+  int out_add;            // EPI_F32: add into the fp32 output instead of overwriting it
+  // cross-entropy epilogues (rows = tokens, columns = vocabulary entries ce_col0 + n)
+  const int* ce_labels;   // label of each row; outside [0, ce_V) = left out of the loss
+  const float* ce_lse;    // EPI_CE_DZ: logsumexp of each row (from the forward)
+  const int* ce_count;    // EPI_CE_DZ: number of kept rows (mean reduction), NULL = sum reduction
+  float ce_g;             // EPI_CE_DZ: upstream gradient of the reduced loss
+  int ce_col0;            // vocabulary index of this launch's column 0 (vocabulary chunks)
+  int ce_V;               // vocabulary size
 };
 
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
@@ -161,7 +172,7 @@ __device__ __forceinline__ void seg_kb_range(const GemmArgs& p, int s, int ks, i
 }
 
 // Drain wait used after an abort: ignores the abort flag, bounded by the limit.
-__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const WaitCtl& c) {
+static __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const WaitCtl& c) {
   const uint64_t t0 = global_ns();
   while (!mbar_test(bar, parity)) {
     if (global_ns() - t0 > c.limit_ns) {
@@ -481,6 +492,10 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
                                        __uint_as_float(r[4 * h + 1]) * p.alpha,
                                        __uint_as_float(r[4 * h + 2]) * p.alpha,
                                        __uint_as_float(r[4 * h + 3]) * p.alpha);
+                if (p.out_add) {
+                  const float4 old = *reinterpret_cast<const float4*>(o + 4 * h);
+                  v.x += old.x; v.y += old.y; v.z += old.z; v.w += old.w;
+                }
                 st_out(reinterpret_cast<float4*>(o + 4 * h), v, p.stream_out);
               }
             }
@@ -612,6 +627,81 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
                           make_float4(__uint_as_float(r[4 * h]) * p.alpha, __uint_as_float(r[4 * h + 1]) * p.alpha,
                                       __uint_as_float(r[4 * h + 2]) * p.alpha, __uint_as_float(r[4 * h + 3]) * p.alpha));
           }
+        }
+      }
+    } else if (EPI == EPI_CE_LSE) {
+      // Online max / sum of exponentials over this warp's 16-column chunks of the tile:
+      // m = running max, s = sum exp(z - m) (base-2 exponentials of pre-scaled values).
+      constexpr float kLog2e = 1.4426950408889634f;
+      const int lab = row_ok ? __ldg(p.ce_labels + row) : -1;
+      float m = -INFINITY, sum = 0.f, zl = 0.f;
+      bool has = false;
+#pragma unroll 1
+      for (int c = c0; c < p.bn; c += 32) {
+        const int n = n0 + c;
+        if (n >= p.N) break;  // warp-uniform: the rest of the tile is past the vocabulary
+        uint32_t r[16];
+        tmem_ld16(tbase + c, r);
+        tmem_wait16(r);
+        if (!row_ok) continue;
+        float v[16], cm = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          v[e] = n + e < p.N ? __uint_as_float(r[e]) : -INFINITY;
+          cm = fmaxf(cm, v[e]);
+          if (p.ce_col0 + n + e == lab) {
+            zl = v[e];
+            has = true;
+          }
+        }
+        const float mn = fmaxf(m, cm);
+        const float ms = mn * kLog2e;
+        float acc = sum * exp2f(fmaf(m, kLog2e, -ms));
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc += exp2f(fmaf(v[e], kLog2e, -ms));
+        sum = acc;
+        m = mn;
+      }
+      if (row_ok) {
+        const int half = (warp - 2) >> 2;
+        reinterpret_cast<float2*>(p.out[0])[static_cast<long long>(2 * nt + half) * p.M + row] = make_float2(m, sum);
+        if (has) static_cast<float*>(p.out[1])[row] = zl;
+      }
+    } else if (EPI == EPI_CE_DZ) {
+      // dZ = g' (exp(z - lse) - [column == label]); 0 for rows left out of the loss
+      constexpr float kLog2e = 1.4426950408889634f;
+      const int lab = row_ok ? __ldg(p.ce_labels + row) : -1;
+      const bool keep = lab >= 0 && lab < p.ce_V;
+      float gs = 0.f, l2 = 0.f;
+      if (keep) {
+        gs = p.ce_count ? p.ce_g / static_cast<float>(max(1, __ldg(p.ce_count))) : p.ce_g;
+        l2 = __ldg(p.ce_lse + row) * kLog2e;
+      }
+#pragma unroll 1
+      for (int c = c0; c < p.bn; c += 32) {
+        const int n = n0 + c;
+        if (n >= p.N) break;
+        uint32_t r[16];
+        tmem_ld16(tbase + c, r);
+        tmem_wait16(r);
+        if (!row_ok) continue;
+        uint16_t* o = static_cast<uint16_t*>(p.out[0]) + row * p.ld_out + n;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (n + 8 * h >= p.N) continue;
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float dz[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int k = 8 * h + 2 * j + e;
+              const float pr = exp2f(fmaf(__uint_as_float(r[k]), kLog2e, -l2));
+              dz[e] = gs * (pr - (p.ce_col0 + n + k == lab ? 1.f : 0.f));
+            }
+            w[j] = pack_bf16x2(dz[0], dz[1]);
+          }
+          st_out(reinterpret_cast<uint4*>(o + 8 * h), make_uint4(w[0], w[1], w[2], w[3]), p.stream_out);
         }
       }
     }
@@ -826,7 +916,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
 }
 
 template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE, int Q4>
-__global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
+static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
   static_assert(!FUSE || (NACC == 2 && !B_MN), "fused wide MMA: two K-major B halves");
   static_assert(!Q4 || !A_MN, "4-bit B: K-major A");
   extern __shared__ uint8_t smem_raw[];

@@ -1,364 +1,19 @@
-// Host side of liblora_mlp.so: argument validation, TMA tensor-map construction,
-// the launch sequence of the LoRA-MLP forward/backward, per-phase timing and the
-// extern "C" entry points declared in include/lora_mlp.h.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-#include <cuda_runtime.h>
-
-#include <algorithm>
-#include <cmath>
-#include <cstdarg>
-#include <cstdio>
-#include <cstdlib>
-#include <cstring>
-#include <mutex>
-#include <vector>
-
-#include "lora_mlp.h"
-#include "gemm_sm100.cuh"
-#include "rowops.cuh"
+// Host side of liblora_mlp.so for the MLP sub-block and the library-wide calls:
+// argument validation, the launch sequence of the LoRA-MLP forward/backward, the
+// library-owned device memory, per-phase timing and status, and those extern "C"
+// entry points of include/lora_mlp.h.  (Q/K/V, o_proj and RoPE: lora_attn.cu;
+// the LM-head cross-entropy: lora_ce.cu.)
+#include "host.cuh"
 
 using namespace lm;
+using namespace lm::host;
 
 namespace {
-
-thread_local char g_err[512] = "no error";
-
-int fail(int code, const char* fmt, ...) {
-  va_list ap;
-  va_start(ap, fmt);
-  vsnprintf(g_err, sizeof(g_err), fmt, ap);
-  va_end(ap);
-  return code;
-}
-
-#define CUDA_TRY(expr)                                                                   \
-  do {                                                                                   \
-    cudaError_t e_ = (expr);                                                             \
-    if (e_ != cudaSuccess)                                                               \
-      return fail(LORA_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));        \
-  } while (0)
-
-#define TRY(expr)            \
-  do {                       \
-    int rc_ = (expr);        \
-    if (rc_ != LORA_OK) return rc_; \
-  } while (0)
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-int round_up(int x, int m) { return (x + m - 1) / m * m; }
-
-bool debug_mode() {
-  static int v = [] {
-    const char* e = getenv("LORA_MLP_DEBUG");
-    return (e && e[0] && e[0] != '0') ? 1 : 0;
-  }();
-  return v != 0;
-}
-
-unsigned long long wait_limit_ns() {
-  const char* e = getenv("LORA_MLP_WAIT_LIMIT_MS");
-  long long ms = e ? atoll(e) : 5000;
-  if (ms < 1) ms = 1;
-  return static_cast<unsigned long long>(ms) * 1000000ull;
-}
-
-// ------------------------------------------------------------------ driver API
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-int get_encoder() {
-  if (g_encode) return LORA_OK;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
-    return fail(LORA_ERR_CUDA, "cannot resolve cuTensorMapEncodeTiled");
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  return LORA_OK;
-}
-
-// 2-D bf16 tensor map, 128-byte swizzle: `inner` contiguous elements per row,
-// `outer` rows `ld` elements apart, box of box_inner x box_outer elements.
-int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
-             uint32_t box_inner, uint32_t box_outer) {
-  TRY(get_encoder());
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): inner=%llu outer=%llu ld=%llu box=%ux%u",
-                static_cast<int>(r), (unsigned long long)inner, (unsigned long long)outer,
-                (unsigned long long)ld, box_inner, box_outer);
-  return LORA_OK;
-}
-// Untyped 2-D map without swizzle (4-bit codes as bytes, block absmax as fp32).
-int make_map_raw(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint32_t esize, uint64_t inner,
-                 uint64_t outer, uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
-  TRY(get_encoder());
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * esize};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled (raw) failed (%d): inner=%llu outer=%llu box=%ux%u",
-                static_cast<int>(r), (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
-  return LORA_OK;
-}
-// 4-bit weight W [rows x cols] (codes: rows x cols/2 bytes; absmax: rows x cols/64 fp32)
-// read with K = cols contiguous (forward use): boxes {32 B, n_rows} and {4 floats, n_rows}.
-int map_q4_k(CUtensorMap* mq, CUtensorMap* ma, const uint8_t* q, const float* am, uint64_t rows, uint64_t cols,
-             uint32_t n_rows) {
-  TRY(make_map_raw(mq, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cols / 2, rows, cols / 2, 32, n_rows));
-  return make_map_raw(ma, am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols / 64, rows, cols / 64, 4, n_rows);
-}
-// The same weight read with N = cols contiguous and K = rows (backward use): boxes
-// {n_cols / 2 B, 64 K rows} and {4 floats, 64 K rows}.
-int map_q4_mn(CUtensorMap* mq, CUtensorMap* ma, const uint8_t* q, const float* am, uint64_t rows, uint64_t cols,
-              uint32_t n_cols) {
-  TRY(make_map_raw(mq, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cols / 2, rows, cols / 2, n_cols / 2, 64));
-  return make_map_raw(ma, am, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols / 64, rows, cols / 64, 4, 64);
-}
-
-// Operand with K contiguous: [rows x K], box 64 (K) x box_rows.
-int map_k(CUtensorMap* m, const void* p, uint64_t rows, uint64_t K, uint64_t ld, uint32_t box_rows) {
-  return make_map(m, p, K, rows, ld, 64, box_rows);
-}
-// Operand with M/N contiguous: [K x MN], box 64 (MN) x 64 (K).
-int map_mn(CUtensorMap* m, const void* p, uint64_t K, uint64_t MN, uint64_t ld) {
-  return make_map(m, p, MN, K, ld, 64, 64);
-}
-// The same operand as a 3-D view {64 elements, K rows, MN/64 chunks} (MN % 64 == 0),
-// box {64, 64, chunks}: one load fills `chunks` chunk-major 8 KB sub-tiles.
-int map_mn3(CUtensorMap* m, const void* p, uint64_t K, uint64_t MN, uint64_t ld, uint32_t chunks) {
-  TRY(get_encoder());
-  cuuint64_t dims[3] = {64, K, MN / 64};
-  cuuint64_t strides[2] = {ld * 2, 128};
-  cuuint32_t box[3] = {64, 64, chunks};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d): K=%llu MN=%llu ld=%llu chunks=%u",
-                static_cast<int>(r), (unsigned long long)K, (unsigned long long)MN, (unsigned long long)ld, chunks);
-  return LORA_OK;
-}
-
-// --------------------------------------------------------------------- timing
-const char* kPhaseNames[LORA_NUM_PHASES] = {
-    "rmsnorm_fwd", "proj_P_gate_up", "gemm_gate_up_swiglu", "proj_P_down", "gemm_down",
-    "proj_Q_down", "gemm_dact_swiglu_bwd", "proj_Q_gate_up", "gemm_dH", "rmsnorm_bwd",
-    "zero_grads", "reduce_dA_gate_up", "reduce_dB_gate_up", "reduce_dB_down", "reduce_dA_down",
-    "norm_weight_grad", "other", "qkv_gemm", "qkv_gemm_dH", "qkv_lowrank"};
-enum Phase {
-  PH_RMS_FWD = 0, PH_P_GU, PH_GATEUP, PH_P_D, PH_DOWN, PH_Q_D, PH_DACT, PH_Q_GU, PH_DH,
-  PH_RMS_BWD, PH_ZERO, PH_RED_DA_GU, PH_RED_DB_GU, PH_RED_DB_D, PH_RED_DA_D, PH_DW, PH_OTHER,
-  PH_QKV_GEMM, PH_QKV_DH, PH_QKV_LOWRANK
-};
-
-struct Timing {
-  std::mutex mu;
-  bool on = false;
-  struct Rec { cudaEvent_t a, b; int phase; };
-  std::vector<Rec> pending;
-  std::vector<cudaEvent_t> pool;
-  cudaEvent_t get() {
-    if (!pool.empty()) {
-      cudaEvent_t e = pool.back();
-      pool.pop_back();
-      return e;
-    }
-    cudaEvent_t e = nullptr;
-    cudaEventCreate(&e);
-    return e;
-  }
-} g_timing;
-
-struct PhaseScope {
-  cudaStream_t st;
-  int phase;
-  cudaEvent_t a = nullptr, b = nullptr;
-  PhaseScope(cudaStream_t s, int ph) : st(s), phase(ph) {
-    std::lock_guard<std::mutex> lk(g_timing.mu);
-    if (!g_timing.on) return;
-    a = g_timing.get();
-    b = g_timing.get();
-    cudaEventRecord(a, st);
-  }
-  ~PhaseScope() {
-    if (!a) return;
-    cudaEventRecord(b, st);
-    std::lock_guard<std::mutex> lk(g_timing.mu);
-    g_timing.pending.push_back({a, b, phase});
-  }
-};
-
-// ------------------------------------------------------------------ launches
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
-
-constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
-
-// Launch one GEMM.  PAIR = 2 runs clusters of two CTAs sharing 256-row tiles
-// (tcgen05 cta_group::2); the caller sets tiles_m = ceil(M / (128 * PAIR)).
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1, int FUSE = 0, int Q4 = 0>
-int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
-  static_assert(PAIR == 1 || (PAIR == 2 && !A_MN), "CTA pairs take a K-major A operand");
-  if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
-    return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
-  a.stage_bytes = BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
-  a.cr_bytes = 0;
-  if (Q4) {  // 4-bit B: expanded B slots per stage; codes + absmax in a ring of their own
-    const Q4Layout QL = q4_layout(a.bn, PAIR, FUSE, B_MN, NACC);
-    a.stage_bytes = BM * BK * 2 + QL.slots * QL.b_unit;
-    a.cr_bytes = (QL.slots * (QL.q_unit + QL.m_unit) + 1023) & ~1023u;
-  }
-  a.stage_bytes = (a.stage_bytes + 1023) & ~1023u;
-  const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit code table)
-  const int ring = Q4 ? kCodeRing * static_cast<int>(a.cr_bytes) : 0;
-  const int avail = kSmemLimit - 1024 - extra - ring;
-  a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
-  static const int stage_cap = [] {
-    const char* e = getenv("LORA_MLP_MAX_STAGES");  // tuning knob: cap the TMA ring depth
-    return e ? atoi(e) : 0;
-  }();
-  if (stage_cap >= 2) a.stages = std::min(a.stages, stage_cap);
-  if (a.stages < 2) return fail(LORA_ERR_UNSUPPORTED, "internal: stage does not fit");
-  int cols = 2 * NACC * a.bn;
-  uint32_t tc = 32;
-  while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
-  if (tc > 512) return fail(LORA_ERR_UNSUPPORTED, "internal: TMEM columns %d > 512", cols);
-  a.tmem_cols = tc;
-  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + ring + extra;
-  // more than half of TMEM per CTA: keep one CTA per SM so allocation never waits
-  if (tc > 256) smem = std::max(smem, kSmemLimit / 2 + 4096);
-  a.limit_ns = wait_limit_ns();
-  const long long tiles = static_cast<long long>(a.tiles_m) * a.tiles_n * a.splits;
-  if (tiles <= 0) return LORA_OK;
-  if (tiles > 0x7fffffffLL) return fail(LORA_ERR_UNSUPPORTED, "too many tiles");
-  const int units = static_cast<int>(std::min<long long>(tiles, sm_count() / PAIR));
-  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR, FUSE, Q4>;
-  CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  PhaseScope ps(st, phase);
-  if (PAIR == 1) {
-    kern<<<units, gemm_threads(Q4), smem, st>>>(a);
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(units * PAIR, 1, 1);
-    cfg.blockDim = dim3(gemm_threads(Q4), 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = PAIR;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, a));
-  }
-  CUDA_TRY(cudaGetLastError());
-  return LORA_OK;
-}
-
-int launch_rms_fwd(cudaStream_t st, const void* X, const void* w, void* H, float* rstd, long long T, int d,
-                   float eps) {
-  const int nvec = d / 8;
-  int threads = kRowThreads, vpt = (nvec + threads - 1) / threads;
-  if (vpt > 8) {
-    vpt = 8;
-    threads = round_up((nvec + 7) / 8, 32);
-  }
-  if (threads > 1024) return fail(LORA_ERR_UNSUPPORTED, "d = %d too large for the row kernel", d);
-  int v = vpt <= 1 ? 1 : vpt <= 2 ? 2 : vpt <= 4 ? 4 : 8;
-  auto X16 = static_cast<const uint16_t*>(X);
-  auto w16 = static_cast<const uint16_t*>(w);
-  auto H16 = static_cast<uint16_t*>(H);
-  PhaseScope ps(st, PH_RMS_FWD);
-  for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
-    unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
-    switch (v) {
-      case 1: rmsnorm_fwd_kernel<1><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-      case 2: rmsnorm_fwd_kernel<2><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-      case 4: rmsnorm_fwd_kernel<4><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-      default: rmsnorm_fwd_kernel<8><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-    }
-  }
-  CUDA_TRY(cudaGetLastError());
-  return LORA_OK;
-}
-
-int launch_rms_bwd(cudaStream_t st, const float* dH, const void* X, const void* w, const float* rstd, void* dX,
-                   long long T, int d, const void* dY = nullptr) {
-  const int nvec = d / 8;
-  int threads = kRowThreads, vpt = (nvec + threads - 1) / threads;
-  if (vpt > 4) {
-    vpt = 4;
-    threads = round_up((nvec + 3) / 4, 32);
-  }
-  if (threads > 1024) return fail(LORA_ERR_UNSUPPORTED, "d = %d too large for the row kernel", d);
-  int v = vpt <= 1 ? 1 : vpt <= 2 ? 2 : 4;
-  auto X16 = static_cast<const uint16_t*>(X);
-  auto w16 = static_cast<const uint16_t*>(w);
-  auto dX16 = static_cast<uint16_t*>(dX);
-  auto dY16 = static_cast<const uint16_t*>(dY);
-  PhaseScope ps(st, PH_RMS_BWD);
-  for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
-    unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
-    switch (v) {
-      case 1: rmsnorm_bwd_kernel<1><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
-      case 2: rmsnorm_bwd_kernel<2><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
-      default: rmsnorm_bwd_kernel<4><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
-    }
-  }
-  CUDA_TRY(cudaGetLastError());
-  return LORA_OK;
-}
 
 // --------------------------------------------------------------- layouts
 struct WsLayout {
   size_t status, Q, Qd, dG, dU, dH, part, total;
 };
-
-// K-split count of a rank-r projection: about two waves of CTAs on a 148-SM part,
-// at most 8 splits (fixed, so workspace sizes do not depend on the device).
-constexpr int kProjMaxSplits = 16;
-// Number of K splits for `tiles` output tiles over nkb k-blocks: the split that
-// fills whole waves of a 148-SM part best (at most max_splits), preferring fewer
-// splits among those within 3 % of the best.  Depends only on the sizes, so
-// workspace sizes do not depend on the device.
-int balanced_splits(long long tiles, long long nkb, int max_splits) {
-  const double sms = 148.0;
-  int best = 1;
-  double best_eff = 0.0;
-  for (int s = 1; s <= max_splits && s <= nkb; ++s) {
-    const long long per = (nkb + s - 1) / s;
-    const long long ss = (nkb + per - 1) / per;        // splits actually formed
-    const double w = static_cast<double>(tiles * ss) / sms;
-    double eff = w / std::ceil(w);
-    if (tiles * ss < sms) eff = w;                      // a partial single wave
-    if (eff > best_eff + 0.03) { best_eff = eff; best = static_cast<int>(ss); }
-  }
-  return best;
-}
-int proj_splits(long long T, long long K) {
-  const long long tiles = (T + 127) / 128;
-  const long long nkb = (K + 63) / 64;
-  return balanced_splits(tiles, nkb, kProjMaxSplits);
-}
 
 int check_dims(const lora_mlp_dims* D) {
   if (!D) return fail(LORA_ERR_INVALID_ARG, "dims is NULL");
@@ -415,204 +70,6 @@ WsLayout ws_layout(const lora_mlp_dims* D) {
   return L;
 }
 
-template <class P>
-P* at(void* base, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(base) + off); }
-template <class P>
-const P* at(const void* base, size_t off) { return reinterpret_cast<const P*>(static_cast<const char*>(base) + off); }
-
-int check_ptrs(std::initializer_list<const void*> ps) {
-  for (const void* p : ps) {
-    if (!p) return fail(LORA_ERR_INVALID_ARG, "a required pointer is NULL");
-    if (!aligned16(p)) return fail(LORA_ERR_ALIGNMENT, "pointer %p is not 16-byte aligned", p);
-  }
-  return LORA_OK;
-}
-
-// Every call clears its status word first (in every mode), so the word reports the
-// bounded waits of the most recent call that used it (lora_mlp_status reads it).
-int begin_call(int* status, cudaStream_t st) {
-  if (status) CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
-  return LORA_OK;
-}
-
-int end_call(int* status, cudaStream_t st) {
-  if (!debug_mode()) return LORA_OK;
-  CUDA_TRY(cudaStreamSynchronize(st));
-  if (status) {
-    int v = 0;
-    CUDA_TRY(cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost));
-    if (v) return fail(LORA_ERR_TIMEOUT, "device-side bounded wait gave up (code 0x%x)", v);
-  }
-  return LORA_OK;
-}
-
-GemmArgs new_args(int* status) {
-  GemmArgs a;
-  memset(&a, 0, sizeof(a));
-  a.splits = 1;
-  a.alpha = 1.0f;
-  a.status = status;
-  for (int s = 0; s < kMaxSegs; ++s) a.seg[s].b_map[0] = a.seg[s].b_map[1] = -1;
-  return a;
-}
-
-// Banded tile order for a dense GEMM: `group_m` row tiles per band (the band's A
-// panels are re-read from L2 by every N tile).  LORA_MLP_RASTER=0 selects the plain
-// M-fastest order instead (tuning comparison).
-void set_band(GemmArgs& a, int group_m) {
-  static const int off = [] {
-    const char* e = getenv("LORA_MLP_RASTER");
-    return e && e[0] == '0' ? 1 : 0;
-  }();
-  if (off || group_m >= a.tiles_m) return;
-  a.raster = 2;
-  a.group_m = group_m;
-}
-
-void set_hints(GemmArgs& a, int a_hint, int b_hint) {
-  for (int s = 0; s < a.nseg; ++s) {
-    a.seg[s].a_hint = a_hint;
-    a.seg[s].b_hint = b_hint;
-  }
-}
-
-void set_seg(GemmArgs& a, int s, int amap, int ak0, int b0, int bk0, int b1, int bk1, int klen) {
-  a.seg[s].a_map = amap;
-  a.seg[s].a_k0 = ak0;
-  a.seg[s].b_map[0] = b0;
-  a.seg[s].b_k0[0] = bk0;
-  a.seg[s].b_map[1] = b1;
-  a.seg[s].b_k0[1] = bk1;
-  a.seg[s].k_len = klen;
-  a.nseg = std::max(a.nseg, s + 1);
-}
-
-// Tile shape of a dense GEMM (M = T rows, N columns): CTA pair (256-row tiles) or
-// single CTA, N tile 256 or 128 — the option that fills whole waves of the 148 SMs
-// best (ties within 2 % go to the larger tile, then to the pair).
-struct TileChoice { int pair, bn; };
-TileChoice pick_tiles(long long T, int N, bool mn_major) {
-  TileChoice best{T > 128 ? 2 : 1, N >= 256 ? 256 : (mn_major ? round_up(N, 64) : round_up(N, 16))};
-  if (N < 256 || T <= 128) return best;
-  // Cost = whole waves x time of one tile.  A tile of N = 128 takes about 0.8 of an
-  // N = 256 tile's time (measured: the per-k-block issue and barrier work of the MMA
-  // thread does not shrink with N), so N = 128 only pays where it saves many waves.
-  double best_cost = 1e30;
-  const int bns[2] = {256, 128};
-  for (int pair = 2; pair >= 1; --pair) {
-    for (int bn : bns) {
-      const long long units = ((T + 128LL * pair - 1) / (128LL * pair)) * ((N + bn - 1) / bn);
-      const double waves = std::ceil(units / (148.0 / pair));
-      const double cost = waves * (bn == 256 ? 1.0 : 0.8);
-      if (cost < best_cost - 1e-9) {
-        best_cost = cost;
-        best = TileChoice{pair, bn};
-      }
-    }
-  }
-  return best;
-}
-
-// Rank-r projection out[T x cols] (bf16) = scale * sum of K-split fp32 partials.
-// The GEMM args must already hold maps/segments/M/N/bn/tiles and NACC columns.
-template <int B_MN, int NACC>
-int launch_proj(GemmArgs& a, long long T, long long K, int cols, float* part, void* out, float scale,
-                cudaStream_t st, int phase) {
-  const int s = proj_splits(T, K);
-  const long long nkb = (K + BK - 1) / BK;
-  const long long per = (nkb + s - 1) / s;
-  a.splits = s;
-  a.k_chunk = static_cast<int>(per * BK);
-  a.out[0] = part;
-  a.ld_out = cols;
-  a.split_stride = T * cols;
-  a.alpha = 1.0f;
-  TRY((launch_gemm<0, B_MN, NACC, EPI_F32>(a, st, phase)));
-  const long long n = T * cols;
-  const long long blocks = (n / 4 + 255) / 256;
-  PhaseScope ps(st, phase);
-  splitk_finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, s, T * cols, n, scale,
-                                                                        static_cast<uint16_t*>(out));
-  CUDA_TRY(cudaGetLastError());
-  return LORA_OK;
-}
-
-// Split the T reduction of an adapter-gradient GEMM so that the tiles fill whole
-// waves (at most 12 splits: every split adds one set of fp32 atomics per output).
-void choose_splits(GemmArgs& a, long long K) {
-  const long long tiles = static_cast<long long>(a.tiles_m) * a.tiles_n;
-  const long long nkb = (K + BK - 1) / BK;
-  const int s = balanced_splits(tiles, nkb, 12);
-  const long long per = (nkb + s - 1) / s;
-  a.k_chunk = static_cast<int>(per * BK);
-  a.splits = static_cast<int>((nkb + per - 1) / per);
-}
-
-// ------------------------------------------------- attention Q/K/V projections
-int check_qkv_dims(const lora_qkv_dims* D) {
-  if (!D) return fail(LORA_ERR_INVALID_ARG, "dims is NULL");
-  if (D->T < 1 || D->T >= (1LL << 31)) return fail(LORA_ERR_INVALID_ARG, "T = %lld out of range", (long long)D->T);
-  if (D->d < 8 || D->nq < 8 || D->nkv < 8 || D->r < 1) return fail(LORA_ERR_INVALID_ARG, "d, nq, nkv >= 8, r >= 1");
-  if (D->d % 8 || D->nq % 8 || D->nkv % 8 || D->r % 8)
-    return fail(LORA_ERR_ALIGNMENT, "d, nq, nkv, r must be multiples of 8; got %d %d %d %d", D->d, D->nq, D->nkv, D->r);
-  if (D->d > 65536) return fail(LORA_ERR_UNSUPPORTED, "d = %d > 65536", D->d);
-  if (D->r > 128) return fail(LORA_ERR_UNSUPPORTED, "r = %d > 128", D->r);
-  return LORA_OK;
-}
-
-lora_qkv_ctx_layout qkv_ctx_layout(const lora_qkv_dims* D) {
-  const size_t T = D->T, d = D->d, rp = round_up(D->r, 16);
-  lora_qkv_ctx_layout L{};
-  size_t o = 0;
-  L.rstd = o; o = up256(o + T * 4);
-  L.H = o;    o = up256(o + T * d * 2);
-  L.P = o;    o = up256(o + T * 3 * rp * 2);
-  L.total = o;
-  L.rp = static_cast<int32_t>(rp);
-  return L;
-}
-
-struct QkvWsLayout {
-  size_t status, Q, dH, part, total;
-};
-QkvWsLayout qkv_ws_layout(const lora_qkv_dims* D) {
-  const size_t T = D->T, d = D->d, rp = round_up(D->r, 16);
-  QkvWsLayout L{};
-  size_t o = 0;
-  L.status = o; o = 256;
-  L.Q = o;  o = up256(o + T * 3 * rp * 2);   // s (dQ Bq | dK Bk | dV Bv)
-  L.dH = o; o = up256(o + T * d * 4);
-  size_t part = 0;
-  for (long long K : {static_cast<long long>(D->d), static_cast<long long>(D->nq), static_cast<long long>(D->nkv)})
-    part = std::max(part, size_t(proj_splits(T, K)) * T * rp);
-  L.part = o; o = up256(o + part * 4);
-  L.total = o;
-  return L;
-}
-
-// Rank-r projection written into a column block of a wider bf16 matrix:
-// out[:, 0:rp] (row stride ld_out) = scale * sum of K-split fp32 partials.
-template <int B_MN>
-int launch_proj_into(GemmArgs& a, long long T, long long K, int rp, float* part, void* out, long long ld_out,
-                     float scale, cudaStream_t st, int phase) {
-  const int s = proj_splits(T, K);
-  const long long nkb = (K + BK - 1) / BK;
-  const long long per = (nkb + s - 1) / s;
-  a.splits = s;
-  a.k_chunk = static_cast<int>(per * BK);
-  a.out[0] = part;
-  a.ld_out = rp;
-  a.split_stride = T * rp;
-  a.alpha = 1.0f;
-  TRY((launch_gemm<0, B_MN, 1, EPI_F32>(a, st, phase)));
-  const long long n = T * rp;
-  const long long blocks = (n / 4 + 255) / 256;
-  PhaseScope ps(st, phase);
-  splitk_finalize_strided_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      part, s, T * rp, T, rp, ld_out, scale, static_cast<uint16_t*>(out));
-  CUDA_TRY(cudaGetLastError());
-  return LORA_OK;
-}
 
 }  // namespace
 
@@ -632,11 +89,7 @@ static __device__ __align__(256) int g_lib_status;
 // current, and cached under that context's unique id (cuCtxGetId: unlike the CUcontext
 // handle, an id is never reused within the process, so a context destroyed by
 // cudaDeviceReset and its successor get different entries).
-struct LibSyms {
-  unsigned long long ctx_id;
-  float* scratch;
-  int* status;
-};
+namespace {
 std::mutex g_syms_mu;
 std::vector<LibSyms> g_syms;
 PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
@@ -657,7 +110,9 @@ int resolve_ctx_fns() {
   return LORA_OK;
 }
 
-int lib_syms(LibSyms* out) {
+}  // namespace
+
+int lm::host::lib_syms(LibSyms* out) {
   std::lock_guard<std::mutex> lk(g_syms_mu);
   TRY(resolve_ctx_fns());
   CUcontext ctx = nullptr;
@@ -863,6 +318,8 @@ int lora_mlp_status(const void* workspace, int32_t* code, void* stream) {
   int v = 0;
   CUDA_TRY(cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost));
   if (code) *code = v;
+  if ((v & 0xF00) == kDevBadIndex)
+    return fail(LORA_ERR_INVALID_ARG, "a device-side index input was out of range (code 0x%x)", v);
   if (v) return fail(LORA_ERR_TIMEOUT, "device-side bounded wait gave up (code 0x%x)", v);
   return LORA_OK;
 }
@@ -1292,188 +749,6 @@ int lora_lowrank_proj_noalloc(int64_t T, int32_t K, int32_t r, float scale, cons
   TRY(begin_call(a.status, st));
   TRY((launch_proj<0, 1>(a, T, K, rp, part, P, scale, st, PH_OTHER)));
   return end_call(a.status, st);
-}
-
-
-int lora_qkv_ctx_layout_get(const lora_qkv_dims* dims, lora_qkv_ctx_layout* out) {
-  TRY(check_qkv_dims(dims));
-  if (!out) return fail(LORA_ERR_INVALID_ARG, "out is NULL");
-  *out = qkv_ctx_layout(dims);
-  return LORA_OK;
-}
-
-int lora_qkv_workspace_bytes(const lora_qkv_dims* dims, size_t* bytes) {
-  TRY(check_qkv_dims(dims));
-  if (!bytes) return fail(LORA_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = qkv_ws_layout(dims).total;
-  return LORA_OK;
-}
-
-int lora_qkv_fwd(const lora_qkv_dims* D, const void* X, const void* rms_w, const lora_qkv_weights* W,
-                 const lora_qkv_adapters* A, void* Qo, void* Ko, void* Vo, void* ctx, void* workspace,
-                 void* stream) {
-  TRY(check_qkv_dims(D));
-  if (!W || !A) return fail(LORA_ERR_INVALID_ARG, "weights/adapters is NULL");
-  TRY(check_ptrs({X, rms_w, Qo, Ko, Vo, ctx, workspace, W->Wq, W->Wk, W->Wv, A->Aq, A->Bq, A->Ak, A->Bk, A->Av,
-                  A->Bv}));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long T = D->T;
-  const int d = D->d, r = D->r, rp = round_up(r, 16);
-  const lora_qkv_ctx_layout L = qkv_ctx_layout(D);
-  const QkvWsLayout WL = qkv_ws_layout(D);
-  int* status = at<int>(workspace, WL.status);
-  void* H = at<char>(ctx, L.H);
-  float* rstd = at<float>(ctx, L.rstd);
-  char* P = at<char>(ctx, L.P);
-  float* part = at<float>(workspace, WL.part);
-  TRY(begin_call(status, st));
-  TRY(launch_rms_fwd(st, X, rms_w, H, rstd, T, d, D->eps));
-  const void* Wx[3] = {W->Wq, W->Wk, W->Wv};
-  const void* Ax[3] = {A->Aq, A->Ak, A->Av};
-  const void* Bx[3] = {A->Bq, A->Bk, A->Bv};
-  void* Ox[3] = {Qo, Ko, Vo};
-  const int nx[3] = {D->nq, D->nkv, D->nkv};
-  // P_x = s H A_x^T into columns [x rp, x rp + rp) of P [T x 3rp]
-  for (int x = 0; x < 3; ++x) {
-    GemmArgs a = new_args(status);
-    TRY(map_k(&a.maps[0], H, T, d, d, 128));
-    TRY(map_k(&a.maps[1], Ax[x], r, d, d, rp));
-    set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
-    a.M = static_cast<int>(T); a.N = rp; a.bn = rp;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
-    TRY((launch_proj_into<0>(a, T, d, rp, part, P + static_cast<size_t>(x) * rp * 2, 3LL * rp, D->scale, st,
-                             PH_QKV_LOWRANK)));
-  }
-  // Out_x = H W_x^T + P_x B_x^T: the LoRA term as a K = rp extension of the dense GEMM
-  for (int x = 0; x < 3; ++x) {
-    GemmArgs a = new_args(status);
-    const TileChoice tcx = pick_tiles(T, nx[x], false);
-    const int bn = tcx.bn;
-    const int pair = (tcx.pair == 2 && bn >= 32) ? 2 : 1;
-    TRY(map_k(&a.maps[0], H, T, d, d, 128));
-    TRY(map_k(&a.maps[1], Wx[x], nx[x], d, d, bn / pair));
-    TRY(map_k(&a.maps[2], P + static_cast<size_t>(x) * rp * 2, T, rp, 3 * rp, 128));
-    TRY(map_k(&a.maps[3], Bx[x], nx[x], r, r, bn / pair));
-    set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
-    set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
-    a.M = static_cast<int>(T); a.N = nx[x]; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (nx[x] + bn - 1) / bn;
-    a.out[0] = Ox[x]; a.ld_out = nx[x];
-    a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_QKV_GEMM)));
-    else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_QKV_GEMM)));
-  }
-  return end_call(status, st);
-}
-
-int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const void* dV, const void* X,
-                 const void* rms_w, const lora_qkv_weights* W, const lora_qkv_adapters* A, const void* ctx,
-                 void* dX, const lora_qkv_grads* gr, void* workspace, void* stream) {
-  TRY(check_qkv_dims(D));
-  if (!W || !A || !gr) return fail(LORA_ERR_INVALID_ARG, "weights/adapters/grads is NULL");
-  TRY(check_ptrs({dQ, dK, dV, X, rms_w, ctx, dX, workspace, W->Wq, W->Wk, W->Wv, A->Aq, A->Bq, A->Ak, A->Bk,
-                  A->Av, A->Bv, gr->dAq, gr->dBq, gr->dAk, gr->dBk, gr->dAv, gr->dBv}));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long T = D->T;
-  const int d = D->d, r = D->r, rp = round_up(r, 16);
-  const lora_qkv_ctx_layout L = qkv_ctx_layout(D);
-  const QkvWsLayout WL = qkv_ws_layout(D);
-  int* status = at<int>(workspace, WL.status);
-  const void* H = at<char>(ctx, L.H);
-  const float* rstd = at<float>(ctx, L.rstd);
-  const char* P = at<char>(ctx, L.P);
-  char* Q = at<char>(workspace, WL.Q);
-  float* dH = at<float>(workspace, WL.dH);
-  float* part = at<float>(workspace, WL.part);
-  const void* dZ[3] = {dQ, dK, dV};
-  const void* Wx[3] = {W->Wq, W->Wk, W->Wv};
-  const void* Ax[3] = {A->Aq, A->Ak, A->Av};
-  const void* Bx[3] = {A->Bq, A->Bk, A->Bv};
-  float* dAx[3] = {gr->dAq, gr->dAk, gr->dAv};
-  float* dBx[3] = {gr->dBq, gr->dBk, gr->dBv};
-  const int nx[3] = {D->nq, D->nkv, D->nkv};
-  const int qbn = rp <= 64 ? 64 : 128;
-  TRY(begin_call(status, st));
-  // Q_x = s dZ_x B_x into columns [x rp, x rp + rp) of Q [T x 3rp]
-  for (int x = 0; x < 3; ++x) {
-    GemmArgs a = new_args(status);
-    TRY(map_k(&a.maps[0], dZ[x], T, nx[x], nx[x], 128));
-    TRY(map_mn(&a.maps[1], Bx[x], nx[x], r, r));
-    set_seg(a, 0, 0, 0, 1, 0, -1, 0, nx[x]);
-    a.M = static_cast<int>(T); a.N = rp; a.bn = qbn;
-    a.tiles_m = static_cast<int>((T + BM - 1) / BM); a.tiles_n = 1;
-    TRY((launch_proj_into<1>(a, T, nx[x], rp, part, Q + static_cast<size_t>(x) * rp * 2, 3LL * rp, D->scale, st,
-                             PH_QKV_LOWRANK)));
-  }
-  // dH = dQ Wq + dK Wk + dV Wv + [Q_q | Q_k | Q_v] [Aq; Ak; Av]   (fp32; six K segments)
-  {
-    GemmArgs a = new_args(status);
-    const TileChoice tcx = pick_tiles(T, d, true);
-    const int bn = tcx.bn;
-    const int pair = (tcx.pair == 2 && bn % 128 == 0) ? 2 : 1;
-    a.mn3d_b = d % 64 == 0;
-    for (int x = 0; x < 3; ++x) {
-      TRY(map_k(&a.maps[2 * x], dZ[x], T, nx[x], nx[x], 128));
-      if (a.mn3d_b) {
-        TRY(map_mn3(&a.maps[2 * x + 1], Wx[x], nx[x], d, d, bn / pair / 64));
-        TRY(map_mn3(&a.maps[7 + x], Ax[x], r, d, d, bn / pair / 64));
-      } else {
-        TRY(map_mn(&a.maps[2 * x + 1], Wx[x], nx[x], d, d));
-        TRY(map_mn(&a.maps[7 + x], Ax[x], r, d, d));
-      }
-      set_seg(a, x, 2 * x, 0, 2 * x + 1, 0, -1, 0, nx[x]);
-    }
-    TRY(map_k(&a.maps[6], Q, T, 3 * rp, 3 * rp, 128));
-    for (int x = 0; x < 3; ++x) set_seg(a, 3 + x, 6, x * rp, 7 + x, 0, -1, 0, rp);
-    a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
-    a.out[0] = dH; a.ld_out = d;
-    set_band(a, 4);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_QKV_DH)));
-    else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_QKV_DH)));
-  }
-  TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));
-  {
-    ZeroList z{};
-    for (int x = 0; x < 3; ++x) {
-      z.p[2 * x] = dAx[x]; z.n[2 * x] = static_cast<long long>(r) * d;
-      z.p[2 * x + 1] = dBx[x]; z.n[2 * x + 1] = static_cast<long long>(nx[x]) * r;
-    }
-    PhaseScope ps(st, PH_ZERO);
-    zero_grads_kernel<<<296, 256, 0, st>>>(z);
-    CUDA_TRY(cudaGetLastError());
-  }
-  const int rbn = r <= 64 ? 64 : 128;
-  // dA_x = Q_x^T H  ([r x d], written transposed from [d x r] tiles)
-  for (int x = 0; x < 3; ++x) {
-    GemmArgs a = new_args(status);
-    a.mn3d_a = d % 64 == 0;
-    if (a.mn3d_a) TRY(map_mn3(&a.maps[0], H, T, d, d, 2));
-    else TRY(map_mn(&a.maps[0], H, T, d, d));
-    TRY(map_mn(&a.maps[1], Q + static_cast<size_t>(x) * rp * 2, T, r, 3 * rp));
-    set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
-    a.M = d; a.N = r; a.bn = rbn; a.tiles_m = (d + BM - 1) / BM; a.tiles_n = 1;
-    a.rng[0] = OutRange{dAx[x], 0, 1, d};
-    a.nrng = 1;
-    choose_splits(a, T);
-    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_QKV_LOWRANK)));
-  }
-  // dB_x = dZ_x^T P_x  ([n_x x r])
-  for (int x = 0; x < 3; ++x) {
-    GemmArgs a = new_args(status);
-    a.mn3d_a = nx[x] % 64 == 0;
-    if (a.mn3d_a) TRY(map_mn3(&a.maps[0], dZ[x], T, nx[x], nx[x], 2));
-    else TRY(map_mn(&a.maps[0], dZ[x], T, nx[x], nx[x]));
-    TRY(map_mn(&a.maps[1], P + static_cast<size_t>(x) * rp * 2, T, r, 3 * rp));
-    set_seg(a, 0, 0, 0, 1, 0, -1, 0, static_cast<int>(T));
-    a.M = nx[x]; a.N = r; a.bn = rbn; a.tiles_m = (nx[x] + BM - 1) / BM; a.tiles_n = 1;
-    a.rng[0] = OutRange{dBx[x], 0, 0, r};
-    a.nrng = 1;
-    choose_splits(a, T);
-    TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_QKV_LOWRANK)));
-  }
-  return end_call(status, st);
 }
 
 }  // extern "C"

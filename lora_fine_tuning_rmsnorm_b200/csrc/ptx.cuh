@@ -13,6 +13,7 @@ enum DevErr : int {
   kDevTimeoutMma = 0x200,
   kDevTimeoutEpilogue = 0x300,
   kDevTimeoutDrain = 0x400,
+  kDevBadIndex = 0x500,  // a device-side index input (a position id) was out of range
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -85,7 +86,7 @@ struct WaitCtl {
 
 // Slow path of mbar_wait: sleep in suspend-hinted try_waits, checking the abort
 // flag and the time limit between them.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c, int code) {
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_test_sleep(bar, parity, 200000u)) return true;

@@ -31,7 +31,7 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 
 // VPT = 16-byte vectors (8 bf16) per thread; blockDim.x * VPT * 8 >= d.
 template <int VPT>
-__global__ void __launch_bounds__(1024) rmsnorm_fwd_kernel(const uint16_t* __restrict__ X,
+static __global__ void __launch_bounds__(1024) rmsnorm_fwd_kernel(const uint16_t* __restrict__ X,
                                                            const uint16_t* __restrict__ w,
                                                            uint16_t* __restrict__ H,
                                                            float* __restrict__ rstd, int d,
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_fwd_kernel(const uint16_t* __res
 
 // dX = rstd * (g - xhat * mean(g * xhat)), g = dH * w, xhat = x * rstd.
 template <int VPT>
-__global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restrict__ dH,
+static __global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restrict__ dH,
                                                            const uint16_t* __restrict__ X,
                                                            const uint16_t* __restrict__ w,
                                                            const float* __restrict__ rstd,
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restri
 // One warp per 64-element block: two elements per lane, absmax by warp max,
 // code index = number of midpoints the value exceeds (decided exactly: the sign of
 // a fused multiply-add w - absmax * m_i is the sign of the exact difference).
-__global__ void quantize4_kernel(const uint16_t* __restrict__ W, long long nblocks,
+static __global__ void quantize4_kernel(const uint16_t* __restrict__ W, long long nblocks,
                                  const float* __restrict__ code, uint8_t* __restrict__ codes,
                                  float* __restrict__ absmax) {
   __shared__ float mid[15];
@@ -165,7 +165,7 @@ __global__ void quantize4_kernel(const uint16_t* __restrict__ W, long long nbloc
 
 // out[i] = bf16(scale * sum_s part[s * stride + i]) for the K-split partial sums
 // of a rank-r projection (deterministic: fixed summation order).
-__global__ void splitk_finalize_kernel(const float* __restrict__ part, int splits, long long stride,
+static __global__ void splitk_finalize_kernel(const float* __restrict__ part, int splits, long long stride,
                                        long long n, float scale, uint16_t* __restrict__ out) {
   const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i4 >= n) return;
@@ -182,7 +182,7 @@ __global__ void splitk_finalize_kernel(const float* __restrict__ part, int split
 
 // The same sum of K-split partials, written into columns [0, cols) of an output with
 // row stride ld_out (a column block of a wider matrix).  cols is a multiple of 4.
-__global__ void splitk_finalize_strided_kernel(const float* __restrict__ part, int splits, long long stride,
+static __global__ void splitk_finalize_strided_kernel(const float* __restrict__ part, int splits, long long stride,
                                                long long rows, int cols, long long ld_out, float scale,
                                                uint16_t* __restrict__ out) {
   const long long i4 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
@@ -204,7 +204,7 @@ struct ZeroList {
   float* p[kZeroMax];  // NULL entries (n = 0) are skipped
   long long n[kZeroMax];
 };
-__global__ void zero_grads_kernel(ZeroList z) {
+static __global__ void zero_grads_kernel(ZeroList z) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (int k = 0; k < kZeroMax; ++k)
     for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < z.n[k]; i += stride)
@@ -214,7 +214,7 @@ __global__ void zero_grads_kernel(ZeroList z) {
 // Norm-weight gradient of H = X * rstd * w: dw_j += sum over a chunk of `rows` rows of
 // dH_tj * x_tj * rstd_t, added to dw (zeroed by the caller) with fp32 atomics.  A thread
 // owns 4 consecutive columns, so every row of dH / X is read coalesced.
-__global__ void __launch_bounds__(256) norm_weight_grad_kernel(const float* __restrict__ dH,
+static __global__ void __launch_bounds__(256) norm_weight_grad_kernel(const float* __restrict__ dH,
                                                                const uint16_t* __restrict__ X,
                                                                const float* __restrict__ rstd,
                                                                float* __restrict__ dw, long long T, int d,
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(256) norm_weight_grad_kernel(const float* __re
 // vector it loads serves 4 rows; the B values of the block's rows are shared by all of its
 // threads (broadcast loads).  W and Wm may alias: each element is read and written by
 // one thread only.
-__global__ void __launch_bounds__(128) merge_weights_kernel(const uint16_t* W, const uint16_t* __restrict__ A,
+static __global__ void __launch_bounds__(128) merge_weights_kernel(const uint16_t* W, const uint16_t* __restrict__ A,
                                                             const uint16_t* __restrict__ B, uint16_t* Wm,
                                                             long long rows, long long cols, int r, float s) {
   const long long j = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;

@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "lora_mlp.h")
 LORA_OK = 0
 ERRORS = {-1: "INVALID_ARG", -2: "ALIGNMENT", -3: "UNSUPPORTED", -4: "CUDA", -5: "TIMEOUT"}
 WFMT_BF16, WFMT_4BIT = 0, 1
-NUM_PHASES = 20
+NUM_PHASES = 28
 
 
 class LoraError(RuntimeError):
@@ -71,6 +71,19 @@ class QkvCtxLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("rstd", "H", "P", "total")] + [("rp", ctypes.c_int32)]
 
 
+class ODims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("n_in", ctypes.c_int32), ("n_out", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+class CeDims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("V", ctypes.c_int32), ("vocab_chunk", ctypes.c_int32),
+                ("reduction", ctypes.c_int32)]
+
+
+CE_MEAN, CE_SUM = 0, 1
+
+
 def header_functions() -> list[str]:
     """Names of the functions include/lora_mlp.h declares."""
     txt = open(HEADER).read()
@@ -110,6 +123,14 @@ def lib() -> ctypes.CDLL:
         "lora_gemm_bf16": [i64, i64, i64, vp, i32, vp, i32, vp, i32, vp],
         "lora_lowrank_proj_noalloc": [i64, i32, i32, f32, vp, vp, vp, vp],
         "lora_mlp_status": [vp, ctypes.POINTER(ctypes.c_int32), vp],
+        "lora_o_ctx_bytes": [ctypes.POINTER(ODims), ctypes.POINTER(ctypes.c_size_t)],
+        "lora_o_workspace_bytes": [ctypes.POINTER(ODims), ctypes.POINTER(ctypes.c_size_t)],
+        "lora_o_fwd": [ctypes.POINTER(ODims), vp, vp, vp, vp, vp, vp, vp, vp],
+        "lora_o_bwd": [ctypes.POINTER(ODims), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "lora_rope": [i64, i32, i32, i32, vp, i64, vp, vp, vp, vp, i32, vp],
+        "lora_ce_workspace_bytes": [ctypes.POINTER(CeDims), ctypes.POINTER(ctypes.c_size_t)],
+        "lora_ce_fwd": [ctypes.POINTER(CeDims), vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "lora_ce_bwd": [ctypes.POINTER(CeDims), vp, vp, vp, vp, vp, f32, vp, vp, vp],
         "lora_mlp_timing_enable": [i32],
         "lora_mlp_timing_collect": [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)],
     }
@@ -308,3 +329,62 @@ def lora_qkv_bwd(dims: QkvDims, dQ, dK, dV, X, rms_w, weights: QkvWeights, adapt
     _check(lib().lora_qkv_bwd(ctypes.byref(dims), _p(dQ), _p(dK), _p(dV), _p(X), _p(rms_w), ctypes.byref(weights),
                               ctypes.byref(adapters), _p(ctx), _p(dX), ctypes.byref(grads), _p(workspace),
                               _stream(stream)))
+
+
+# ------------------------------------------------------------------ o_proj LoRA linear
+def o_dims(T, n_in, n_out, r, scale=1.0) -> ODims:
+    return ODims(T, n_in, n_out, r, scale)
+
+
+def o_ctx_bytes(dims: ODims) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().lora_o_ctx_bytes(ctypes.byref(dims), ctypes.byref(out)))
+    return out.value
+
+
+def o_workspace_bytes(dims: ODims) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().lora_o_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)))
+    return out.value
+
+
+def lora_o_fwd(dims: ODims, X, Wo, Ao, Bo, Y, ctx, workspace, stream=None):
+    _check(lib().lora_o_fwd(ctypes.byref(dims), _p(X), _p(Wo), _p(Ao), _p(Bo), _p(Y), _p(ctx), _p(workspace),
+                            _stream(stream)))
+
+
+def lora_o_bwd(dims: ODims, dY, X, Wo, Ao, Bo, ctx, dX, dAo, dBo, workspace, stream=None):
+    _check(lib().lora_o_bwd(ctypes.byref(dims), _p(dY), _p(X), _p(Wo), _p(Ao), _p(Bo), _p(ctx), _p(dX), _p(dAo),
+                            _p(dBo), _p(workspace), _stream(stream)))
+
+
+# ------------------------------------------------------------------ RoPE
+def lora_rope(Q, K, pos, cos, sin, hd, backward=False, stream=None):
+    """Rotate Q [T x hq hd] and K [T x hk hd] (bf16, in place) at positions pos [T] int32
+    with the fp32 tables cos, sin [n_pos x hd/2]; backward applies the inverse rotation."""
+    T = pos.shape[0]
+    hq = 0 if Q is None else Q.shape[1] // hd
+    hk = 0 if K is None else K.shape[1] // hd
+    _check(lib().lora_rope(T, hq, hk, hd, _p(pos), cos.shape[0], _p(cos), _p(sin), _p(Q), _p(K),
+                           1 if backward else 0, _stream(stream)))
+
+
+# ------------------------------------------------------------------ LM-head cross-entropy
+def ce_dims(T, d, V, vocab_chunk=0, reduction=CE_MEAN) -> CeDims:
+    return CeDims(T, d, V, vocab_chunk, reduction)
+
+
+def ce_workspace_bytes(dims: CeDims) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().lora_ce_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)))
+    return out.value
+
+
+def lora_ce_fwd(dims: CeDims, H, W, labels, loss_rows, lse, loss, n_valid, workspace, stream=None):
+    _check(lib().lora_ce_fwd(ctypes.byref(dims), _p(H), _p(W), _p(labels), _p(loss_rows), _p(lse), _p(loss),
+                             _p(n_valid), _p(workspace), _stream(stream)))
+
+
+def lora_ce_bwd(dims: CeDims, H, W, labels, lse, n_valid, dloss, dH, workspace, stream=None):
+    _check(lib().lora_ce_bwd(ctypes.byref(dims), _p(H), _p(W), _p(labels), _p(lse), _p(n_valid), float(dloss),
+                             _p(dH), _p(workspace), _stream(stream)))

@@ -174,3 +174,88 @@ class QkvProblem:
     def step(self, stream=None):
         self.forward(stream)
         self.backward(stream)
+
+
+class OProblem:
+    """All device buffers of one o_proj LoRA-linear fwd+bwd step for an OShape."""
+
+    def __init__(self, shape: synth.OShape, bits: dict | None = None, seed: int = synth.BASE_SEED, device="cuda"):
+        self.shape = s = shape
+        bits = bits if bits is not None else synth.make_o_inputs_bits(s, seed)
+        self.t = {k: bf16_tensor(v, device) for k, v in bits.items()}
+        self.dims = ops.o_dims(s.T, s.n_in, s.n_out, s.r, scale=s.scale)
+        self.Y = torch.empty(s.T, s.n_out, dtype=torch.bfloat16, device=device)
+        self.dX = torch.empty(s.T, s.n_in, dtype=torch.bfloat16, device=device)
+        self.dAo = torch.empty(s.r, s.n_in, dtype=torch.float32, device=device)
+        self.dBo = torch.empty(s.n_out, s.r, dtype=torch.float32, device=device)
+        self.ctx = torch.empty(ops.o_ctx_bytes(self.dims), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(ops.o_workspace_bytes(self.dims), dtype=torch.uint8, device=device)
+
+    def forward(self, stream=None):
+        t = self.t
+        ops.lora_o_fwd(self.dims, t["X"], t["Wo"], t["Ao"], t["Bo"], self.Y, self.ctx, self.ws, stream)
+
+    def backward(self, stream=None):
+        t = self.t
+        ops.lora_o_bwd(self.dims, t["dY"], t["X"], t["Wo"], t["Ao"], t["Bo"], self.ctx, self.dX, self.dAo, self.dBo,
+                       self.ws, stream)
+
+    def step(self, stream=None):
+        self.forward(stream)
+        self.backward(stream)
+
+
+class RopeProblem:
+    """Device buffers of one RoPE forward (Q, K in place) + backward (dQ, dK in place)."""
+
+    def __init__(self, shape: synth.RopeShape, data: dict | None = None, seed: int = synth.BASE_SEED,
+                 device="cuda"):
+        self.shape = s = shape
+        data = data if data is not None else synth.make_rope_inputs(s, seed)
+        self.t = {k: bf16_tensor(data[k], device) for k in ("Q", "K", "dQ", "dK")}
+        self.pos = torch.from_numpy(np.ascontiguousarray(data["pos"], dtype=np.int32)).to(device)
+        self.cos = torch.from_numpy(np.ascontiguousarray(data["cos"], dtype=np.float32)).to(device)
+        self.sin = torch.from_numpy(np.ascontiguousarray(data["sin"], dtype=np.float32)).to(device)
+
+    def forward(self, stream=None):
+        ops.lora_rope(self.t["Q"], self.t["K"], self.pos, self.cos, self.sin, self.shape.hd, False, stream)
+
+    def backward(self, stream=None):
+        ops.lora_rope(self.t["dQ"], self.t["dK"], self.pos, self.cos, self.sin, self.shape.hd, True, stream)
+
+    def step(self, stream=None):
+        self.forward(stream)
+        self.backward(stream)
+
+
+class CeProblem:
+    """Device buffers of one fused LM-head cross-entropy forward + backward for a CeShape."""
+
+    def __init__(self, shape: synth.CeShape, data: dict | None = None, seed: int = synth.BASE_SEED, device="cuda",
+                 vocab_chunk: int = 0, reduction: int = ops.CE_MEAN, dloss: float = 1.0):
+        self.shape = s = shape
+        data = data if data is not None else synth.make_ce_inputs(s, seed)
+        self.H = bf16_tensor(data["H"], device)
+        self.W = bf16_tensor(data["W"], device)
+        self.labels = torch.from_numpy(np.ascontiguousarray(data["labels"], dtype=np.int32)).to(device)
+        self.dims = ops.ce_dims(s.T, s.d, s.V, vocab_chunk, reduction)
+        self.dloss = dloss
+        self.loss_rows = torch.empty(s.T, dtype=torch.float32, device=device)
+        self.lse = torch.empty(s.T, dtype=torch.float32, device=device)
+        self.stats = torch.zeros(4, dtype=torch.int32, device=device)   # [0] loss (fp32 bits), [1] n_valid
+        self.loss = self.stats[0:1].view(torch.float32)
+        self.n_valid = self.stats[1:2]
+        self.dH = torch.empty(s.T, s.d, dtype=torch.float32, device=device)
+        self.ws = torch.empty(ops.ce_workspace_bytes(self.dims), dtype=torch.uint8, device=device)
+
+    def forward(self, stream=None):
+        ops.lora_ce_fwd(self.dims, self.H, self.W, self.labels, self.loss_rows, self.lse, self.loss, self.n_valid,
+                        self.ws, stream)
+
+    def backward(self, stream=None):
+        ops.lora_ce_bwd(self.dims, self.H, self.W, self.labels, self.lse, self.n_valid, self.dloss, self.dH, self.ws,
+                        stream)
+
+    def step(self, stream=None):
+        self.forward(stream)
+        self.backward(stream)

@@ -152,3 +152,39 @@ def test_gemm_flags_and_status_argument_checks(L):
     assert b"single-CTA" in L.lora_mlp_last_error()
     code = ctypes.c_int32(0)
     assert L.lora_mlp_status(ctypes.c_void_p(0x1004), ctypes.byref(code), None) == -2  # misaligned workspace
+
+
+def test_o_proj_and_rope_argument_checks(L):
+    out = ctypes.c_size_t()
+    good = ctypes.c_void_p(0x1000)
+    for bad, code in (((64, 130, 64, 8), -2), ((0, 128, 64, 8), -1), ((64, 128, 64, 136), -3), ((64, 128, 0, 8), -1)):
+        assert L.lora_o_workspace_bytes(ctypes.byref(ops.o_dims(*bad)), ctypes.byref(out)) == code, bad
+    dims = ops.o_dims(8192, 4096, 4096, 16)
+    assert ops.o_ctx_bytes(dims) >= 8192 * 16 * 2
+    assert ops.o_workspace_bytes(dims) >= 256 + 8192 * 16 * 2
+    assert L.lora_o_fwd(ctypes.byref(dims), good, None, good, good, good, good, good, None) == -1
+    assert L.lora_o_bwd(ctypes.byref(dims), good, good, good, good, good, good, good, good, ctypes.c_void_p(0x1008),
+                        good, None) == -2
+    # rope: hd a multiple of 16, head counts, pointers
+    assert L.lora_rope(16, 2, 1, 24, good, 16, good, good, good, good, 0, None) == -2
+    assert L.lora_rope(16, 0, 0, 64, good, 16, good, good, good, good, 0, None) == -1
+    assert L.lora_rope(16, 2, 1, 64, good, 16, good, good, good, good, 2, None) == -1
+    assert L.lora_rope(16, 2, 1, 64, None, 16, good, good, good, good, 0, None) == -1
+    assert L.lora_rope(16, 2, 1, 64, good, 16, good, good, good, None, 0, None) == -1   # K needed when hk > 0
+
+
+def test_ce_argument_checks(L):
+    out = ctypes.c_size_t()
+    good = ctypes.c_void_p(0x1000)
+    for bad, code in (((64, 130, 344), -2), ((64, 128, 340), -2), ((0, 128, 344), -1), ((64, 4, 344), -1)):
+        assert L.lora_ce_workspace_bytes(ctypes.byref(ops.ce_dims(*bad)), ctypes.byref(out)) == code, bad
+    assert L.lora_ce_workspace_bytes(ctypes.byref(ops.ce_dims(64, 128, 344, vocab_chunk=100)), ctypes.byref(out)) == -1
+    assert L.lora_ce_workspace_bytes(ctypes.byref(ops.ce_dims(64, 128, 344, reduction=2)), ctypes.byref(out)) == -1
+    big = ops.ce_workspace_bytes(ops.ce_dims(8192, 4096, 128256))
+    assert big >= 8192 * 32768 * 2                         # one vocabulary chunk of dZ (bf16)
+    assert ops.ce_workspace_bytes(ops.ce_dims(8192, 4096, 128256, vocab_chunk=8192)) < big
+    dims = ops.ce_dims(64, 128, 344)
+    assert L.lora_ce_fwd(ctypes.byref(dims), good, good, good, good, good, ctypes.c_void_p(0x1002), good, good,
+                         None) == -2                        # loss not 4-byte aligned
+    assert L.lora_ce_fwd(ctypes.byref(dims), good, None, good, good, good, good, good, good, None) == -1
+    assert L.lora_ce_bwd(ctypes.byref(dims), good, good, good, good, good, float("nan"), good, good, None) == -1
