@@ -32,10 +32,10 @@ TENSOR_ORDER = ("X", "w", "Wg", "Wu", "Wd", "Ag", "Bg", "Au", "Bu", "Ad", "Bd", 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round-to-nearest-even), returned as uint16 bits."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
+    u = a.view(np.uint32)
+    # u + 0x7FFF + lsb stays below 2^32 for every non-NaN pattern (at most 0xFF80_7FFF)
+    r = ((u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(a)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
     if nan.any():
         r[nan] = 0x7FC0
     return r

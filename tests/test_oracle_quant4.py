@@ -120,3 +120,66 @@ def test_stored_codebook_is_the_oracles():
     from tests.parity import load_codebook
     np.testing.assert_array_equal(np.asarray(load_codebook(), dtype=np.float64),
                                   q4.codebook16().astype(np.float64))
+
+
+# ------------------------------------------------------------ double quantisation of absmax
+def _absmax_sample(n=1000, seed=3):
+    rng = np.random.default_rng(seed)
+    a = np.abs(rng.standard_normal(n)).astype(np.float32) * np.float32(0.05)
+    a[17] = 0.0
+    a[300:556] = 0.0                  # one whole second-level block of zeros
+    return a
+
+
+def test_absmax8_rule_in_exact_rational_arithmetic():
+    a = _absmax_sample(600)
+    codes, s2 = q4.quantize_absmax8(a)
+    for i in range(0, 600, 7):
+        s = Fraction(float(s2[i // 256]))
+        x = Fraction(float(a[i]))
+        # the nearest level s k / 255, ties to the lower one
+        best = min(range(256), key=lambda k: (abs(x - s * k / 255), k))
+        assert codes[i] == best, (i, codes[i], best)
+
+
+def test_absmax8_block_max_gets_255_and_zero_blocks_give_zero():
+    a = _absmax_sample()
+    codes, s2 = q4.quantize_absmax8(a)
+    assert s2.size == 4 and s2[1] >= 0
+    for b in range(4):
+        blk = a[b * 256:(b + 1) * 256]
+        if blk.max() > 0:
+            assert codes[b * 256 + int(np.argmax(blk))] == 255
+    assert np.all(codes[300:556][a[300:556] == 0] == 0)
+    zero_block = np.zeros(256, dtype=np.float32)
+    c0, s0 = q4.quantize_absmax8(zero_block)
+    assert s0[0] == 0 and np.all(c0 == 0)
+
+
+def test_absmax8_error_bound_and_idempotence():
+    a = _absmax_sample(2000, 9)
+    codes, s2 = q4.quantize_absmax8(a)
+    ahat = q4.dequantize_absmax8(codes, s2)
+    s = np.repeat(s2.astype(np.float64), 256)[:a.size]
+    assert np.all(np.abs(ahat - a.astype(np.float64)) <= s / 510.0 * (1 + 1e-12))
+    # re-quantising the levels themselves (rounded to fp32) returns the same codes
+    codes2, s22 = q4.quantize_absmax8(ahat.astype(np.float32))
+    np.testing.assert_array_equal(s22, s2)
+    np.testing.assert_array_equal(codes2, codes)
+
+
+def test_absmax8_ties_go_to_the_lower_level():
+    s = np.float32(1.0)
+    # a constant exactly halfway between levels 3/255 and 4/255 (3.5/255 = 7/510) when representable:
+    a = np.array([s, np.float32(7.0 / 510.0)], dtype=np.float32)
+    codes, _ = q4.quantize_absmax8(a)
+    x = Fraction(float(a[1]))
+    if x == Fraction(7, 510):
+        assert codes[1] == 3
+    else:   # not representable: nearest level by exact comparison
+        assert codes[1] == (4 if x > Fraction(7, 510) else 3)
+    # exact ties by construction: scale2 = 510 * 2^-k makes 510 a = (2j - 1) scale2 representable
+    s = np.float32(510.0)
+    a = np.array([s] + [np.float32(2 * j - 1) for j in (1, 2, 100, 255)], dtype=np.float32)
+    codes, _ = q4.quantize_absmax8(a)
+    np.testing.assert_array_equal(codes, [255, 0, 1, 99, 254])
