@@ -133,8 +133,27 @@ struct GemmArgs {
   int ce_V;               // vocabulary size
 };
 
+// Tile-scheduling constants, copied out of the launch parameters once per role: every
+// inline-asm statement in the role loops clobbers memory, so a field read inside a loop
+// would be re-read from the parameter space (through the small constant cache) on every
+// iteration, on the critical path from "stage freed" to "copy issued".
+struct Sched {
+  int tiles_m, tiles_n, splits, raster, group_m, k_chunk, total;
+};
+__device__ __forceinline__ Sched sched_of(const GemmArgs& p) {
+  Sched s;
+  s.tiles_m = p.tiles_m;
+  s.tiles_n = p.tiles_n;
+  s.splits = p.splits;
+  s.raster = p.raster;
+  s.group_m = p.group_m;
+  s.k_chunk = p.k_chunk;
+  s.total = p.tiles_m * p.tiles_n * p.splits;
+  return s;
+}
+
 // Work unit u (a CTA, or a CTA pair when PAIR = 2) -> tile coordinates.
-__device__ __forceinline__ void decode_tile(const GemmArgs& p, int t, int& mt, int& nt, int& ks) {
+__device__ __forceinline__ void decode_tile(const Sched& p, int t, int& mt, int& nt, int& ks) {
   if (p.raster == 2) {
     // a band of group_m row tiles stays in L2 while the wave sweeps the N tiles
     const int per_split = p.tiles_m * p.tiles_n;
@@ -159,8 +178,9 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& p, int t, int& mt, i
   }
 }
 
-__device__ __forceinline__ void seg_kb_range(const GemmArgs& p, int s, int ks, int& lo, int& hi) {
-  const int nkb = (p.seg[s].k_len + BK - 1) / BK;
+// k-block range [lo, hi) of a segment of k_len elements in K split ks.
+__device__ __forceinline__ void seg_kb_range(const Sched& p, int k_len, int ks, int& lo, int& hi) {
+  const int nkb = (k_len + BK - 1) / BK;
   if (p.splits > 1) {
     const int per = p.k_chunk / BK;
     lo = ks * per;
@@ -170,6 +190,19 @@ __device__ __forceinline__ void seg_kb_range(const GemmArgs& p, int s, int ks, i
     hi = nkb;
   }
 }
+
+// One segment's launch constants in registers (see Sched).
+struct SegR {
+  int a_map, a_k0, b_map0, b_map1, b_k00, b_k01, k_len, a_hint, b_hint, q4, b_am0, b_am1;
+};
+__device__ __forceinline__ SegR seg_of(const GemmArgs& p, int s) {
+  const Seg& g = p.seg[s];
+  return SegR{g.a_map, g.a_k0, g.b_map[0], g.b_map[1], g.b_k0[0], g.b_k0[1], g.k_len, g.a_hint, g.b_hint,
+              g.q4, g.b_am[0], g.b_am[1]};
+}
+__device__ __forceinline__ int seg_bmap(const SegR& g, int a) { return a ? g.b_map1 : g.b_map0; }
+__device__ __forceinline__ int seg_bk0(const SegR& g, int a) { return a ? g.b_k01 : g.b_k00; }
+__device__ __forceinline__ int seg_bam(const SegR& g, int a) { return a ? g.b_am1 : g.b_am0; }
 
 // Drain wait used after an abort: ignores the abort flag, bounded by the limit.
 static __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, const WaitCtl& c) {
@@ -188,9 +221,14 @@ static __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, co
 template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                               uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
-  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const Sched sc = sched_of(p);
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
-  const int bnl = p.bn / PAIR;  // B rows (N) held by this CTA
+  // launch constants in registers (see Sched)
+  const int M = p.M, N = p.N, bn = p.bn, nstages = p.stages, nseg = p.nseg;
+  const int mn3d_a = p.mn3d_a, mn3d_b = p.mn3d_b, no_loads = p.test_no_loads;
+  const uint32_t stage_bytes = p.stage_bytes;
+  const CUtensorMap* maps = p.maps;
+  const int bnl = bn / PAIR;  // B rows (N) held by this CTA
   int stage = 0;
   uint32_t phase = 0;
   uint32_t issued_mask = 0, issued_par = 0;
@@ -198,49 +236,52 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   const uint32_t b_bytes = static_cast<uint32_t>(bnl) * BK * 2;
   const uint64_t pol_first = policy_evict_first(), pol_last = policy_evict_last();
   bool ok = true;
-  for (int t = unit0; t < total && ok; t += nunits) {
+  for (int t = unit0; t < sc.total && ok; t += nunits) {
     int mt, nt, ks;
-    decode_tile(p, t, mt, nt, ks);
-    const int mbase = mt * BM * PAIR, n0 = nt * p.bn;
-    for (int s = 0; s < p.nseg && ok; ++s) {
-      const Seg& sg = p.seg[s];
+    decode_tile(sc, t, mt, nt, ks);
+    const int mbase = mt * BM * PAIR, n0 = nt * bn;
+    for (int s = 0; s < nseg && ok; ++s) {
+      const SegR sg = seg_of(p, s);
       int kb0, kb1;
-      seg_kb_range(p, s, ks, kb0, kb1);
+      seg_kb_range(sc, sg.k_len, ks, kb0, kb1);
       // Bytes landing per stage for CTA rank rr.  Boxes that would lie entirely
       // outside the matrix are skipped: the rows / columns they feed are never stored.
       auto bytes_of = [&](uint32_t rr) -> uint32_t {
         const int m0r = mbase + static_cast<int>(rr) * BM;
         uint32_t by = 0;
-        if (A_MN) by += p.mn3d_a ? (m0r < p.M ? 16384u : 0u) : (m0r < p.M ? 8192u : 0u) + (m0r + 64 < p.M ? 8192u : 0u);
-        else by += (m0r < p.M ? a_bytes : 0u);
+        if (A_MN) by += mn3d_a ? (m0r < M ? 16384u : 0u) : (m0r < M ? 8192u : 0u) + (m0r + 64 < M ? 8192u : 0u);
+        else by += (m0r < M ? a_bytes : 0u);
         const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rr) * bnl;
         uint32_t bb = 0;
         if (B_MN) {
-          if (p.mn3d_b) {
-            bb = nb0 < p.N ? b_bytes : 0u;
+          if (mn3d_b) {
+            bb = nb0 < N ? b_bytes : 0u;
           } else {
             for (int c = 0; c < bnl / 64; ++c)
-              if (nb0 + 64 * c < p.N) bb += 8192u;
+              if (nb0 + 64 * c < N) bb += 8192u;
           }
         } else {
-          bb = nb0 < p.N ? b_bytes : 0u;
+          bb = nb0 < N ? b_bytes : 0u;
         }
         if (!(Q4 && sg.q4)) {  // 4-bit B is written by the dequant warps instead
 #pragma unroll
           for (int a = 0; a < NACC; ++a)
-            if (sg.b_map[a] >= 0) by += bb;
+            if (seg_bmap(sg, a) >= 0) by += bb;
         }
         return by;
       };
       const uint32_t stage_tx = PAIR == 1 ? bytes_of(0) : (rank == 0 ? bytes_of(0) + bytes_of(1) : 0u);
+      const int m0 = mbase + static_cast<int>(rank) * BM;
+      const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rank) * bnl;
+      const CUtensorMap* am = maps + sg.a_map;
       for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t full = full0 + 8 * stage, empty = empty0 + 8 * stage;
         if (!mbar_wait(empty, phase ^ 1, wc, kDevTimeoutProducer)) {
           ok = false;
           break;
         }
-        if (p.test_no_loads) {  // nothing issued, nothing armed: no copy can be in flight
-          if (++stage == p.stages) {
+        if (no_loads) {  // nothing issued, nothing armed: no copy can be in flight
+          if (++stage == nstages) {
             stage = 0;
             phase ^= 1;
           }
@@ -248,11 +289,8 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         }
         if (stage_tx) mbar_expect_tx(full, stage_tx);
         const uint32_t bar = PAIR == 1 ? full : mapa_shared(full, 0);
-        const int m0 = mbase + static_cast<int>(rank) * BM;
-        const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rank) * bnl;
-        const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * p.stage_bytes);
+        const uint32_t sA = smem_u32(tiles + static_cast<size_t>(stage) * stage_bytes);
         const int k = kb * BK;
-        const CUtensorMap* am = &p.maps[sg.a_map];
         int hint = sg.a_hint;
         auto load = [&](uint32_t dst, const CUtensorMap* m, int x, int y) {
           if (hint == HINT_NONE) {
@@ -269,12 +307,12 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
           if (PAIR == 1) tma_load_3d(dst, m, bar, 0, y, z);
           else tma_load_3d_pair(dst, m, bar, 0, y, z);
         };
-        if (A_MN && p.mn3d_a) {
-          if (m0 < p.M) load3(sA, am, sg.a_k0 + k, m0 / 64);
+        if (A_MN && mn3d_a) {
+          if (m0 < M) load3(sA, am, sg.a_k0 + k, m0 / 64);
         } else if (A_MN) {
-          if (m0 < p.M) load(sA, am, m0, sg.a_k0 + k);
-          if (m0 + 64 < p.M) load(sA + 8192, am, m0 + 64, sg.a_k0 + k);
-        } else if (m0 < p.M) {
+          if (m0 < M) load(sA, am, m0, sg.a_k0 + k);
+          if (m0 + 64 < M) load(sA + 8192, am, m0 + 64, sg.a_k0 + k);
+        } else if (m0 < M) {
           load(sA, am, sg.a_k0 + k, m0);
         }
         hint = sg.b_hint;
@@ -287,28 +325,28 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             if (PAIR == 2 && static_cast<uint32_t>(r) != rank) continue;
-            const uint32_t dst = PAIR == 2 ? sB : sB + r * p.bn * BK * 2;
-            load(dst, &p.maps[sg.b_map[r]], sg.b_k0[r] + k, n0);
+            const uint32_t dst = PAIR == 2 ? sB : sB + r * bn * BK * 2;
+            load(dst, maps + seg_bmap(sg, r), seg_bk0(sg, r) + k, n0);
           }
         } else {
 #pragma unroll
           for (int a = 0; a < NACC; ++a) {
-            if (sg.b_map[a] < 0) continue;
+            if (seg_bmap(sg, a) < 0) continue;
             const uint32_t sB = sA + a_bytes + a * b_bytes;
-            const CUtensorMap* bm = &p.maps[sg.b_map[a]];
-            if (B_MN && p.mn3d_b) {
-              if (nb0 < p.N) load3(sB, bm, sg.b_k0[a] + k, nb0 / 64);
+            const CUtensorMap* bm = maps + seg_bmap(sg, a);
+            if (B_MN && mn3d_b) {
+              if (nb0 < N) load3(sB, bm, seg_bk0(sg, a) + k, nb0 / 64);
             } else if (B_MN) {
               for (int c = 0; c < bnl / 64; ++c)
-                if (nb0 + 64 * c < p.N) load(sB + c * 8192, bm, nb0 + 64 * c, sg.b_k0[a] + k);
-            } else if (nb0 < p.N) {
-              load(sB, bm, sg.b_k0[a] + k, nb0);
+                if (nb0 + 64 * c < N) load(sB + c * 8192, bm, nb0 + 64 * c, seg_bk0(sg, a) + k);
+            } else if (nb0 < N) {
+              load(sB, bm, seg_bk0(sg, a) + k, nb0);
             }
           }
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == p.stages) {
+        if (++stage == nstages) {
           stage = 0;
           phase ^= 1;
         }
@@ -318,7 +356,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   if (!ok) {
     // Aborting: make sure no TMA write into shared memory is still in flight (the
     // even CTA's full barriers also count the odd CTA's bytes).
-    for (int s = 0; s < p.stages; ++s) {
+    for (int s = 0; s < nstages; ++s) {
       if (!(issued_mask & (1u << s))) continue;
       if (rank == 0) drain_wait(full0 + 8 * s, (issued_par >> s) & 1, wc);
     }
@@ -330,7 +368,8 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
                                          uint32_t empty0, uint32_t tfull0, uint32_t tempty0,
                                          uint32_t drain_bar, uint32_t tmem_base,
                                          const WaitCtl& wc, uint32_t dq0) {
-  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const Sched sc = sched_of(p);
+  const int total = sc.total;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const uint32_t idesc = idesc_bf16(BM * PAIR, FUSE ? 2 * p.bn : p.bn, A_MN, B_MN);
   const uint32_t a_bytes = BM * BK * 2;
@@ -347,7 +386,7 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
   bool ready = false;  // the current stage's full barrier was seen complete by a peek
   for (int t = unit0; t < total && ok; t += nunits, ++it) {
     int mt, nt, ks;
-    decode_tile(p, t, mt, nt, ks);
+    decode_tile(sc, t, mt, nt, ks);
     const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
     if (!mbar_wait(tempty0 + 8 * buf, aphase ^ 1, wc, kDevTimeoutMma)) {
       ok = false;
@@ -356,14 +395,14 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
     tc_fence_after();
     uint32_t started = 0;
     for (int s = 0; s < nseg && ok; ++s) {
-      const Seg& sg = p.seg[s];
+      const SegR sg = seg_of(p, s);
       int kb0, kb1;
-      seg_kb_range(p, s, ks, kb0, kb1);
+      seg_kb_range(sc, sg.k_len, ks, kb0, kb1);
       const int k_len = sg.k_len;
       uint32_t bmask = 0;  // accumulators this segment feeds
 #pragma unroll
       for (int a = 0; a < NACC; ++a)
-        if (sg.b_map[a] >= 0) bmask |= 1u << a;
+        if (seg_bmap(sg, a) >= 0) bmask |= 1u << a;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!ready && !mbar_wait(full0 + 8 * stage, phase, wc, kDevTimeoutMma)) {
           ok = false;
@@ -455,62 +494,78 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int q = warp & 3;             // TMEM lane quarter this warp may access
   const int c0 = ((warp - 2) >> 2) * 16;  // first 16-column chunk of this warp; stride 32
-  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const Sched sc = sched_of(p);
+  const int total = sc.total;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
+  // launch constants in registers (see Sched)
+  const int bn = p.bn, N = p.N, M = p.M, stream_out = p.stream_out, out_acc_col = p.out_acc_col;
+  const int out_add = p.out_add, nrng = p.nrng;
+  const float alpha = p.alpha;
+  const long long ld_out = p.ld_out, ld_in = p.ld_in, split_stride = p.split_stride;
+  void* const out0 = p.out[0];
+  void* const out1 = p.out[1];
+  void* const out2 = p.out[2];
+  const void* const in0 = p.in[0];
+  const void* const in1 = p.in[1];
+  const int* const ce_labels = p.ce_labels;
+  const float* const ce_lse = p.ce_lse;
+  const int* const ce_count = p.ce_count;
+  const float ce_g = p.ce_g;
+  const int ce_col0 = p.ce_col0, ce_V = p.ce_V;
   uint32_t it = 0;
   for (int t = unit0; t < total; t += nunits, ++it) {
     int mt, nt, ks;
-    decode_tile(p, t, mt, nt, ks);
+    decode_tile(sc, t, mt, nt, ks);
     const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
     int ok = 1;
     if (lane == 0) ok = mbar_wait(tfull0 + 8 * buf, aphase, wc, kDevTimeoutEpilogue) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) break;
     tc_fence_after();
-    const int m0 = mt * BM * PAIR + static_cast<int>(rank) * BM, n0 = nt * p.bn;
+    const int m0 = mt * BM * PAIR + static_cast<int>(rank) * BM, n0 = nt * bn;
     const long long row = static_cast<long long>(m0) + 32 * q + lane;
-    const bool row_ok = row < p.M;
-    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (NACC * p.bn);
+    const bool row_ok = row < M;
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (NACC * bn);
 
     if (EPI == EPI_F32 || EPI == EPI_BF16) {
 #pragma unroll 1
       for (int a = 0; a < NACC; ++a) {
 #pragma unroll 1
-        for (int c = c0; c < p.bn; c += 32) {
+        for (int c = c0; c < bn; c += 32) {
           uint32_t r[16];
-          tmem_ld16(tbase + a * p.bn + c, r);
+          tmem_ld16(tbase + a * bn + c, r);
           tmem_wait16(r);
           const int n = n0 + c;
           if (!row_ok) continue;
           if (EPI == EPI_F32) {
-            float* o = static_cast<float*>(p.out[0]) + ks * p.split_stride + row * p.ld_out +
-                       a * p.out_acc_col + n;
+            float* o = static_cast<float*>(out0) + ks * split_stride + row * ld_out +
+                       a * out_acc_col + n;
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              if (n + 4 * h < p.N) {
-                float4 v = make_float4(__uint_as_float(r[4 * h]) * p.alpha,
-                                       __uint_as_float(r[4 * h + 1]) * p.alpha,
-                                       __uint_as_float(r[4 * h + 2]) * p.alpha,
-                                       __uint_as_float(r[4 * h + 3]) * p.alpha);
-                if (p.out_add) {
+              if (n + 4 * h < N) {
+                float4 v = make_float4(__uint_as_float(r[4 * h]) * alpha,
+                                       __uint_as_float(r[4 * h + 1]) * alpha,
+                                       __uint_as_float(r[4 * h + 2]) * alpha,
+                                       __uint_as_float(r[4 * h + 3]) * alpha);
+                if (out_add) {
                   const float4 old = *reinterpret_cast<const float4*>(o + 4 * h);
                   v.x += old.x; v.y += old.y; v.z += old.z; v.w += old.w;
                 }
-                st_out(reinterpret_cast<float4*>(o + 4 * h), v, p.stream_out);
+                st_out(reinterpret_cast<float4*>(o + 4 * h), v, stream_out);
               }
             }
           } else {
-            uint16_t* o = static_cast<uint16_t*>(p.out[0]) + row * p.ld_out + a * p.out_acc_col + n;
+            uint16_t* o = static_cast<uint16_t*>(out0) + row * ld_out + a * out_acc_col + n;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              if (n + 8 * h < p.N) {
+              if (n + 8 * h < N) {
                 float v8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(r[8 * h + e]) * p.alpha;
-                if (p.in[0]) {  // residual input (bf16, same layout as the output) added in fp32
+                for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(r[8 * h + e]) * alpha;
+                if (in0) {  // residual input (bf16, same layout as the output) added in fp32
                   float x8[8];
-                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.in[0]) +
-                                                                       row * p.ld_in + n + 8 * h));
+                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in0) +
+                                                                       row * ld_in + n + 8 * h));
                   x8[0] = bf16lo(xv.x); x8[1] = bf16hi(xv.x); x8[2] = bf16lo(xv.y); x8[3] = bf16hi(xv.y);
                   x8[4] = bf16lo(xv.z); x8[5] = bf16hi(xv.z); x8[6] = bf16lo(xv.w); x8[7] = bf16hi(xv.w);
 #pragma unroll
@@ -521,7 +576,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
                 v.y = pack_bf16x2(v8[2], v8[3]);
                 v.z = pack_bf16x2(v8[4], v8[5]);
                 v.w = pack_bf16x2(v8[6], v8[7]);
-                st_out(reinterpret_cast<uint4*>(o + 8 * h), v, p.stream_out);
+                st_out(reinterpret_cast<uint4*>(o + 8 * h), v, stream_out);
               }
             }
           }
@@ -529,17 +584,17 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       }
     } else if (EPI == EPI_SWIGLU_FWD) {
 #pragma unroll 1
-      for (int c = c0; c < p.bn; c += 32) {
+      for (int c = c0; c < bn; c += 32) {
         uint32_t rg[16], ru[16];
         tmem_ld16(tbase + c, rg);
-        tmem_ld16(tbase + p.bn + c, ru);
+        tmem_ld16(tbase + bn + c, ru);
         tmem_wait32(rg, ru);
         const int n = n0 + c;
         if (!row_ok) continue;
-        const long long off = row * p.ld_out + n;
+        const long long off = row * ld_out + n;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (n + 8 * h >= p.N) continue;
+          if (n + 8 * h >= N) continue;
           uint32_t pg[4], pu[4], pa[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -549,22 +604,22 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             pu[j] = pack_bf16x2(u0, u1);
             pa[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
           }
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h), make_uint4(pg[0], pg[1], pg[2], pg[3]), p.stream_out);
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h), make_uint4(pu[0], pu[1], pu[2], pu[3]), p.stream_out);
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[2]) + off + 8 * h), make_uint4(pa[0], pa[1], pa[2], pa[3]), p.stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out0) + off + 8 * h), make_uint4(pg[0], pg[1], pg[2], pg[3]), stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out1) + off + 8 * h), make_uint4(pu[0], pu[1], pu[2], pu[3]), stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out2) + off + 8 * h), make_uint4(pa[0], pa[1], pa[2], pa[3]), stream_out);
         }
       }
     } else if (EPI == EPI_SWIGLU_BWD) {
 #pragma unroll 1
-      for (int c = c0; c < p.bn; c += 32) {
+      for (int c = c0; c < bn; c += 32) {
         const int n = n0 + c;
         uint4 gv[2], uv[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (row_ok && n + 8 * h < p.N) {
-            const long long off = row * p.ld_in + n + 8 * h;
-            gv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.in[0]) + off));
-            uv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.in[1]) + off));
+          if (row_ok && n + 8 * h < N) {
+            const long long off = row * ld_in + n + 8 * h;
+            gv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in0) + off));
+            uv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in1) + off));
           } else {
             gv[h] = make_uint4(0, 0, 0, 0);
             uv[h] = make_uint4(0, 0, 0, 0);
@@ -574,10 +629,10 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         tmem_ld16(tbase + c, r);
         tmem_wait16(r);
         if (!row_ok) continue;
-        const long long off = row * p.ld_out + n;
+        const long long off = row * ld_out + n;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (n + 8 * h >= p.N) continue;
+          if (n + 8 * h >= N) continue;
           const uint32_t gw[4] = {gv[h].x, gv[h].y, gv[h].z, gv[h].w};
           const uint32_t uw[4] = {uv[h].x, uv[h].y, uv[h].z, uv[h].w};
           uint32_t pdg[4], pdu[4];
@@ -596,36 +651,36 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             pdg[j] = pack_bf16x2(dg[0], dg[1]);
             pdu[j] = pack_bf16x2(du[0], du[1]);
           }
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[0]) + off + 8 * h), make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]), p.stream_out);
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out[1]) + off + 8 * h), make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]), p.stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out0) + off + 8 * h), make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]), stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out1) + off + 8 * h), make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]), stream_out);
         }
       }
     } else if (EPI == EPI_ATOMIC) {
 #pragma unroll 1
-      for (int ri = 0; ri < p.nrng; ++ri) {
-        const OutRange& R = p.rng[ri];
+      for (int ri = 0; ri < nrng; ++ri) {
+        const OutRange R = p.rng[ri];
 #pragma unroll 1
-        for (int c = c0; c < p.bn; c += 32) {
+        for (int c = c0; c < bn; c += 32) {
           const int n = n0 + c;
-          if (n >= p.N) break;  // warp-uniform: remaining chunks are padding columns
+          if (n >= N) break;  // warp-uniform: remaining chunks are padding columns
           uint32_t r[16];
-          tmem_ld16(tbase + R.acc * p.bn + c, r);
+          tmem_ld16(tbase + R.acc * bn + c, r);
           tmem_wait16(r);
           if (!row_ok) continue;
           if (R.trans) {
             // out[n * ld + m]: lanes hold consecutive m -> coalesced across the warp
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (n + j < p.N) atomicAdd(R.out + static_cast<long long>(n + j) * R.ld + row, __uint_as_float(r[j]) * p.alpha);
+              if (n + j < N) atomicAdd(R.out + static_cast<long long>(n + j) * R.ld + row, __uint_as_float(r[j]) * alpha);
           } else {
             // out[m * ld + n]: 16 consecutive columns of one row -> four 16-byte vector atomics
             float* o = R.out + row * R.ld + n;
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-              if (n + 4 * h < p.N)
+              if (n + 4 * h < N)
                 atomicAdd(reinterpret_cast<float4*>(o + 4 * h),
-                          make_float4(__uint_as_float(r[4 * h]) * p.alpha, __uint_as_float(r[4 * h + 1]) * p.alpha,
-                                      __uint_as_float(r[4 * h + 2]) * p.alpha, __uint_as_float(r[4 * h + 3]) * p.alpha));
+                          make_float4(__uint_as_float(r[4 * h]) * alpha, __uint_as_float(r[4 * h + 1]) * alpha,
+                                      __uint_as_float(r[4 * h + 2]) * alpha, __uint_as_float(r[4 * h + 3]) * alpha));
           }
         }
       }
@@ -633,13 +688,13 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       // Online max / sum of exponentials over this warp's 16-column chunks of the tile:
       // m = running max, s = sum exp(z - m) (base-2 exponentials of pre-scaled values).
       constexpr float kLog2e = 1.4426950408889634f;
-      const int lab = row_ok ? __ldg(p.ce_labels + row) : -1;
+      const int lab = row_ok ? __ldg(ce_labels + row) : -1;
       float m = -INFINITY, sum = 0.f, zl = 0.f;
       bool has = false;
 #pragma unroll 1
-      for (int c = c0; c < p.bn; c += 32) {
+      for (int c = c0; c < bn; c += 32) {
         const int n = n0 + c;
-        if (n >= p.N) break;  // warp-uniform: the rest of the tile is past the vocabulary
+        if (n >= N) break;  // warp-uniform: the rest of the tile is past the vocabulary
         uint32_t r[16];
         tmem_ld16(tbase + c, r);
         tmem_wait16(r);
@@ -647,9 +702,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         float v[16], cm = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          v[e] = n + e < p.N ? __uint_as_float(r[e]) : -INFINITY;
+          v[e] = n + e < N ? __uint_as_float(r[e]) : -INFINITY;
           cm = fmaxf(cm, v[e]);
-          if (p.ce_col0 + n + e == lab) {
+          if (ce_col0 + n + e == lab) {
             zl = v[e];
             has = true;
           }
@@ -664,31 +719,31 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       }
       if (row_ok) {
         const int half = (warp - 2) >> 2;
-        reinterpret_cast<float2*>(p.out[0])[static_cast<long long>(2 * nt + half) * p.M + row] = make_float2(m, sum);
-        if (has) static_cast<float*>(p.out[1])[row] = zl;
+        reinterpret_cast<float2*>(out0)[static_cast<long long>(2 * nt + half) * M + row] = make_float2(m, sum);
+        if (has) static_cast<float*>(out1)[row] = zl;
       }
     } else if (EPI == EPI_CE_DZ) {
       // dZ = g' (exp(z - lse) - [column == label]); 0 for rows left out of the loss
       constexpr float kLog2e = 1.4426950408889634f;
-      const int lab = row_ok ? __ldg(p.ce_labels + row) : -1;
-      const bool keep = lab >= 0 && lab < p.ce_V;
+      const int lab = row_ok ? __ldg(ce_labels + row) : -1;
+      const bool keep = lab >= 0 && lab < ce_V;
       float gs = 0.f, l2 = 0.f;
       if (keep) {
-        gs = p.ce_count ? p.ce_g / static_cast<float>(max(1, __ldg(p.ce_count))) : p.ce_g;
-        l2 = __ldg(p.ce_lse + row) * kLog2e;
+        gs = ce_count ? ce_g / static_cast<float>(max(1, __ldg(ce_count))) : ce_g;
+        l2 = __ldg(ce_lse + row) * kLog2e;
       }
 #pragma unroll 1
-      for (int c = c0; c < p.bn; c += 32) {
+      for (int c = c0; c < bn; c += 32) {
         const int n = n0 + c;
-        if (n >= p.N) break;
+        if (n >= N) break;
         uint32_t r[16];
         tmem_ld16(tbase + c, r);
         tmem_wait16(r);
         if (!row_ok) continue;
-        uint16_t* o = static_cast<uint16_t*>(p.out[0]) + row * p.ld_out + n;
+        uint16_t* o = static_cast<uint16_t*>(out0) + row * ld_out + n;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (n + 8 * h >= p.N) continue;
+          if (n + 8 * h >= N) continue;
           uint32_t w[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -697,11 +752,11 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             for (int e = 0; e < 2; ++e) {
               const int k = 8 * h + 2 * j + e;
               const float pr = exp2f(fmaf(__uint_as_float(r[k]), kLog2e, -l2));
-              dz[e] = gs * (pr - (p.ce_col0 + n + k == lab ? 1.f : 0.f));
+              dz[e] = gs * (pr - (ce_col0 + n + k == lab ? 1.f : 0.f));
             }
             w[j] = pack_bf16x2(dz[0], dz[1]);
           }
-          st_out(reinterpret_cast<uint4*>(o + 8 * h), make_uint4(w[0], w[1], w[2], w[3]), p.stream_out);
+          st_out(reinterpret_cast<uint4*>(o + 8 * h), make_uint4(w[0], w[1], w[2], w[3]), stream_out);
         }
       }
     }
@@ -722,25 +777,30 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 template <int B_MN, int NACC, int PAIR, int FUSE>
 __device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* ring, uint32_t crfull0,
                                                    uint32_t crempty0, const WaitCtl& wc, uint32_t rank) {
-  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const Sched sc = sched_of(p);
+  // launch constants in registers (see Sched)
+  const int bn = p.bn, nseg = p.nseg;
+  const uint32_t cr_bytes = p.cr_bytes;
+  const CUtensorMap* maps = p.maps;
+  const int total = sc.total;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
-  const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
+  const Q4Layout QL = q4_layout(bn, PAIR, FUSE, B_MN, NACC);
   int e = 0;
   uint32_t phase = 0, issued_mask = 0, issued_par = 0;
   bool ok = true;
   for (int t = unit0; t < total && ok; t += nunits) {
     int mt, nt, ks;
-    decode_tile(p, t, mt, nt, ks);
-    const int n0 = nt * p.bn;
-    for (int s = 0; s < p.nseg && ok; ++s) {
-      const Seg& sg = p.seg[s];
+    decode_tile(sc, t, mt, nt, ks);
+    const int n0 = nt * bn;
+    for (int s = 0; s < nseg && ok; ++s) {
+      const SegR sg = seg_of(p, s);
       if (!sg.q4) continue;
       int kb0, kb1;
-      seg_kb_range(p, s, ks, kb0, kb1);
+      seg_kb_range(sc, sg.k_len, ks, kb0, kb1);
       uint32_t code_tx = 0;
       for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
         if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
-        if (sg.b_map[u] >= 0) code_tx += QL.q_unit + QL.m_unit;
+        if (seg_bmap(sg, u) >= 0) code_tx += QL.q_unit + QL.m_unit;
       }
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(crempty0 + 8 * e, phase ^ 1, wc, kDevTimeoutProducer)) {
@@ -750,17 +810,17 @@ __device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* r
         const uint32_t bar = crfull0 + 8 * e;
         if (code_tx) mbar_expect_tx(bar, code_tx);
         else mbar_arrive(bar);
-        const uint32_t sQ = smem_u32(ring + static_cast<size_t>(e) * p.cr_bytes);
+        const uint32_t sQ = smem_u32(ring + static_cast<size_t>(e) * cr_bytes);
         const uint32_t sM = sQ + QL.slots * QL.q_unit;
 #pragma unroll
         for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
           if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
-          if (sg.b_map[u] < 0) continue;
+          if (seg_bmap(sg, u) < 0) continue;
           const int slot = (FUSE && PAIR == 2) ? 0 : u;
-          const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (p.bn / PAIR);  // first B row / column here
-          const CUtensorMap* qm = &p.maps[sg.b_map[u]];
-          const CUtensorMap* mm = &p.maps[sg.b_am[u]];
-          const int kk = sg.b_k0[u] + kb * BK;
+          const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (bn / PAIR);  // first B row / column here
+          const CUtensorMap* qm = &maps[seg_bmap(sg, u)];
+          const CUtensorMap* mm = &maps[seg_bam(sg, u)];
+          const int kk = seg_bk0(sg, u) + kb * BK;
           if (B_MN) {
             tma_load_2d(sQ + slot * QL.q_unit, qm, bar, nq / 2, kk);
             tma_load_2d(sM + slot * QL.m_unit, mm, bar, (nq / 64) & ~3, kk);
@@ -809,22 +869,26 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
   const int lane = threadIdx.x % 32;
   const int group = (tid >> 5) / kGroupWarps;
   const int gtid = tid % (32 * kGroupWarps);
-  const int total = p.tiles_m * p.tiles_n * p.splits;
+  const Sched sc = sched_of(p);
+  // launch constants in registers (see Sched)
+  const int bn = p.bn, nseg = p.nseg, nstages = p.stages;
+  const uint32_t cr_bytes = p.cr_bytes, stage_bytes = p.stage_bytes;
+  const int total = sc.total;
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   const uint32_t a_bytes = BM * BK * 2;
-  const Q4Layout QL = q4_layout(p.bn, PAIR, FUSE, B_MN, NACC);
+  const Q4Layout QL = q4_layout(bn, PAIR, FUSE, B_MN, NACC);
   const float* code = tab + lane;  // code value e at code[32 * e] (lane-replicated: conflict-free)
   int stage = 0, turn = 0, e = 0;
   uint32_t phase = 0, cphase = 0;
   bool ok = true;
   for (int t = unit0; t < total && ok; t += nunits) {
     int mt, nt, ks;
-    decode_tile(p, t, mt, nt, ks);
-    const int n0 = nt * p.bn;
-    for (int s = 0; s < p.nseg && ok; ++s) {
-      const Seg& sg = p.seg[s];
+    decode_tile(sc, t, mt, nt, ks);
+    const int n0 = nt * bn;
+    for (int s = 0; s < nseg && ok; ++s) {
+      const SegR sg = seg_of(p, s);
       int kb0, kb1;
-      seg_kb_range(p, s, ks, kb0, kb1);
+      seg_kb_range(sc, sg.k_len, ks, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (turn == group) {
           // the stage's previous contents consumed by the MMA (B slot free), codes landed
@@ -839,16 +903,16 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
             break;
           }
           if (sg.q4) {
-            uint8_t* base = tiles + static_cast<size_t>(stage) * p.stage_bytes;
-            const uint8_t* sQ = ring + static_cast<size_t>(e) * p.cr_bytes;
+            uint8_t* base = tiles + static_cast<size_t>(stage) * stage_bytes;
+            const uint8_t* sQ = ring + static_cast<size_t>(e) * cr_bytes;
             const float* sM = reinterpret_cast<const float*>(sQ + QL.slots * QL.q_unit);
             const int kk = kb * BK;
             const int chunks = QL.cols >> 6;
             for (int u = 0; u < (FUSE ? 2 : NACC); ++u) {
               if (FUSE && PAIR == 2 && static_cast<uint32_t>(u) != rank) continue;
-              if (sg.b_map[u] < 0) continue;
+              if (seg_bmap(sg, u) < 0) continue;
               const int slot = (FUSE && PAIR == 2) ? 0 : u;
-              const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (p.bn / PAIR);
+              const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (bn / PAIR);
               const uint8_t* q = sQ + slot * QL.q_unit;
               const float* am = sM + slot * (QL.m_unit / 4);
               uint8_t* dst = base + a_bytes + slot * QL.b_unit;
@@ -906,7 +970,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
           cphase ^= 1;
         }
         if (++turn == kDqGroups) turn = 0;
-        if (++stage == p.stages) {
+        if (++stage == nstages) {
           stage = 0;
           phase ^= 1;
         }
