@@ -291,13 +291,22 @@ def sub_records(args, pb8, bits8, clk, pk):
     del pb
     # 8B shape, 4-bit frozen weights (quantised on the GPU: one-off set-up, not timed)
     s8 = pb8.shape
-    pb8.use_4bit(load_codebook())
+    pb8.use_4bit(load_codebook(), drop_bf16=False)
     for _ in range(3):
         pb8.step()
     ms, ph = timed(pb8.step, steps, stream, clk, "config_4bit")
     rec("config_4bit", f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape with 4-bit frozen W (block 64): T={s8.T} d={s8.d} "
         f"f={s8.f} r={s8.r} alpha=16", s8.T, configs.algorithmic_flops(s8), ms, ph, "gemm_gate_up_swiglu",
         4.0 * s8.T * s8.d * s8.f + 4.0 * s8.T * s8.r * s8.f, dtype=dtype_for("8b-4bit"))
+    # the same with double-quantised block constants (8-bit codes + an fp32 scale per 256)
+    pb8.use_4bit(load_codebook(), double_quant=True)
+    for _ in range(3):
+        pb8.step()
+    ms, ph = timed(pb8.step, steps, stream, clk, "config_4bit_dq")
+    rec("config_4bit_dq", f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape with 4-bit frozen W, double-quantised block "
+        f"constants: T={s8.T} d={s8.d} f={s8.f} r={s8.r} alpha=16", s8.T, configs.algorithmic_flops(s8), ms, ph,
+        "gemm_gate_up_swiglu", 4.0 * s8.T * s8.d * s8.f + 4.0 * s8.T * s8.r * s8.f,
+        dtype="bf16 activations, 4-bit codebook weights, 8-bit block constants")
     # attention Q/K/V projections of the 8B model
     sq = configs.QKV_8B
     qp = QkvProblem(sq)

@@ -56,15 +56,17 @@ enum lora_status {
 };
 
 enum lora_wfmt {
-  LORA_WFMT_BF16 = 0, /* frozen Wg, Wu, Wd given as bf16                              */
-  LORA_WFMT_4BIT = 1  /* frozen weights given as 4-bit blockwise codes (qblock = 64)  */
+  LORA_WFMT_BF16 = 0,    /* frozen Wg, Wu, Wd given as bf16                              */
+  LORA_WFMT_4BIT = 1,    /* frozen weights given as 4-bit blockwise codes (qblock = 64)  */
+  LORA_WFMT_4BIT_DQ = 2  /* the same codes with double-quantised block constants: 8-bit  */
+                         /* codes of the absmax values plus an fp32 scale per 256 of them */
 };
 
 /* Problem sizes.  T tokens, hidden d, intermediate f, LoRA rank r.
  * Limits: 1 <= T < 2^31; d, f multiples of 8 with 8 <= d <= 65536, 8 <= f;
  * r a multiple of 8 with 8 <= r <= 128.  scale = alpha / r (any finite value).
  * wfmt = LORA_WFMT_BF16 or LORA_WFMT_4BIT (then qblock must be 64 and d, f
- * multiples of 256).  residual = 1 adds the decoder layer's residual connection
+ * multiples of 256; the same for LORA_WFMT_4BIT_DQ).  residual = 1 adds the decoder layer's residual connection
  * around the sub-block ("Unsloth加速原理揭秘", §3.1, the LoRA forward ending in a
  * residual add): Y = X + MLP(RMSNorm(X)) and dX gets + dY; 0 = the sub-block alone. */
 typedef struct lora_mlp_dims {
@@ -87,7 +89,14 @@ typedef struct lora_mlp_dims {
  * expand them to bf16 tiles in-kernel (w = bf16(codebook[idx] * absmax), fp32
  * product rounded once) right before the tensor-core MMA; no bf16 copy of W is
  * ever written to memory.
- * Unused members may be NULL. */
+ * wfmt = LORA_WFMT_4BIT_DQ (double quantisation, "Unsloth 深度实战…", §1.4: the
+ * quantisation constants are quantised too) replaces absmax_x by
+ *   absmax8_x [n] uint8 and scale2_x [ceil(n / 256)] fp32, n = (block count) = out*in/64:
+ *   absmax = fl32(fl32(scale2[i / 256] * k) / 255), k = absmax8[i]
+ * (from lora_quantize_absmax8); each call expands them to fp32 in its workspace
+ * (3 * n floats) before the GEMMs.
+ * Unused members may be NULL.  (The absmax8 / scale2 members were appended after the
+ * others; callers of the bf16 and plain 4-bit formats may leave them zero.) */
 typedef struct lora_mlp_weights {
   const void* Wg;
   const void* Wu;
@@ -99,6 +108,12 @@ typedef struct lora_mlp_weights {
   const float* absmax_u;
   const float* absmax_d;
   const float* codebook;
+  const uint8_t* absmax8_g;
+  const uint8_t* absmax8_u;
+  const uint8_t* absmax8_d;
+  const float* scale2_g;
+  const float* scale2_u;
+  const float* scale2_d;
 } lora_mlp_weights;
 
 /* LoRA adapters, bf16: Ag, Au [r x d]; Bg, Bu [f x r]; Ad [r x f]; Bd [d x r]. */
@@ -345,6 +360,17 @@ int lora_merge_weights(int64_t rows, int64_t cols, int32_t r, float scale, const
  * absmax [numel/64] fp32. */
 int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float* codebook16,
                        uint8_t* codes, float* absmax, void* stream);
+
+/* Double quantisation of the 4-bit block constants ("Unsloth 深度实战…", §1.4: the
+ * quantisation constants are themselves quantised; the pages give no format, so this
+ * is a reading): absmax [n] fp32 (>= 0, as lora_quantize_4bit writes it) in blocks of
+ * block2 = 256 consecutive values (the last may be shorter); scale2[b] = the block's
+ * largest value; codes8[i] = #{ j in 1..255 : 510 absmax[i] > (2j - 1) scale2[b] },
+ * i.e. the nearest of the levels scale2 k / 255, ties to the lower one, decided exactly
+ * (fp64 products); an all-zero block gives scale2 0 and codes 0.  codes8 [n] bytes,
+ * scale2 [ceil(n / 256)] fp32.  Asynchronous; nothing is allocated. */
+int lora_quantize_absmax8(const float* absmax, int64_t n, int32_t block2, uint8_t* codes8, float* scale2,
+                          void* stream);
 
 /* Plain tensor-core GEMM (the core the fused path is built on), fp32 out:
  *   C[M x N] = A' B'^T,  A' [M x K] = A (a_mn = 0, A row-major [M x K]) or A^T

@@ -296,11 +296,17 @@ inline int launch_rms_fwd(cudaStream_t st, const void* X, const void* w, void* H
   PhaseScope ps(st, PH_RMS_FWD);
   for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
     unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
-    switch (v) {
-      case 1: rmsnorm_fwd_kernel<1><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-      case 2: rmsnorm_fwd_kernel<2><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-      case 4: rmsnorm_fwd_kernel<4><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
-      default: rmsnorm_fwd_kernel<8><<<rows, threads, 0, st>>>(X16 + r0 * d, w16, H16 + r0 * d, rstd + r0, d, eps); break;
+    const uint16_t* x = X16 + r0 * d;
+    uint16_t* h = H16 + r0 * d;
+    if (threads <= kRowThreads) {
+      switch (v) {
+        case 1: rmsnorm_fwd_kernel<1, kRowThreads><<<rows, threads, 0, st>>>(x, w16, h, rstd + r0, d, eps); break;
+        case 2: rmsnorm_fwd_kernel<2, kRowThreads><<<rows, threads, 0, st>>>(x, w16, h, rstd + r0, d, eps); break;
+        case 4: rmsnorm_fwd_kernel<4, kRowThreads><<<rows, threads, 0, st>>>(x, w16, h, rstd + r0, d, eps); break;
+        default: rmsnorm_fwd_kernel<8, kRowThreads><<<rows, threads, 0, st>>>(x, w16, h, rstd + r0, d, eps); break;
+      }
+    } else {
+      rmsnorm_fwd_kernel<8, 1024><<<rows, threads, 0, st>>>(x, w16, h, rstd + r0, d, eps);
     }
   }
   CUDA_TRY(cudaGetLastError());
@@ -324,10 +330,18 @@ inline int launch_rms_bwd(cudaStream_t st, const float* dH, const void* X, const
   PhaseScope ps(st, PH_RMS_BWD);
   for (long long r0 = 0; r0 < T; r0 += 0x7fffffffLL) {
     unsigned int rows = static_cast<unsigned int>(std::min<long long>(T - r0, 0x7fffffffLL));
-    switch (v) {
-      case 1: rmsnorm_bwd_kernel<1><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
-      case 2: rmsnorm_bwd_kernel<2><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
-      default: rmsnorm_bwd_kernel<4><<<rows, threads, 0, st>>>(dH + r0 * d, X16 + r0 * d, w16, rstd + r0, dY16 ? dY16 + r0 * d : nullptr, dX16 + r0 * d, d); break;
+    const float* g = dH + r0 * d;
+    const uint16_t* x = X16 + r0 * d;
+    const uint16_t* y = dY16 ? dY16 + r0 * d : nullptr;
+    uint16_t* o = dX16 + r0 * d;
+    if (threads <= kRowThreads) {
+      switch (v) {
+        case 1: rmsnorm_bwd_kernel<1, kRowThreads><<<rows, threads, 0, st>>>(g, x, w16, rstd + r0, y, o, d); break;
+        case 2: rmsnorm_bwd_kernel<2, kRowThreads><<<rows, threads, 0, st>>>(g, x, w16, rstd + r0, y, o, d); break;
+        default: rmsnorm_bwd_kernel<4, kRowThreads><<<rows, threads, 0, st>>>(g, x, w16, rstd + r0, y, o, d); break;
+      }
+    } else {
+      rmsnorm_bwd_kernel<4, 1024><<<rows, threads, 0, st>>>(g, x, w16, rstd + r0, y, o, d);
     }
   }
   CUDA_TRY(cudaGetLastError());

@@ -12,7 +12,7 @@ namespace {
 
 // --------------------------------------------------------------- layouts
 struct WsLayout {
-  size_t status, Q, Qd, dG, dU, dH, part, total;
+  size_t status, Q, Qd, dG, dU, dH, part, am, total;
 };
 
 int check_dims(const lora_mlp_dims* D) {
@@ -23,9 +23,10 @@ int check_dims(const lora_mlp_dims* D) {
     return fail(LORA_ERR_ALIGNMENT, "d, f, r must be multiples of 8 (16-byte rows); got %d %d %d", D->d, D->f, D->r);
   if (D->d > 65536) return fail(LORA_ERR_UNSUPPORTED, "d = %d > 65536", D->d);
   if (D->r > 128) return fail(LORA_ERR_UNSUPPORTED, "r = %d > 128", D->r);
-  if (D->wfmt != LORA_WFMT_BF16 && D->wfmt != LORA_WFMT_4BIT) return fail(LORA_ERR_INVALID_ARG, "bad wfmt");
+  if (D->wfmt != LORA_WFMT_BF16 && D->wfmt != LORA_WFMT_4BIT && D->wfmt != LORA_WFMT_4BIT_DQ)
+    return fail(LORA_ERR_INVALID_ARG, "bad wfmt");
   if (D->residual != 0 && D->residual != 1) return fail(LORA_ERR_INVALID_ARG, "residual must be 0 or 1");
-  if (D->wfmt == LORA_WFMT_4BIT) {
+  if (D->wfmt != LORA_WFMT_BF16) {
     if (D->qblock != 64) return fail(LORA_ERR_UNSUPPORTED, "qblock must be 64");
     if (D->d % 256 || D->f % 256) return fail(LORA_ERR_UNSUPPORTED, "4-bit weights need d, f multiples of 256");
   }
@@ -66,8 +67,47 @@ WsLayout ws_layout(const lora_mlp_dims* D) {
   part = std::max(part, size_t(proj_splits(T, d)) * T * rp);       // Qd = s dY Bd
   part = std::max(part, size_t(proj_splits(T, f)) * T * 2 * rp);   // Q  = s [dG Bg | dU Bu]
   L.part = o; o = up256(o + part * 4);
+  // double-quantised constants: the fp32 absmax of Wg, Wu and Wd, decoded at each call
+  L.am = o;
+  if (D->wfmt == LORA_WFMT_4BIT_DQ) o = up256(o + 3 * (f * d / 64) * 4);
   L.total = o;
   return L;
+}
+
+// Weight constants of a 4-bit call: the caller's fp32 absmax, or for double-quantised
+// constants their fp32 expansion in the workspace (one decode launch per call).
+struct Absmax3 {
+  const float *g, *u, *d;
+};
+int absmax_for_call(const lora_mlp_dims* D, const lora_mlp_weights* W, void* workspace, const WsLayout& WL,
+                    cudaStream_t st, Absmax3* out) {
+  if (D->wfmt != LORA_WFMT_4BIT_DQ) {
+    *out = Absmax3{W->absmax_g, W->absmax_u, W->absmax_d};
+    return LORA_OK;
+  }
+  const long long n = static_cast<long long>(D->f) * D->d / 64;
+  float* base = at<float>(workspace, WL.am);
+  Absmax8List L{};
+  const uint8_t* codes[3] = {W->absmax8_g, W->absmax8_u, W->absmax8_d};
+  const float* sc[3] = {W->scale2_g, W->scale2_u, W->scale2_d};
+  for (int m = 0; m < 3; ++m) {
+    L.codes[m] = codes[m];
+    L.scale2[m] = sc[m];
+    L.out[m] = base + m * n;
+    L.n[m] = n;
+  }
+  PhaseScope ps(st, PH_OTHER);
+  absmax8_decode_kernel<<<296, 256, 0, st>>>(L);
+  CUDA_TRY(cudaGetLastError());
+  *out = Absmax3{base, base + n, base + 2 * n};
+  return LORA_OK;
+}
+
+int check_weights(const lora_mlp_dims* D, const lora_mlp_weights* W) {
+  if (D->wfmt == LORA_WFMT_BF16) return check_ptrs({W->Wg, W->Wu, W->Wd});
+  TRY(check_ptrs({W->Qg, W->Qu, W->Qd, W->codebook}));
+  if (D->wfmt == LORA_WFMT_4BIT) return check_ptrs({W->absmax_g, W->absmax_u, W->absmax_d});
+  return check_ptrs({W->absmax8_g, W->absmax8_u, W->absmax8_d, W->scale2_g, W->scale2_u, W->scale2_d});
 }
 
 
@@ -253,6 +293,20 @@ int lora_quantize_4bit(const void* W, int64_t numel, int32_t block, const float*
   return LORA_OK;
 }
 
+int lora_quantize_absmax8(const float* absmax, int64_t n, int32_t block2, uint8_t* codes8, float* scale2,
+                          void* stream) {
+  if (block2 != kAbsmax8Block) return fail(LORA_ERR_UNSUPPORTED, "block2 must be %d", kAbsmax8Block);
+  if (n < 1) return fail(LORA_ERR_INVALID_ARG, "n must be positive");
+  TRY(check_ptrs({absmax, codes8, scale2}));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long nblk = (n + kAbsmax8Block - 1) / kAbsmax8Block;
+  const long long blocks = std::min<long long>((nblk + 7) / 8, 148LL * 16);
+  PhaseScope ps(st, PH_OTHER);
+  absmax8_quantize_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(absmax, n, codes8, scale2);
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
+
 int lora_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int32_t a_mn, const void* B, int32_t b_mn,
                    float* C, int32_t flags, void* stream) {
   if (M < 1 || N < 1 || K < 1 || M >= (1LL << 31) || N >= (1LL << 31) || K >= (1LL << 31))
@@ -328,10 +382,9 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
                  const lora_mlp_adapters* A, void* Y, void* ctx, void* workspace, void* stream) {
   TRY(check_dims(D));
   if (!W || !A) return fail(LORA_ERR_INVALID_ARG, "weights/adapters is NULL");
-  const bool q4 = D->wfmt == LORA_WFMT_4BIT;
+  const bool q4 = D->wfmt != LORA_WFMT_BF16;
   TRY(check_ptrs({X, rms_w, Y, ctx, workspace, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd}));
-  if (q4) TRY(check_ptrs({W->Qg, W->Qu, W->Qd, W->absmax_g, W->absmax_u, W->absmax_d, W->codebook}));
-  else TRY(check_ptrs({W->Wg, W->Wu, W->Wd}));
+  TRY(check_weights(D, W));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long T = D->T;
   const int d = D->d, f = D->f, r = D->r, rp = rp_of(D);
@@ -347,6 +400,8 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
   void* P = at<char>(ctx, L.P);
   void* Pd = at<char>(ctx, L.Pd);
   TRY(begin_call(status, st));
+  Absmax3 am{};
+  if (q4) TRY(absmax_for_call(D, W, workspace, WL, st, &am));
 
   // S1: RMSNorm (cached rstd)
   TRY(launch_rms_fwd(st, X, rms_w, H, rstd, T, d, D->eps));
@@ -373,8 +428,8 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     GemmArgs a = new_args(status);
     const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
-    TRY(map_q4_k(&a.maps[1], &a.maps[6], W->Qg, W->absmax_g, f, d, 128));
-    TRY(map_q4_k(&a.maps[2], &a.maps[7], W->Qu, W->absmax_u, f, d, 128));
+    TRY(map_q4_k(&a.maps[1], &a.maps[6], W->Qg, am.g, f, d, 128));
+    TRY(map_q4_k(&a.maps[2], &a.maps[7], W->Qu, am.u, f, d, 128));
     TRY(map_k(&a.maps[3], P, T, 2 * rp, 2 * rp, 128));
     TRY(map_k(&a.maps[4], A->Bg, f, r, r, 128));
     TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
@@ -426,7 +481,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     const int bn = 256;  // d is a multiple of 256 for 4-bit weights
     const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], Act, T, f, f, 128));
-    TRY(map_q4_k(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn / pair));
+    TRY(map_q4_k(&a.maps[1], &a.maps[4], W->Qd, am.d, d, f, bn / pair));
     TRY(map_k(&a.maps[2], Pd, T, rp, rp, 128));
     TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn / pair));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
@@ -469,12 +524,11 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
                  void* stream) {
   TRY(check_dims(D));
   if (!W || !A || !gr) return fail(LORA_ERR_INVALID_ARG, "weights/adapters/grads is NULL");
-  const bool q4 = D->wfmt == LORA_WFMT_4BIT;
+  const bool q4 = D->wfmt != LORA_WFMT_BF16;
   TRY(check_ptrs({dY, X, rms_w, ctx, dX, workspace, A->Ag, A->Bg, A->Au, A->Bu, A->Ad, A->Bd,
                   gr->dAg, gr->dBg, gr->dAu, gr->dBu, gr->dAd, gr->dBd}));
   if (gr->dw) TRY(check_ptrs({gr->dw}));
-  if (q4) TRY(check_ptrs({W->Qg, W->Qu, W->Qd, W->absmax_g, W->absmax_u, W->absmax_d, W->codebook}));
-  else TRY(check_ptrs({W->Wg, W->Wu, W->Wd}));
+  TRY(check_weights(D, W));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long T = D->T;
   const int d = D->d, f = D->f, r = D->r, rp = rp_of(D);
@@ -497,6 +551,8 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   const int tm = static_cast<int>((T + BM - 1) / BM);
   const int qbn = rp <= 64 ? 64 : 128;
   TRY(begin_call(status, st));
+  Absmax3 am{};
+  if (q4) TRY(absmax_for_call(D, W, workspace, WL, st, &am));
 
   float* part = at<float>(workspace, WL.part);
   // S5a: Qd = s * dY Bd
@@ -514,7 +570,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     const int bn = 256;
     const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], dY, T, d, d, 128));
-    TRY(map_q4_mn(&a.maps[1], &a.maps[4], W->Qd, W->absmax_d, d, f, bn / pair));
+    TRY(map_q4_mn(&a.maps[1], &a.maps[4], W->Qd, am.d, d, f, bn / pair));
     TRY(map_k(&a.maps[2], Qd, T, rp, rp, 128));
     a.mn3d_b = 1;
     TRY(map_mn3(&a.maps[3], A->Ad, r, f, f, bn / pair / 64));
@@ -573,9 +629,9 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     const int bn = 256;
     const int pair = T > 128 ? 2 : 1;
     TRY(map_k(&a.maps[0], dG, T, f, f, 128));
-    TRY(map_q4_mn(&a.maps[1], &a.maps[7], W->Qg, W->absmax_g, f, d, bn / pair));
+    TRY(map_q4_mn(&a.maps[1], &a.maps[7], W->Qg, am.g, f, d, bn / pair));
     TRY(map_k(&a.maps[2], dU, T, f, f, 128));
-    TRY(map_q4_mn(&a.maps[3], &a.maps[8], W->Qu, W->absmax_u, f, d, bn / pair));
+    TRY(map_q4_mn(&a.maps[3], &a.maps[8], W->Qu, am.u, f, d, bn / pair));
     TRY(map_k(&a.maps[4], Q, T, 2 * rp, 2 * rp, 128));
     a.mn3d_b = 1;
     TRY(map_mn3(&a.maps[5], A->Ag, r, d, d, bn / pair / 64));

@@ -16,7 +16,45 @@
 
 namespace lm {
 
+// One work item: 8 pairs of one head of one token (see above).
+struct RopeItem {
+  uint4* pa;
+  uint4* pb;
+  uint4 va, vb;
+  float4 c0, c1, s0, s1;
+};
+__device__ __forceinline__ void rope_load(RopeItem& it, uint16_t* head, int i0, int half, const float* cosT,
+                                          const float* sinT, long long p) {
+  it.pa = reinterpret_cast<uint4*>(head + i0);
+  it.pb = reinterpret_cast<uint4*>(head + i0 + half);
+  it.va = *it.pa;
+  it.vb = *it.pb;
+  const float4* pc = reinterpret_cast<const float4*>(cosT + p * half + i0);
+  const float4* ps = reinterpret_cast<const float4*>(sinT + p * half + i0);
+  it.c0 = __ldg(pc);
+  it.c1 = __ldg(pc + 1);
+  it.s0 = __ldg(ps);
+  it.s1 = __ldg(ps + 1);
+}
+__device__ __forceinline__ void rope_apply(const RopeItem& it, float sgn) {
+  const float c[8] = {it.c0.x, it.c0.y, it.c0.z, it.c0.w, it.c1.x, it.c1.y, it.c1.z, it.c1.w};
+  const float sn[8] = {sgn * it.s0.x, sgn * it.s0.y, sgn * it.s0.z, sgn * it.s0.w,
+                       sgn * it.s1.x, sgn * it.s1.y, sgn * it.s1.z, sgn * it.s1.w};
+  const uint32_t wa[4] = {it.va.x, it.va.y, it.va.z, it.va.w}, wb[4] = {it.vb.x, it.vb.y, it.vb.z, it.vb.w};
+  uint32_t oa[4], ob[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float a0 = bf16lo(wa[k]), a1 = bf16hi(wa[k]), b0 = bf16lo(wb[k]), b1 = bf16hi(wb[k]);
+    const float cc0 = c[2 * k], cc1 = c[2 * k + 1], s0k = sn[2 * k], s1k = sn[2 * k + 1];
+    oa[k] = pack_bf16x2(fmaf(a0, cc0, -b0 * s0k), fmaf(a1, cc1, -b1 * s1k));
+    ob[k] = pack_bf16x2(fmaf(b0, cc0, a0 * s0k), fmaf(b1, cc1, a1 * s1k));
+  }
+  *it.pa = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+  *it.pb = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+}
+
 // blockDim.x threads per token row; a CTA walks rows blockIdx.x, + gridDim.x, ...
+// (one row's state per thread keeps six 320-thread CTAs resident per SM for the 8B heads).
 // sgn = +1 forward, -1 backward (the inverse rotation).
 static __global__ void __launch_bounds__(512) rope_kernel(uint16_t* __restrict__ Q, uint16_t* __restrict__ K,
                                                           const int32_t* __restrict__ pos,
@@ -34,27 +72,9 @@ static __global__ void __launch_bounds__(512) rope_kernel(uint16_t* __restrict__
     }
     for (int j = threadIdx.x; j < per_row; j += blockDim.x) {
       const int h = j / per_head, i0 = (j - h * per_head) * 8;
-      uint16_t* head = h < hq ? Q + (t * hq + h) * hd : K + (t * hk + (h - hq)) * hd;
-      uint4* pa = reinterpret_cast<uint4*>(head + i0);
-      uint4* pb = reinterpret_cast<uint4*>(head + i0 + half);
-      const float4* pc = reinterpret_cast<const float4*>(cosT + p * half + i0);
-      const float4* ps = reinterpret_cast<const float4*>(sinT + p * half + i0);
-      const uint4 va = *pa, vb = *pb;
-      const float4 c0 = __ldg(pc), c1 = __ldg(pc + 1), s0 = __ldg(ps), s1 = __ldg(ps + 1);
-      const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      const float sn[8] = {sgn * s0.x, sgn * s0.y, sgn * s0.z, sgn * s0.w,
-                           sgn * s1.x, sgn * s1.y, sgn * s1.z, sgn * s1.w};
-      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-      uint32_t oa[4], ob[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float a0 = bf16lo(wa[k]), a1 = bf16hi(wa[k]), b0 = bf16lo(wb[k]), b1 = bf16hi(wb[k]);
-        const float cc0 = c[2 * k], cc1 = c[2 * k + 1], s0k = sn[2 * k], s1k = sn[2 * k + 1];
-        oa[k] = pack_bf16x2(fmaf(a0, cc0, -b0 * s0k), fmaf(a1, cc1, -b1 * s1k));
-        ob[k] = pack_bf16x2(fmaf(b0, cc0, a0 * s0k), fmaf(b1, cc1, a1 * s1k));
-      }
-      *pa = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-      *pb = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+      RopeItem it;
+      rope_load(it, h < hq ? Q + (t * hq + h) * hd : K + (t * hk + (h - hq)) * hd, i0, half, cosT, sinT, p);
+      rope_apply(it, sgn);
     }
   }
 }

@@ -29,9 +29,10 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
 }
 
-// VPT = 16-byte vectors (8 bf16) per thread; blockDim.x * VPT * 8 >= d.
-template <int VPT>
-static __global__ void __launch_bounds__(1024) rmsnorm_fwd_kernel(const uint16_t* __restrict__ X,
+// VPT = 16-byte vectors (8 bf16) per thread; blockDim.x * VPT * 8 >= d; MAXT bounds
+// blockDim.x (the common 128-thread launch gets the registers to hold its row unspilled).
+template <int VPT, int MAXT>
+static __global__ void __launch_bounds__(MAXT) rmsnorm_fwd_kernel(const uint16_t* __restrict__ X,
                                                            const uint16_t* __restrict__ w,
                                                            uint16_t* __restrict__ H,
                                                            float* __restrict__ rstd, int d,
@@ -73,8 +74,8 @@ static __global__ void __launch_bounds__(1024) rmsnorm_fwd_kernel(const uint16_t
 }
 
 // dX = rstd * (g - xhat * mean(g * xhat)), g = dH * w, xhat = x * rstd.
-template <int VPT>
-static __global__ void __launch_bounds__(1024) rmsnorm_bwd_kernel(const float* __restrict__ dH,
+template <int VPT, int MAXT>
+static __global__ void __launch_bounds__(MAXT) rmsnorm_bwd_kernel(const float* __restrict__ dH,
                                                            const uint16_t* __restrict__ X,
                                                            const uint16_t* __restrict__ w,
                                                            const float* __restrict__ rstd,
@@ -280,6 +281,63 @@ static __global__ void __launch_bounds__(128) merge_weights_kernel(const uint16_
       *reinterpret_cast<uint4*>(Wm + off) = ov;
     }
   }
+}
+
+// Double quantisation of the 4-bit block constants ("Unsloth 深度实战…", §1.4: the
+// quantisation constants are quantised as well).  One warp per block of 256 absmax
+// values: scale2 = the block's largest value; each value a gets the 8-bit code
+// k = #{ j in 1..255 : 510 a > (2j - 1) scale2 } (nearest of the levels scale2 k / 255,
+// ties to the lower one), decided exactly: both products are exact in double.
+constexpr int kAbsmax8Block = 256;
+static __global__ void absmax8_quantize_kernel(const float* __restrict__ absmax, long long n,
+                                               uint8_t* __restrict__ codes8, float* __restrict__ scale2) {
+  const int lane = threadIdx.x % 32;
+  const long long nblk = (n + kAbsmax8Block - 1) / kAbsmax8Block;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  for (long long b = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32; b < nblk;
+       b += warps) {
+    const long long i0 = b * kAbsmax8Block;
+    float v[kAbsmax8Block / 32];
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < kAbsmax8Block / 32; ++e) {
+      const long long i = i0 + e * 32 + lane;
+      v[e] = i < n ? absmax[i] : 0.f;
+      mx = fmaxf(mx, v[e]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) scale2[b] = mx;
+    const double sd = mx;
+#pragma unroll
+    for (int e = 0; e < kAbsmax8Block / 32; ++e) {
+      const long long i = i0 + e * 32 + lane;
+      if (i >= n) continue;
+      const double x = 510.0 * static_cast<double>(v[e]);
+      int k = 0;
+      if (sd > 0.0) {
+        k = static_cast<int>(floor((x / sd + 1.0) * 0.5));  // estimate, then settle exactly
+        k = k < 0 ? 0 : (k > 255 ? 255 : k);
+        while (k < 255 && x > sd * (2 * (k + 1) - 1)) ++k;
+        while (k > 0 && !(x > sd * (2 * k - 1))) --k;
+      }
+      codes8[i] = static_cast<uint8_t>(k);
+    }
+  }
+}
+
+// absmax[i] = scale2[i / 256] * codes8[i] / 255 in fp32, for up to three matrices.
+struct Absmax8List {
+  const uint8_t* codes[3];
+  const float* scale2[3];
+  float* out[3];
+  long long n[3];
+};
+static __global__ void absmax8_decode_kernel(Absmax8List L) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (int m = 0; m < 3; ++m)
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < L.n[m]; i += stride)
+      L.out[m][i] = L.scale2[m][i / kAbsmax8Block] * static_cast<float>(L.codes[m][i]) / 255.0f;
 }
 
 }  // namespace lm

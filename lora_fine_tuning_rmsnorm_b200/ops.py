@@ -16,7 +16,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "lora_mlp.h")
 
 LORA_OK = 0
 ERRORS = {-1: "INVALID_ARG", -2: "ALIGNMENT", -3: "UNSUPPORTED", -4: "CUDA", -5: "TIMEOUT"}
-WFMT_BF16, WFMT_4BIT = 0, 1
+WFMT_BF16, WFMT_4BIT, WFMT_4BIT_DQ = 0, 1, 2
 NUM_PHASES = 28
 
 
@@ -32,9 +32,12 @@ class Dims(ctypes.Structure):
                 ("qblock", ctypes.c_int32), ("residual", ctypes.c_int32)]
 
 
+WEIGHT_FIELDS = ("Wg", "Wu", "Wd", "Qg", "Qu", "Qd", "absmax_g", "absmax_u", "absmax_d", "codebook",
+                 "absmax8_g", "absmax8_u", "absmax8_d", "scale2_g", "scale2_u", "scale2_d")
+
+
 class Weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in
-                ("Wg", "Wu", "Wd", "Qg", "Qu", "Qd", "absmax_g", "absmax_u", "absmax_d", "codebook")]
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
 class Adapters(ctypes.Structure):
@@ -113,6 +116,7 @@ def lib() -> ctypes.CDLL:
         "lora_rmsnorm_fwd": [i64, i32, f32, vp, vp, vp, vp, vp],
         "lora_rmsnorm_bwd": [i64, i32, vp, vp, vp, vp, vp, vp],
         "lora_quantize_4bit": [vp, i64, i32, vp, vp, vp, vp],
+        "lora_quantize_absmax8": [vp, i64, i32, vp, vp, vp],
         "lora_merge_weights": [i64, i64, i32, f32, vp, vp, vp, vp, vp],
         "lora_qkv_ctx_layout_get": [ctypes.POINTER(QkvDims), ctypes.POINTER(QkvCtxLayout)],
         "lora_qkv_workspace_bytes": [ctypes.POINTER(QkvDims), ctypes.POINTER(ctypes.c_size_t)],
@@ -204,9 +208,12 @@ def ctx_views(dims: Dims, ctx):
                 Pd=v(L.Pd, T * rp, torch.bfloat16, (T, rp)))
 
 
-def make_weights(Wg=None, Wu=None, Wd=None, Qg=None, Qu=None, Qd=None, absmax_g=None, absmax_u=None,
-                 absmax_d=None, codebook=None) -> Weights:
-    return Weights(*[_p(t) for t in (Wg, Wu, Wd, Qg, Qu, Qd, absmax_g, absmax_u, absmax_d, codebook)])
+def make_weights(**tensors) -> Weights:
+    """Weights struct from tensors named as its fields (the others NULL)."""
+    unknown = set(tensors) - set(WEIGHT_FIELDS)
+    if unknown:
+        raise TypeError(f"unknown weight fields {sorted(unknown)}")
+    return Weights(*[_p(tensors.get(n)) for n in WEIGHT_FIELDS])
 
 
 def make_adapters(Ag, Bg, Au, Bu, Ad, Bd) -> Adapters:
@@ -254,6 +261,12 @@ def lora_rmsnorm_bwd(dH, X, w, rstd, dX, stream=None):
 def lora_quantize_4bit(W, codebook, codes, absmax, block=64, stream=None):
     _check(lib().lora_quantize_4bit(_p(W), W.numel(), block, _p(codebook), _p(codes), _p(absmax),
                                     _stream(stream)))
+
+
+def lora_quantize_absmax8(absmax, codes8, scale2, block2=256, stream=None):
+    """Double quantisation of the 4-bit block constants: absmax fp32 -> codes8 uint8, scale2 fp32."""
+    _check(lib().lora_quantize_absmax8(_p(absmax), absmax.numel(), block2, _p(codes8), _p(scale2),
+                                       _stream(stream)))
 
 
 GEMM_CTA_PAIR = 1

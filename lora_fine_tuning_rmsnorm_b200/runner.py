@@ -41,10 +41,11 @@ class Problem:
         self.ctx = ops.alloc_ctx(self.dims, device)
         self.ws = ops.alloc_workspace(self.dims, device)
 
-    def use_4bit(self, codebook, drop_bf16: bool = True):
+    def use_4bit(self, codebook, drop_bf16: bool = True, double_quant: bool = False):
         """Quantise the frozen Wg, Wu, Wd to 4-bit blockwise codes on the GPU (one-off
         set-up, lora_quantize_4bit) and switch the weights to them.  `codebook` is the
-        16-entry fp32 code table (an input of the method)."""
+        16-entry fp32 code table (an input of the method).  double_quant also quantises
+        the block constants (lora_quantize_absmax8) and switches to that format."""
         cb = torch.as_tensor(np.asarray(codebook, dtype=np.float32)).to(self.device)
         codes, absmax = {}, {}
         for k, name in (("g", "Wg"), ("u", "Wu"), ("d", "Wd")):
@@ -57,6 +58,18 @@ class Problem:
         self.q4 = (codes, absmax, cb)
         self.weights = ops.make_weights(Qg=codes["g"], Qu=codes["u"], Qd=codes["d"], absmax_g=absmax["g"],
                                         absmax_u=absmax["u"], absmax_d=absmax["d"], codebook=cb)
+        if double_quant:
+            a8, s2 = {}, {}
+            for k in ("g", "u", "d"):
+                n = absmax[k].numel()
+                a8[k] = torch.empty(n, dtype=torch.uint8, device=self.device)
+                s2[k] = torch.empty((n + 255) // 256, dtype=torch.float32, device=self.device)
+                ops.lora_quantize_absmax8(absmax[k], a8[k], s2[k])
+            self.dims.wfmt = ops.WFMT_4BIT_DQ
+            self.dq = (a8, s2)
+            self.weights = ops.make_weights(Qg=codes["g"], Qu=codes["u"], Qd=codes["d"], codebook=cb,
+                                            absmax8_g=a8["g"], absmax8_u=a8["u"], absmax8_d=a8["d"],
+                                            scale2_g=s2["g"], scale2_u=s2["u"], scale2_d=s2["d"])
         if drop_bf16:  # the bf16 copies are no longer needed on the device
             for name in ("Wg", "Wu", "Wd"):
                 self.t[name] = None

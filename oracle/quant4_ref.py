@@ -97,8 +97,11 @@ def quantize_absmax8(absmax: np.ndarray, block2: int = 256):
     s = np.repeat(scale2.astype(np.float64), block2)[:n]
     lhs = 510.0 * a.astype(np.float64)                               # exact
     thr = np.arange(1, 510, 2, dtype=np.float64)                     # 2j - 1, j = 1..255
-    codes8 = (lhs[:, None] > s[:, None] * thr[None, :]).sum(axis=1)  # exact products, strict: ties go down
-    return codes8.astype(np.uint8), scale2
+    codes8 = np.empty(n, dtype=np.uint8)
+    for i0 in range(0, n, 65536):                                    # row chunks bound the memory
+        sl = slice(i0, i0 + 65536)
+        codes8[sl] = (lhs[sl, None] > s[sl, None] * thr[None, :]).sum(axis=1)  # exact; strict: ties go down
+    return codes8, scale2
 
 
 def dequantize_absmax8(codes8: np.ndarray, scale2: np.ndarray, block2: int = 256) -> np.ndarray:

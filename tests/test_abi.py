@@ -188,3 +188,25 @@ def test_ce_argument_checks(L):
                          None) == -2                        # loss not 4-byte aligned
     assert L.lora_ce_fwd(ctypes.byref(dims), good, None, good, good, good, good, good, good, None) == -1
     assert L.lora_ce_bwd(ctypes.byref(dims), good, good, good, good, good, float("nan"), good, good, None) == -1
+
+
+def test_double_quant_argument_checks(L):
+    good = ctypes.c_void_p(0x1000)
+    assert L.lora_quantize_absmax8(good, 1000, 128, good, good, None) == -3        # block2 must be 256
+    assert L.lora_quantize_absmax8(good, 0, 256, good, good, None) == -1
+    assert L.lora_quantize_absmax8(good, 1000, 256, good, ctypes.c_void_p(0x1004), None) == -2
+    dims = ops.make_dims(64, 256, 512, 8, wfmt=ops.WFMT_4BIT_DQ)
+    out = ctypes.c_size_t()
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == 0
+    plain = ops.workspace_bytes(ops.make_dims(64, 256, 512, 8, wfmt=ops.WFMT_4BIT))
+    assert out.value >= plain + 3 * (256 * 512 // 64) * 4           # the expanded constants
+    dims = ops.make_dims(64, 256, 344, 8, wfmt=ops.WFMT_4BIT_DQ)
+    assert L.lora_mlp_workspace_bytes(ctypes.byref(dims), ctypes.byref(out)) == -3   # f % 256
+    # the double-quantised format needs its own constant arrays, not absmax
+    dims = ops.make_dims(64, 256, 512, 8, wfmt=ops.WFMT_4BIT_DQ)
+    w = ops.make_weights(Qg=None)
+    for f in ("Qg", "Qu", "Qd", "codebook", "absmax_g", "absmax_u", "absmax_d"):
+        setattr(w, f, 0x1000)
+    a = ops.Adapters(*([0x1000] * 6))
+    rc = L.lora_mlp_fwd(ctypes.byref(dims), good, good, ctypes.byref(w), ctypes.byref(a), good, good, good, None)
+    assert rc == -1 and b"NULL" in L.lora_mlp_last_error()
