@@ -40,12 +40,14 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kDqWarps = 8;  // 4-bit weights: warps that expand codes into bf16 B tiles
 constexpr int kDqGroups = 2;  // ... in groups that take alternate stages
 constexpr int kCodeRing = 8;  // 4-bit weights: entries of the code ring (codes + absmax of one stage)
+// Code-ring entries for MT M tiles per unit (two tiles per unit leave less shared memory)
+__host__ __device__ constexpr int code_ring(int mt) { return mt == 2 ? 4 : kCodeRing; }
 // 4-bit CTAs add the dequant warps and one warp that fills the code ring
 __host__ __device__ constexpr int gemm_threads(int q4) { return kGemmThreads + (q4 ? 32 * kDqWarps + 32 : 0); }
 
 // Shared-memory layout of the 4-bit operand in one CTA (host and device use the same):
-// each stage is [A 16 KB][expanded bf16 B: slots x b_unit]; each of the kCodeRing code-ring
-// entries is [codes: slots x q_unit][absmax: slots x m_unit] (cr_bytes, 1 KB aligned).
+// each stage is [A: MT x 16 KB][expanded bf16 B: slots x b_unit]; each of the code_ring(MT)
+// code-ring entries is [codes: slots x q_unit][absmax: slots x m_unit] (cr_bytes, 1 KB aligned).
 // A unit is one B operand (one accumulator, or one gate/up branch) as held by this CTA:
 // `cols` B rows (K-major) or B columns (MN-major) by 64 K, i.e. `cols` 128-byte smem rows.
 struct Q4Layout {
@@ -108,6 +110,8 @@ struct GemmArgs {
   int stages;
   uint32_t stage_bytes;
   uint32_t tmem_cols;
+  int nbuf;        // accumulator sets in TMEM: 2 (the epilogue drains one while the MMA fills the
+                   // other) or 1 (a unit of MT = 2 M tiles fills all 512 columns)
   void* out[3];
   long long ld_out;
   long long split_stride;  // EPI_F32: element offset between the partial sums of K splits
@@ -124,6 +128,8 @@ struct GemmArgs {
   int test_no_loads;      // test of the bounded waits: the producer copies nothing and arms no
                           // barrier, so the MMA's first wait runs out (single-CTA tiles only)
   int out_add;            // EPI_F32: add into the fp32 output instead of overwriting it
+  int l2_prefetch;        // > 0: the copy warp also prefetches into L2 the A / B tiles of the
+                          // k-block this many steps ahead in the same segment
   // cross-entropy epilogues (rows = tokens, columns = vocabulary entries ce_col0 + n)
   const int* ce_labels;   // label of each row; outside [0, ce_V) = left out of the loss
   const float* ce_lse;    // EPI_CE_DZ: logsumexp of each row (from the forward)
@@ -218,14 +224,14 @@ static __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, co
 // FUSE = 1 (gate/up): the two B operands of a segment are two halves of ONE
 // N = 2 * bn MMA (branch 0 -> columns [0, bn), branch 1 -> [bn, 2 bn)), so a k-step
 // issues one wide MMA instead of two; with PAIR = 2, CTA rank r loads branch r.
-template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
+template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4, int MT>
 __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                               uint32_t empty0, const WaitCtl& wc, uint32_t rank) {
   const Sched sc = sched_of(p);
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   // launch constants in registers (see Sched)
   const int M = p.M, N = p.N, bn = p.bn, nstages = p.stages, nseg = p.nseg;
-  const int mn3d_a = p.mn3d_a, mn3d_b = p.mn3d_b, no_loads = p.test_no_loads;
+  const int mn3d_a = p.mn3d_a, mn3d_b = p.mn3d_b, no_loads = p.test_no_loads, pf = p.l2_prefetch;
   const uint32_t stage_bytes = p.stage_bytes;
   const CUtensorMap* maps = p.maps;
   const int bnl = bn / PAIR;  // B rows (N) held by this CTA
@@ -239,7 +245,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   for (int t = unit0; t < sc.total && ok; t += nunits) {
     int mt, nt, ks;
     decode_tile(sc, t, mt, nt, ks);
-    const int mbase = mt * BM * PAIR, n0 = nt * bn;
+    const int mbase = mt * BM * PAIR * MT, n0 = nt * bn;
     for (int s = 0; s < nseg && ok; ++s) {
       const SegR sg = seg_of(p, s);
       int kb0, kb1;
@@ -247,10 +253,13 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
       // Bytes landing per stage for CTA rank rr.  Boxes that would lie entirely
       // outside the matrix are skipped: the rows / columns they feed are never stored.
       auto bytes_of = [&](uint32_t rr) -> uint32_t {
-        const int m0r = mbase + static_cast<int>(rr) * BM;
         uint32_t by = 0;
-        if (A_MN) by += mn3d_a ? (m0r < M ? 16384u : 0u) : (m0r < M ? 8192u : 0u) + (m0r + 64 < M ? 8192u : 0u);
-        else by += (m0r < M ? a_bytes : 0u);
+#pragma unroll
+        for (int h = 0; h < MT; ++h) {  // M tile h of the unit: rows mbase + h * BM * PAIR + ...
+          const int m0r = mbase + h * BM * PAIR + static_cast<int>(rr) * BM;
+          if (A_MN) by += mn3d_a ? (m0r < M ? 16384u : 0u) : (m0r < M ? 8192u : 0u) + (m0r + 64 < M ? 8192u : 0u);
+          else by += (m0r < M ? a_bytes : 0u);
+        }
         const int nb0 = FUSE ? n0 : n0 + static_cast<int>(rr) * bnl;
         uint32_t bb = 0;
         if (B_MN) {
@@ -312,8 +321,10 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         } else if (A_MN) {
           if (m0 < M) load(sA, am, m0, sg.a_k0 + k);
           if (m0 + 64 < M) load(sA + 8192, am, m0 + 64, sg.a_k0 + k);
-        } else if (m0 < M) {
-          load(sA, am, sg.a_k0 + k, m0);
+        } else {
+#pragma unroll
+          for (int h = 0; h < MT; ++h)
+            if (m0 + h * BM * PAIR < M) load(sA + h * a_bytes, am, sg.a_k0 + k, m0 + h * BM * PAIR);
         }
         hint = sg.b_hint;
         if (Q4 && sg.q4) {
@@ -321,7 +332,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
         } else if (FUSE) {
           // branch r fills B rows [r * bn, (r + 1) * bn) of the wide tile; a CTA of a
           // pair holds only its own branch
-          const uint32_t sB = sA + a_bytes;
+          const uint32_t sB = sA + MT * a_bytes;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             if (PAIR == 2 && static_cast<uint32_t>(r) != rank) continue;
@@ -332,7 +343,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
 #pragma unroll
           for (int a = 0; a < NACC; ++a) {
             if (seg_bmap(sg, a) < 0) continue;
-            const uint32_t sB = sA + a_bytes + a * b_bytes;
+            const uint32_t sB = sA + MT * a_bytes + a * b_bytes;
             const CUtensorMap* bm = maps + seg_bmap(sg, a);
             if (B_MN && mn3d_b) {
               if (nb0 < N) load3(sB, bm, seg_bk0(sg, a) + k, nb0 / 64);
@@ -342,6 +353,17 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
             } else if (nb0 < N) {
               load(sB, bm, seg_bk0(sg, a) + k, nb0);
             }
+          }
+        }
+        if (pf && kb + pf < kb1) {  // warm L2 with a later k-block's tiles (K-major operands)
+          const int kp = k + pf * BK;
+          if (!A_MN)
+            for (int h = 0; h < MT; ++h)
+              if (m0 + h * BM * PAIR < M) tma_prefetch_l2_2d(am, sg.a_k0 + kp, m0 + h * BM * PAIR);
+          if (!B_MN && !(Q4 && sg.q4)) {
+            if (FUSE) tma_prefetch_l2_2d(maps + seg_bmap(sg, PAIR == 2 ? static_cast<int>(rank) : 0),
+                                         seg_bk0(sg, PAIR == 2 ? static_cast<int>(rank) : 0) + kp, n0);
+            else if (nb0 < N && seg_bmap(sg, 0) >= 0) tma_prefetch_l2_2d(maps + seg_bmap(sg, 0), seg_bk0(sg, 0) + kp, nb0);
           }
         }
         issued_mask |= 1u << stage;
@@ -363,7 +385,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4>
+template <int A_MN, int B_MN, int NACC, int PAIR, int FUSE, int Q4, int MT>
 __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint32_t full0,
                                          uint32_t empty0, uint32_t tfull0, uint32_t tempty0,
                                          uint32_t drain_bar, uint32_t tmem_base,
@@ -377,7 +399,7 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
   const uint32_t tiles_u32 = smem_u32(tiles);
   // launch constants in registers: the asm statements below clobber memory, which would
   // otherwise make the compiler re-read them from the parameter space in the issue loop
-  const int nstages = p.stages, nseg = p.nseg, bn = p.bn;
+  const int nstages = p.stages, nseg = p.nseg, bn = p.bn, nbuf = p.nbuf;
   const uint32_t stage_bytes = p.stage_bytes;
   int stage = 0;
   uint32_t phase = 0;
@@ -387,13 +409,13 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
   for (int t = unit0; t < total && ok; t += nunits, ++it) {
     int mt, nt, ks;
     decode_tile(sc, t, mt, nt, ks);
-    const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
+    const uint32_t buf = nbuf == 2 ? (it & 1) : 0, aphase = nbuf == 2 ? (it >> 1) & 1 : it & 1;
     if (!mbar_wait(tempty0 + 8 * buf, aphase ^ 1, wc, kDevTimeoutMma)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    uint32_t started = 0;
+    uint32_t started = 0;  // bit h * NACC + a: accumulator a of M tile h has its first product
     for (int s = 0; s < nseg && ok; ++s) {
       const SegR sg = seg_of(p, s);
       int kb0, kb1;
@@ -425,31 +447,36 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, uint8_t* tiles, uint
         }
         // descriptors of k-step 0; later k-steps only move the start address
         // (+32 B in a K-major 128-byte row, +2048 B = 16 rows for MN-major)
-        const uint64_t ad0 = A_MN ? sdesc_sw128(sA, 8192, 1024) : sdesc_sw128(sA, 16, 1024);
         constexpr uint32_t a_step = A_MN ? (2048 >> 4) : (32 >> 4);
         constexpr uint32_t b_step = B_MN ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
-        for (int a = 0; a < (FUSE ? 1 : NACC); ++a) {
-          if (!((bmask >> a) & 1u)) continue;
-          const uint32_t sB = sA + a_bytes + a * b_bytes;
-          const uint64_t bd0 = B_MN ? sdesc_sw128(sB, 8192, 1024) : sdesc_sw128(sB, 16, 1024);
-          const uint32_t d = tmem_base + buf * (NACC * bn) + a * bn;
-          const uint32_t acc0 = (started >> a) & 1;
-          if (rem >= BK) {
+        for (int h = 0; h < MT; ++h) {  // M tile h: its own A sub-tile and accumulator set
+          const uint32_t sAh = sA + h * a_bytes;
+          const uint64_t ad0 = A_MN ? sdesc_sw128(sAh, 8192, 1024) : sdesc_sw128(sAh, 16, 1024);
 #pragma unroll
-            for (int j = 0; j < BK / 16; ++j) {
-              if (PAIR == 1) mma_bf16(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
-              else mma_bf16_pair(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+          for (int a = 0; a < (FUSE ? 1 : NACC); ++a) {
+            if (!((bmask >> a) & 1u)) continue;
+            const uint32_t sB = sA + MT * a_bytes + a * b_bytes;
+            const uint64_t bd0 = B_MN ? sdesc_sw128(sB, 8192, 1024) : sdesc_sw128(sB, 16, 1024);
+            const uint32_t d = tmem_base + buf * (MT * NACC * bn) + h * (NACC * bn) + a * bn;
+            const int bit = h * NACC + a;
+            const uint32_t acc0 = (started >> bit) & 1;
+            if (rem >= BK) {
+#pragma unroll
+              for (int j = 0; j < BK / 16; ++j) {
+                if (PAIR == 1) mma_bf16(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+                else mma_bf16_pair(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+              }
+            } else {
+              const int nsteps = (rem + 15) / 16;
+              for (int j = 0; j < nsteps; ++j) {
+                if (PAIR == 1) mma_bf16(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+                else mma_bf16_pair(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
+              }
             }
-          } else {
-            const int nsteps = (rem + 15) / 16;
-            for (int j = 0; j < nsteps; ++j) {
-              if (PAIR == 1) mma_bf16(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
-              else mma_bf16_pair(d, ad0 + j * a_step, bd0 + j * b_step, idesc, j ? 1u : acc0);
-            }
+            started |= 1u << bit;
+            issued_any = true;
           }
-          started |= 1u << a;
-          issued_any = true;
         }
         // frees the smem stage (in both CTAs of a pair) once these MMAs finish
         if (PAIR == 1) mma_commit(empty0 + 8 * stage);
@@ -488,7 +515,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ float sigmoid_f(float g) { return rcp_approx(1.0f + __expf(-g)); }
 __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
-template <int NACC, int EPI, int PAIR>
+template <int NACC, int EPI, int PAIR, int MT>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0, uint32_t tempty0,
                                               uint32_t tmem_base, const WaitCtl& wc, uint32_t rank) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -499,7 +526,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   // launch constants in registers (see Sched)
   const int bn = p.bn, N = p.N, M = p.M, stream_out = p.stream_out, out_acc_col = p.out_acc_col;
-  const int out_add = p.out_add, nrng = p.nrng;
+  const int out_add = p.out_add, nrng = p.nrng, nbuf = p.nbuf;
   const float alpha = p.alpha;
   const long long ld_out = p.ld_out, ld_in = p.ld_in, split_stride = p.split_stride;
   void* const out0 = p.out[0];
@@ -516,16 +543,19 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   for (int t = unit0; t < total; t += nunits, ++it) {
     int mt, nt, ks;
     decode_tile(sc, t, mt, nt, ks);
-    const uint32_t buf = it & 1, aphase = (it >> 1) & 1;
+    const uint32_t buf = nbuf == 2 ? (it & 1) : 0, aphase = nbuf == 2 ? (it >> 1) & 1 : it & 1;
     int ok = 1;
     if (lane == 0) ok = mbar_wait(tfull0 + 8 * buf, aphase, wc, kDevTimeoutEpilogue) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) break;
     tc_fence_after();
-    const int m0 = mt * BM * PAIR + static_cast<int>(rank) * BM, n0 = nt * bn;
+    const int n0 = nt * bn;
+#pragma unroll 1
+    for (int h = 0; h < MT; ++h) {  // the unit's M tiles, each with its own accumulator set
+    const int m0 = (mt * MT + h) * BM * PAIR + static_cast<int>(rank) * BM;
     const long long row = static_cast<long long>(m0) + 32 * q + lane;
     const bool row_ok = row < M;
-    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (NACC * bn);
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (MT * NACC * bn) + h * (NACC * bn);
 
     if (EPI == EPI_F32 || EPI == EPI_BF16) {
 #pragma unroll 1
@@ -760,6 +790,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         }
       }
     }
+    }  // M tiles of the unit
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
@@ -774,7 +805,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
 // entries once the dequant group that read the entry before has released it.  The copies
 // thus run up to kCodeRing stages ahead of the expansion, outside the per-stage loop of
 // A copy -> expansion -> MMA -> free.
-template <int B_MN, int NACC, int PAIR, int FUSE>
+template <int B_MN, int NACC, int PAIR, int FUSE, int MT>
 __device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* ring, uint32_t crfull0,
                                                    uint32_t crempty0, const WaitCtl& wc, uint32_t rank) {
   const Sched sc = sched_of(p);
@@ -831,7 +862,7 @@ __device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* r
         }
         issued_mask |= 1u << e;
         issued_par = (issued_par & ~(1u << e)) | (phase << e);
-        if (++e == kCodeRing) {
+        if (++e == code_ring(MT)) {
           e = 0;
           phase ^= 1;
         }
@@ -839,7 +870,7 @@ __device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* r
     }
   }
   if (!ok) {  // aborting: no copy into the ring may still be in flight
-    for (int i = 0; i < kCodeRing; ++i)
+    for (int i = 0; i < code_ring(MT); ++i)
       if (issued_mask & (1u << i)) drain_wait(crfull0 + 8 * i, (issued_par >> i) & 1, wc);
   }
 }
@@ -860,7 +891,7 @@ __device__ __forceinline__ void gemm_code_producer(const GemmArgs& p, uint8_t* r
 // A code word holds 8 elements' 4-bit indices in nibble order, which is already the
 // selector layout of prmt: the low 3 bits pick one of 8 entries from a plane pair,
 // bit 3 picks the pair (entries 0..7 or 8..15) through a byte mask.
-template <int B_MN, int NACC, int FUSE, int PAIR>
+template <int B_MN, int NACC, int FUSE, int PAIR, int MT>
 __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, const uint8_t* ring,
                                              uint32_t empty0, uint32_t crfull0, uint32_t crempty0,
                                              uint32_t dq0, const float* tab, const WaitCtl& wc, uint32_t rank) {
@@ -915,7 +946,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
               const int nq = FUSE ? n0 : n0 + static_cast<int>(rank) * (bn / PAIR);
               const uint8_t* q = sQ + slot * QL.q_unit;
               const float* am = sM + slot * (QL.m_unit / 4);
-              uint8_t* dst = base + a_bytes + slot * QL.b_unit;
+              uint8_t* dst = base + MT * a_bytes + slot * QL.b_unit;
               for (int i = gtid; i < QL.cols; i += 32 * kGroupWarps) {
                 const uint4* src;
                 float sc;
@@ -965,7 +996,7 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
             else mbar_arrive_cluster(mapa_shared(dq0 + 8 * stage, 0));
           }
         }
-        if (sg.q4 && ++e == kCodeRing) {
+        if (sg.q4 && ++e == code_ring(MT)) {
           e = 0;
           cphase ^= 1;
         }
@@ -979,14 +1010,15 @@ __device__ __forceinline__ void gemm_dequant(const GemmArgs& p, uint8_t* tiles, 
   }
 }
 
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE, int Q4>
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR, int FUSE, int Q4, int MT>
 static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const __grid_constant__ GemmArgs p) {
   static_assert(!FUSE || (NACC == 2 && !B_MN), "fused wide MMA: two K-major B halves");
   static_assert(!Q4 || !A_MN, "4-bit B: K-major A");
+  static_assert(MT == 1 || (MT == 2 && !A_MN), "two M tiles per unit: K-major A");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = tiles + static_cast<size_t>(p.stages) * p.stage_bytes;  // Q4: code ring
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (Q4 ? static_cast<size_t>(kCodeRing) * p.cr_bytes : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (Q4 ? static_cast<size_t>(code_ring(MT)) * p.cr_bytes : 0));
   const int S = p.stages;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * S;
@@ -995,8 +1027,8 @@ static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const 
   const uint32_t drain_bar = tempty0 + 16;
   const uint32_t dq0 = drain_bar + 8;             // Q4: per stage, one arrival per warp of the expanding group, per CTA
   const uint32_t crfull0 = dq0 + 8 * S;           // Q4: per ring entry, the code copy (TMA bytes)
-  const uint32_t crempty0 = crfull0 + 8 * kCodeRing;  // Q4: per ring entry, released by the expanding group
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? S + 2 * kCodeRing : 0));
+  const uint32_t crempty0 = crfull0 + 8 * code_ring(MT);  // Q4: per ring entry, released by the expanding group
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5 + (Q4 ? S + 2 * code_ring(MT) : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* tab = reinterpret_cast<float*>(tmem_slot + 4);  // Q4: code values replicated per lane, [16][32]
   if (Q4)
@@ -1016,7 +1048,7 @@ static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const 
     mbar_init(drain_bar, 1);
     if (Q4) {
       for (int s = 0; s < S; ++s) mbar_init(dq0 + 8 * s, (kDqWarps / kDqGroups) * PAIR);
-      for (int i = 0; i < kCodeRing; ++i) {
+      for (int i = 0; i < code_ring(MT); ++i) {
         mbar_init(crfull0 + 8 * i, 1);
         mbar_init(crempty0 + 8 * i, kDqWarps / kDqGroups);
       }
@@ -1044,18 +1076,18 @@ static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const 
   const WaitCtl wc{abort_flag, p.status, p.limit_ns};
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, wc, rank);
+    if (lane == 0) gemm_producer<A_MN, B_MN, NACC, PAIR, FUSE, Q4, MT>(p, tiles, full0, empty0, wc, rank);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
-      gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE, Q4>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc, dq0);
+      gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE, Q4, MT>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc, dq0);
     __syncwarp();
   } else if (warp < 2 + kEpiWarps) {
-    gemm_epilogue<NACC, EPI, PAIR>(p, tfull0, tempty0, tmem_base, wc, rank);
+    gemm_epilogue<NACC, EPI, PAIR, MT>(p, tfull0, tempty0, tmem_base, wc, rank);
   } else if (Q4 && warp < 2 + kEpiWarps + kDqWarps) {
-    gemm_dequant<B_MN, NACC, FUSE, PAIR>(p, tiles, ring, empty0, crfull0, crempty0, dq0, tab, wc, rank);
+    gemm_dequant<B_MN, NACC, FUSE, PAIR, MT>(p, tiles, ring, empty0, crfull0, crempty0, dq0, tab, wc, rank);
   } else if (Q4) {
-    if (lane == 0) gemm_code_producer<B_MN, NACC, PAIR, FUSE>(p, ring, crfull0, crempty0, wc, rank);
+    if (lane == 0) gemm_code_producer<B_MN, NACC, PAIR, FUSE, MT>(p, ring, crfull0, crempty0, wc, rank);
     __syncwarp();
   }
   tc_fence_before();

@@ -220,21 +220,24 @@ constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
 
 // Launch one GEMM.  PAIR = 2 runs clusters of two CTAs sharing 256-row tiles
 // (tcgen05 cta_group::2); the caller sets tiles_m = ceil(M / (128 * PAIR)).
-template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1, int FUSE = 0, int Q4 = 0>
+// MT = 2 runs units of two M tiles (2 x 128 x PAIR rows) that share every B stage; the
+// caller sets tiles_m = ceil(M / (128 * PAIR * MT)).
+template <int A_MN, int B_MN, int NACC, int EPI, int PAIR = 1, int FUSE = 0, int Q4 = 0, int MT = 1>
 int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   static_assert(PAIR == 1 || (PAIR == 2 && !A_MN), "CTA pairs take a K-major A operand");
+  static_assert(MT == 1 || (MT == 2 && !A_MN), "two M tiles per unit take a K-major A operand");
   if (a.bn < 16 || a.bn > 256 || a.bn % 16 || (B_MN && a.bn % (64 * PAIR)) || (!B_MN && (a.bn / PAIR) % 8))
     return fail(LORA_ERR_UNSUPPORTED, "internal: bad N tile %d", a.bn);
-  a.stage_bytes = BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
+  a.stage_bytes = MT * BM * BK * 2 + NACC * (a.bn / PAIR) * BK * 2;
   a.cr_bytes = 0;
   if (Q4) {  // 4-bit B: expanded B slots per stage; codes + absmax in a ring of their own
     const Q4Layout QL = q4_layout(a.bn, PAIR, FUSE, B_MN, NACC);
-    a.stage_bytes = BM * BK * 2 + QL.slots * QL.b_unit;
+    a.stage_bytes = MT * BM * BK * 2 + QL.slots * QL.b_unit;
     a.cr_bytes = (QL.slots * (QL.q_unit + QL.m_unit) + 1023) & ~1023u;
   }
   a.stage_bytes = (a.stage_bytes + 1023) & ~1023u;
   const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit code table)
-  const int ring = Q4 ? kCodeRing * static_cast<int>(a.cr_bytes) : 0;
+  const int ring = Q4 ? code_ring(MT) * static_cast<int>(a.cr_bytes) : 0;
   const int avail = kSmemLimit - 1024 - extra - ring;
   a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
   static const int stage_cap = [] {
@@ -243,7 +246,10 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   }();
   if (stage_cap >= 2) a.stages = std::min(a.stages, stage_cap);
   if (a.stages < 2) return fail(LORA_ERR_UNSUPPORTED, "internal: stage does not fit");
-  int cols = 2 * NACC * a.bn;
+  // accumulator sets: two when they fit in TMEM's 512 columns, else one
+  const int set_cols = MT * NACC * a.bn;
+  a.nbuf = 2 * set_cols <= 512 ? 2 : 1;
+  const int cols = a.nbuf * set_cols;
   uint32_t tc = 32;
   while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
   if (tc > 512) return fail(LORA_ERR_UNSUPPORTED, "internal: TMEM columns %d > 512", cols);
@@ -256,7 +262,7 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   if (tiles <= 0) return LORA_OK;
   if (tiles > 0x7fffffffLL) return fail(LORA_ERR_UNSUPPORTED, "too many tiles");
   const int units = static_cast<int>(std::min<long long>(tiles, sm_count() / PAIR));
-  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR, FUSE, Q4>;
+  auto kern = gemm_kernel<A_MN, B_MN, NACC, EPI, PAIR, FUSE, Q4, MT>;
   CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   PhaseScope ps(st, phase);
   if (PAIR == 1) {
@@ -414,6 +420,11 @@ inline GemmArgs new_args(int* status) {
   a.splits = 1;
   a.alpha = 1.0f;
   a.status = status;
+  static const int l2_prefetch = [] {
+    const char* e = getenv("LORA_MLP_L2_PREFETCH");  // tuning knob: L2 prefetch distance in k-blocks
+    return e ? atoi(e) : 0;
+  }();
+  a.l2_prefetch = l2_prefetch;
   for (int s = 0; s < kMaxSegs; ++s) a.seg[s].b_map[0] = a.seg[s].b_map[1] = -1;
   return a;
 }
@@ -473,6 +484,25 @@ inline TileChoice pick_tiles(long long T, int N, bool mn_major) {
     }
   }
   return best;
+}
+
+// M tiles per unit for a K-major-A GEMM with M = T rows and N columns in tiles of bn:
+// two (sharing every B stage: a quarter fewer operand bytes per FLOP, and for 4-bit
+// weights half the expansion work per FLOP, but a single accumulator set in TMEM) when
+// the halved unit count still fills the waves of a 148-SM part about as well.
+// LORA_MLP_MT=1 or 2 forces the choice (tuning comparison).
+inline int pick_mt(long long T, int pair, int bn, long long N) {
+  static const int force = [] {
+    const char* e = getenv("LORA_MLP_MT");
+    return e ? atoi(e) : 0;
+  }();
+  if (force == 1 || force == 2) return force;
+  const double per_wave = 148.0 / pair;
+  const long long nt = (N + bn - 1) / bn;
+  const long long u1 = ((T + 128LL * pair - 1) / (128LL * pair)) * nt;
+  const long long u2 = ((T + 256LL * pair - 1) / (256LL * pair)) * nt;
+  const double w1 = std::ceil(u1 / per_wave), w2 = std::ceil(u2 / per_wave);
+  return (u2 >= 2 * per_wave && 2.0 * 0.9 * w2 < w1) ? 2 : 1;
 }
 
 // Rank-r projection out[T x cols] (bf16) = scale * sum of K-split fp32 partials.

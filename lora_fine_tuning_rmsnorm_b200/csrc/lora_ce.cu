@@ -98,12 +98,14 @@ int lora_ce_fwd(const lora_ce_dims* D, const void* H, const void* W, const int32
     // tiles M-fastest: every LM-head tile is read from HBM once and meets all token
     // tiles while it is in L2; H (re-read by every vocabulary tile) is kept in L2
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, V) : 1;
     a.M = static_cast<int>(T); a.N = V; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (V + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (V + bn - 1) / bn;
     a.out[0] = part; a.out[1] = zlab;
     a.ce_labels = labels; a.ce_col0 = 0; a.ce_V = V;
     nparts = 2 * a.tiles_n;
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_LSE, 2>(a, st, PH_CE_LSE)));
+    if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_LSE, 2, 0, 0, 2>(a, st, PH_CE_LSE)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_LSE, 2>(a, st, PH_CE_LSE)));
     else TRY((launch_gemm<0, 0, 1, EPI_CE_LSE>(a, st, PH_CE_LSE)));
   }
   {
@@ -144,12 +146,14 @@ int lora_ce_bwd(const lora_ce_dims* D, const void* H, const void* W, const int32
       TRY(map_k(&a.maps[1], Wc, N, d, d, bn / pair));
       set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
       set_hints(a, HINT_EVICT_LAST, HINT_NONE);
+      const int mt = pair == 2 ? pick_mt(T, pair, bn, N) : 1;
       a.M = static_cast<int>(T); a.N = N; a.bn = bn;
-      a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (N + bn - 1) / bn;
+      a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (N + bn - 1) / bn;
       a.out[0] = dZ; a.ld_out = chunk;
       a.ce_labels = labels; a.ce_lse = lse; a.ce_count = D->reduction == LORA_CE_MEAN ? n_valid : nullptr;
       a.ce_g = dloss; a.ce_col0 = v0; a.ce_V = V;
-      if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_DZ, 2>(a, st, PH_CE_DZ)));
+      if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_DZ, 2, 0, 0, 2>(a, st, PH_CE_DZ)));
+      else if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_DZ, 2>(a, st, PH_CE_DZ)));
       else TRY((launch_gemm<0, 0, 1, EPI_CE_DZ>(a, st, PH_CE_DZ)));
     }
     // dH (+)= dZ[:, 0:N] W[v0 : v0 + N]   (fp32; the LM head read MN-major)

@@ -437,13 +437,15 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 6; a.seg[0].b_am[1] = 7;
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
     a.codebook = W->codebook;
+    const int mt = pair == 2 ? pick_mt(T, pair, 128, f) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);
-    set_band(a, 16);
+    set_band(a, 16 / mt);
     a.stream_out = 1;
-    if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1, 1>(a, st, PH_GATEUP)));
+    if (mt == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1, 1, 2>(a, st, PH_GATEUP)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1, 1>(a, st, PH_GATEUP)));
     else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1, 1>(a, st, PH_GATEUP)));
   } else {
     GemmArgs a = new_args(status);
@@ -456,13 +458,15 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, 128, f) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + 127) / 128;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);  // H is re-read by every N tile: keep it in L2
-    set_band(a, 16);
+    set_band(a, 16 / mt);
     a.stream_out = 1;
-    if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1>(a, st, PH_GATEUP)));
+    if (mt == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1, 0, 2>(a, st, PH_GATEUP)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1>(a, st, PH_GATEUP)));
     else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1>(a, st, PH_GATEUP)));
   }
   // S4a: Pd = s * Act Ad^T

@@ -67,6 +67,8 @@ class Problem:
                 ops.lora_quantize_absmax8(absmax[k], a8[k], s2[k])
             self.dims.wfmt = ops.WFMT_4BIT_DQ
             self.dq = (a8, s2)
+            # this format's workspace also holds the expanded constants: size it anew
+            self.ws = ops.alloc_workspace(self.dims, self.device)
             self.weights = ops.make_weights(Qg=codes["g"], Qu=codes["u"], Qd=codes["d"], codebook=cb,
                                             absmax8_g=a8["g"], absmax8_u=a8["u"], absmax8_d=a8["d"],
                                             scale2_g=s2["g"], scale2_u=s2["u"], scale2_d=s2["d"])
