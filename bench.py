@@ -36,7 +36,7 @@ METRIC = "LoRA-MLP fwd+bwd tokens/s at Llama-3-8B shape; % of bf16 tensor-core p
 UNIT = "tokens/s"
 CODEBOOK_FILE = os.path.join(ROOT, "tests", "golden", "codebook16.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
-KERNEL_SOURCES = ("gemm_sm100.cuh", "ptx.cuh", "lora_mlp.cu")
+KERNEL_SOURCES = ("gemm_sm100.cuh", "ptx.cuh", "host.cuh", "lora_mlp.cu")
 GEMM_PHASES = ("gemm_gate_up_swiglu", "gemm_down", "gemm_dact_swiglu_bwd", "gemm_dH")
 
 

@@ -128,8 +128,6 @@ struct GemmArgs {
   int test_no_loads;      // test of the bounded waits: the producer copies nothing and arms no
                           // barrier, so the MMA's first wait runs out (single-CTA tiles only)
   int out_add;            // EPI_F32: add into the fp32 output instead of overwriting it
-  int l2_prefetch;        // > 0: the copy warp also prefetches into L2 the A / B tiles of the
-                          // k-block this many steps ahead in the same segment
   // cross-entropy epilogues (rows = tokens, columns = vocabulary entries ce_col0 + n)
   const int* ce_labels;   // label of each row; outside [0, ce_V) = left out of the loss
   const float* ce_lse;    // EPI_CE_DZ: logsumexp of each row (from the forward)
@@ -231,7 +229,7 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
   const int unit0 = blockIdx.x / PAIR, nunits = gridDim.x / PAIR;
   // launch constants in registers (see Sched)
   const int M = p.M, N = p.N, bn = p.bn, nstages = p.stages, nseg = p.nseg;
-  const int mn3d_a = p.mn3d_a, mn3d_b = p.mn3d_b, no_loads = p.test_no_loads, pf = p.l2_prefetch;
+  const int mn3d_a = p.mn3d_a, mn3d_b = p.mn3d_b, no_loads = p.test_no_loads;
   const uint32_t stage_bytes = p.stage_bytes;
   const CUtensorMap* maps = p.maps;
   const int bnl = bn / PAIR;  // B rows (N) held by this CTA
@@ -353,17 +351,6 @@ __device__ __forceinline__ void gemm_producer(const GemmArgs& p, uint8_t* tiles,
             } else if (nb0 < N) {
               load(sB, bm, seg_bk0(sg, a) + k, nb0);
             }
-          }
-        }
-        if (pf && kb + pf < kb1) {  // warm L2 with a later k-block's tiles (K-major operands)
-          const int kp = k + pf * BK;
-          if (!A_MN)
-            for (int h = 0; h < MT; ++h)
-              if (m0 + h * BM * PAIR < M) tma_prefetch_l2_2d(am, sg.a_k0 + kp, m0 + h * BM * PAIR);
-          if (!B_MN && !(Q4 && sg.q4)) {
-            if (FUSE) tma_prefetch_l2_2d(maps + seg_bmap(sg, PAIR == 2 ? static_cast<int>(rank) : 0),
-                                         seg_bk0(sg, PAIR == 2 ? static_cast<int>(rank) : 0) + kp, n0);
-            else if (nb0 < N && seg_bmap(sg, 0) >= 0) tma_prefetch_l2_2d(maps + seg_bmap(sg, 0), seg_bk0(sg, 0) + kp, nb0);
           }
         }
         issued_mask |= 1u << stage;
@@ -648,8 +635,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         for (int h = 0; h < 2; ++h) {
           if (row_ok && n + 8 * h < N) {
             const long long off = row * ld_in + n + 8 * h;
-            gv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in0) + off));
-            uv[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in1) + off));
+            // G and U are read once here: evict-first, so they do not displace the operand tiles
+            gv[h] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in0) + off));
+            uv[h] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in1) + off));
           } else {
             gv[h] = make_uint4(0, 0, 0, 0);
             uv[h] = make_uint4(0, 0, 0, 0);

@@ -420,11 +420,6 @@ inline GemmArgs new_args(int* status) {
   a.splits = 1;
   a.alpha = 1.0f;
   a.status = status;
-  static const int l2_prefetch = [] {
-    const char* e = getenv("LORA_MLP_L2_PREFETCH");  // tuning knob: L2 prefetch distance in k-blocks
-    return e ? atoi(e) : 0;
-  }();
-  a.l2_prefetch = l2_prefetch;
   for (int s = 0; s < kMaxSegs; ++s) a.seg[s].b_map[0] = a.seg[s].b_map[1] = -1;
   return a;
 }
@@ -486,12 +481,15 @@ inline TileChoice pick_tiles(long long T, int N, bool mn_major) {
   return best;
 }
 
-// M tiles per unit for a K-major-A GEMM with M = T rows and N columns in tiles of bn:
-// two (sharing every B stage: a quarter fewer operand bytes per FLOP, and for 4-bit
-// weights half the expansion work per FLOP, but a single accumulator set in TMEM) when
-// the halved unit count still fills the waves of a 148-SM part about as well.
-// LORA_MLP_MT=1 or 2 forces the choice (tuning comparison).
-inline int pick_mt(long long T, int pair, int bn, long long N) {
+// M tiles per unit for a K-major-A GEMM with M = T rows and N columns in tiles of bn.
+// Two M tiles per unit share every B stage (a quarter fewer operand bytes per FLOP, and
+// for 4-bit weights half the expansion work per FLOP) but leave one accumulator set in
+// TMEM, so the epilogue no longer overlaps the next unit's main loop.  `gain` is the
+// measured per-FLOP time of MT = 2 relative to MT = 1 for the kind of GEMM (8B shape:
+// 4-bit gate/up 0.79, cross-entropy logits 0.81-0.87, bf16 gate/up with its three-output
+// epilogue 1.02); MT = 2 is taken when its waves of a 148-SM part cost less.
+// LORA_MLP_MT=1 or 2 forces the choice (tuning comparison, tests).
+inline int pick_mt(long long T, int pair, int bn, long long N, double gain) {
   static const int force = [] {
     const char* e = getenv("LORA_MLP_MT");
     return e ? atoi(e) : 0;
@@ -502,8 +500,11 @@ inline int pick_mt(long long T, int pair, int bn, long long N) {
   const long long u1 = ((T + 128LL * pair - 1) / (128LL * pair)) * nt;
   const long long u2 = ((T + 256LL * pair - 1) / (256LL * pair)) * nt;
   const double w1 = std::ceil(u1 / per_wave), w2 = std::ceil(u2 / per_wave);
-  return (u2 >= 2 * per_wave && 2.0 * 0.9 * w2 < w1) ? 2 : 1;
+  return (u2 >= per_wave && 2.0 * gain * w2 < w1) ? 2 : 1;
 }
+
+// Expected MT = 2 gains by GEMM kind (see pick_mt).
+constexpr double kMtGain4bit = 0.8, kMtGainCe = 0.85, kMtGainBf16Swiglu = 1.02;
 
 // Rank-r projection out[T x cols] (bf16) = scale * sum of K-split fp32 partials.
 // The GEMM args must already hold maps/segments/M/N/bn/tiles and NACC columns.

@@ -98,7 +98,7 @@ int lora_ce_fwd(const lora_ce_dims* D, const void* H, const void* W, const int32
     // tiles M-fastest: every LM-head tile is read from HBM once and meets all token
     // tiles while it is in L2; H (re-read by every vocabulary tile) is kept in L2
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);
-    const int mt = pair == 2 ? pick_mt(T, pair, bn, V) : 1;
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, V, kMtGainCe) : 1;
     a.M = static_cast<int>(T); a.N = V; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (V + bn - 1) / bn;
     a.out[0] = part; a.out[1] = zlab;
@@ -146,7 +146,7 @@ int lora_ce_bwd(const lora_ce_dims* D, const void* H, const void* W, const int32
       TRY(map_k(&a.maps[1], Wc, N, d, d, bn / pair));
       set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
       set_hints(a, HINT_EVICT_LAST, HINT_NONE);
-      const int mt = pair == 2 ? pick_mt(T, pair, bn, N) : 1;
+      const int mt = pair == 2 ? pick_mt(T, pair, bn, N, kMtGainCe) : 1;
       a.M = static_cast<int>(T); a.N = N; a.bn = bn;
       a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (N + bn - 1) / bn;
       a.out[0] = dZ; a.ld_out = chunk;

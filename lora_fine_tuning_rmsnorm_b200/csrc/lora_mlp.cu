@@ -437,7 +437,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 6; a.seg[0].b_am[1] = 7;
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
     a.codebook = W->codebook;
-    const int mt = pair == 2 ? pick_mt(T, pair, 128, f) : 1;
+    const int mt = pair == 2 ? pick_mt(T, pair, 128, f, kMtGain4bit) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
@@ -458,7 +458,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
-    const int mt = pair == 2 ? pick_mt(T, pair, 128, f) : 1;
+    const int mt = pair == 2 ? pick_mt(T, pair, 128, f, kMtGainBf16Swiglu) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
@@ -492,13 +492,15 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 4;
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
     a.codebook = W->codebook;
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, d, kMtGain4bit) : 1;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
     if (D->residual) { a.in[0] = X; a.ld_in = d; }  // Y = X + ...
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 1>(a, st, PH_DOWN)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 1, 2>(a, st, PH_DOWN)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 1>(a, st, PH_DOWN)));
     else TRY((launch_gemm<0, 0, 1, EPI_BF16, 1, 0, 1>(a, st, PH_DOWN)));
   } else {
     GemmArgs a = new_args(status);
@@ -582,13 +584,15 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.seg[0].q4 = 1; a.seg[0].b_am[0] = 4;
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
     a.codebook = W->codebook;
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, f, kMtGain4bit) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
     a.stream_out = 1;
-    set_band(a, 16);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2, 0, 1>(a, st, PH_DACT)));
+    set_band(a, 16 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2, 0, 1, 2>(a, st, PH_DACT)));
+    else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2, 0, 1>(a, st, PH_DACT)));
     else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 1, 0, 1>(a, st, PH_DACT)));
   } else {
     GemmArgs a = new_args(status);
@@ -611,6 +615,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
+    a.stream_out = 1;
     set_band(a, 16);
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
     else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
@@ -647,11 +652,14 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     set_seg(a, 2, 4, 0, 5, 0, -1, 0, rp);
     set_seg(a, 3, 4, rp, 6, 0, -1, 0, rp);
     a.codebook = W->codebook;
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, d, kMtGain4bit) : 1;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
-    set_band(a, 4);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 1>(a, st, PH_DH)));
+    a.stream_out = 1;
+    set_band(a, mt == 2 ? 2 : 4);
+    if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 1, 2>(a, st, PH_DH)));
+    else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 1>(a, st, PH_DH)));
     else TRY((launch_gemm<0, 1, 1, EPI_F32, 1, 0, 1>(a, st, PH_DH)));
   } else {
     GemmArgs a = new_args(status);
@@ -680,6 +688,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
+    a.stream_out = 1;
     set_band(a, 4);
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_DH)));
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));

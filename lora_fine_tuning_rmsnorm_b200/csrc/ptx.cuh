@@ -148,20 +148,6 @@ __device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtens
       : "memory");
 }
 
-// L2-only prefetch of a tensor tile (no shared-memory destination, no barrier): the
-// box is brought into L2 so a later load of it hits there.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int32_t x, int32_t y, int32_t z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-
 // 3-D tiled loads: coordinates {x, y, z} (x innermost).  Used for MN-major
 // operands viewed as [chunk of 64 columns][K row][64 elements], so one box fills
 // several 8 KB chunk-major, 128-byte-swizzled sub-tiles.
