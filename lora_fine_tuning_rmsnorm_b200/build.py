@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "liblora_mlp.so")
 SOURCES = ["lora_mlp.cu", "lora_attn.cu", "lora_ce.cu"]
-HEADERS = ["ptx.cuh", "gemm_sm100.cuh", "rowops.cuh", "host.cuh", "rope.cuh", "ce.cuh"]
+HEADERS = ["ptx.cuh", "gemm_sm100.cuh", "rowops.cuh", "host.cuh", "rope.cuh", "ce.cuh", "lowrank_dual.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -21,6 +21,7 @@
 #include "gemm_sm100.cuh"
 #include "rowops.cuh"
 #include "rope.cuh"
+#include "lowrank_dual.cuh"
 
 namespace lm {
 namespace host {
@@ -57,6 +58,17 @@ inline bool debug_mode() {
   static int v = [] {
     const char* e = getenv("LORA_MLP_DEBUG");
     return (e && e[0] && e[0] != '0') ? 1 : 0;
+  }();
+  return v != 0;
+}
+
+// LORA_MLP_DUAL=0 selects the two-pass form of the rank-r gradients (a projection GEMM
+// for Q and a reduction GEMM for dB, each reading the activation gradient) instead of
+// the single-pass kernel; both compute the same quantities.  Read once per process.
+inline bool dual_enabled() {
+  static int v = [] {
+    const char* e = getenv("LORA_MLP_DUAL");
+    return (e && e[0] == '0') ? 0 : 1;
   }();
   return v != 0;
 }
@@ -159,7 +171,7 @@ inline int map_mn3(CUtensorMap* m, const void* p, uint64_t K, uint64_t MN, uint6
 // --------------------------------------------------------------------- timing
 inline const char* kPhaseNames[LORA_NUM_PHASES] = {
     "rmsnorm_fwd", "proj_P_gate_up", "gemm_gate_up_swiglu", "proj_P_down", "gemm_down",
-    "proj_Q_down", "gemm_dact_swiglu_bwd", "proj_Q_gate_up", "gemm_dH", "rmsnorm_bwd",
+    "lowrank_bwd_down", "gemm_dact_swiglu_bwd", "lowrank_bwd_gate_up", "gemm_dH", "rmsnorm_bwd",
     "zero_grads", "reduce_dA_gate_up", "reduce_dB_gate_up", "reduce_dB_down", "reduce_dA_down",
     "norm_weight_grad", "other", "qkv_gemm", "qkv_gemm_dH", "qkv_lowrank", "o_gemm", "o_gemm_dX", "o_lowrank",
     "rope", "ce_gemm_lse", "ce_finalize", "ce_gemm_dlogits", "ce_gemm_dH"};
@@ -566,6 +578,100 @@ int launch_proj_into(GemmArgs& a, long long T, long long K, int rp, float* part,
   return LORA_OK;
 }
 
+
+// ------------------------------------------------- rank-r gradient pass (dual)
+// One problem of lowrank_dual_kernel: X [T x K] (row stride ldx), B [K x r] (row stride
+// r), P [T x r] (row stride ldp), dB [K x r] fp32 (accumulated).
+struct DualProblem {
+  const void* X;
+  long long ldx;
+  const void* B;
+  const void* P;
+  long long ldp;
+  float* dB;
+};
+struct DualShape {
+  int qn, R, nrb, nc, nreg, grid, slots;
+  long long units;
+};
+// Shape of the unit grid on `max_grid` CTAs; slots = the most CTAs that share one
+// (row region, problem), i.e. the partial slots Q needs.
+inline DualShape dual_shape(long long T, int K, int r, int nx, int max_grid) {
+  DualShape s{};
+  const int rp = round_up(r, 16);
+  s.qn = rp <= 64 ? 64 : 128;
+  s.R = s.qn == 64 ? 4 : 2;  // the Q accumulators (R x qn) and two dB buffers fill 512 TMEM columns
+  s.nrb = static_cast<int>((T + 127) / 128);
+  s.nc = (K + 127) / 128;
+  s.nreg = (s.nrb + s.R - 1) / s.R;
+  s.units = static_cast<long long>(s.nreg) * nx * s.nc;
+  s.grid = static_cast<int>(std::min<long long>(s.units, max_grid));
+  s.slots = 1;
+  for (long long k = 0; k < static_cast<long long>(s.nreg) * nx; ++k) {
+    const long long a = dual_owner(k * s.nc, s.units, s.grid);
+    const long long b = dual_owner(k * s.nc + s.nc - 1, s.units, s.grid);
+    s.slots = std::max(s.slots, static_cast<int>(b - a + 1));
+  }
+  return s;
+}
+// Partial slots to reserve whatever the device's SM count: ranges hold at least
+// floor(U / G) units, so a run of nc units meets at most 1 + ceil((nc - 1) / floor(U / G))
+// of them, largest at the largest grid.
+inline int dual_slots_bound(long long T, int K, int r, int nx) {
+  const DualShape s = dual_shape(T, K, r, nx, kDualMaxGrid);
+  const long long L = std::max<long long>(1, s.units / s.grid);
+  return static_cast<int>(1 + (s.nc - 1 + L - 1) / L);
+}
+
+// Q[:, m rp : (m + 1) rp] = scale * X_m B_m and dB_m += X_m^T P_m for the nx problems
+// (Q bf16, row stride ldq).  `part` holds dual_slots_bound(...) * T * ldq floats; `cnt`
+// holds dual_shape(...).nreg * nx ints that are zero on entry (and left zero).
+inline int launch_dual(const DualProblem* pr, int nx, long long T, int K, int r, float scale, void* Q, int ldq,
+                       float* part, int* cnt, int* status, cudaStream_t st, int phase) {
+  if (nx < 1 || nx > 2 || K < 8 || K % 8 || r < 8 || r % 8 || r > 128)
+    return fail(LORA_ERR_UNSUPPORTED, "internal: bad rank-r pass (nx %d, K %d, r %d)", nx, K, r);
+  DualArgs a;
+  memset(&a, 0, sizeof(a));
+  const int rp = round_up(r, 16);
+  const DualShape s = dual_shape(T, K, r, nx, std::min(sm_count(), kDualMaxGrid));
+  if (s.units <= 0) return LORA_OK;
+  if (s.slots > dual_slots_bound(T, K, r, nx))
+    return fail(LORA_ERR_UNSUPPORTED, "internal: rank-r pass needs %d partial slots", s.slots);
+  for (int m = 0; m < nx; ++m) {
+    TRY(map_k(&a.x[m], pr[m].X, T, K, pr[m].ldx, 128));
+    TRY(map_mn(&a.b[m], pr[m].B, K, r, r));
+    TRY(map_mn(&a.p[m], pr[m].P, T, r, pr[m].ldp));
+    a.dB[m] = pr[m].dB;
+  }
+  a.nx = nx;
+  a.T = T;
+  a.K = K;
+  a.r = r;
+  a.rp = rp;
+  a.qn = s.qn;
+  a.R = s.R;
+  a.nrb = s.nrb;
+  a.nc = s.nc;
+  a.nreg = s.nreg;
+  a.units = s.units;
+  a.scale = scale;
+  a.Q = static_cast<uint16_t*>(Q);
+  a.ldq = ldq;
+  a.part = part;
+  a.part_slot = T * ldq;
+  a.cnt = cnt;
+  a.status = status;
+  a.limit_ns = wait_limit_ns();
+  a.stage_bytes = kDualXBytes + static_cast<uint32_t>(s.qn) * 512u;  // X + P + B tiles: the bytes of one stage's copies
+  a.stages = std::min(kDualMaxStages, (kSmemLimit - 1024 - 256) / static_cast<int>(a.stage_bytes));
+  if (a.stages < 2) return fail(LORA_ERR_UNSUPPORTED, "internal: rank-r stage does not fit");
+  const int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + 256;
+  CUDA_TRY(cudaFuncSetAttribute(lowrank_dual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  PhaseScope ps(st, phase);
+  lowrank_dual_kernel<<<s.grid, kDualThreads, smem, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return LORA_OK;
+}
 
 // Device addresses of the library's own device memory in the current CUDA context
 // (defined in lora_mlp.cu): the no-alloc projection's scratch and the status word of

@@ -12,7 +12,8 @@ namespace {
 
 // --------------------------------------------------------------- layouts
 struct WsLayout {
-  size_t status, Q, Qd, dG, dU, dH, part, am, total;
+  size_t status, Q, Qd, dG, dU, dH, part, am, cnt, total;
+  long long ncnt;  // arrival counters of the rank-r gradient passes (down, then gate/up)
 };
 
 int check_dims(const lora_mlp_dims* D) {
@@ -66,10 +67,14 @@ WsLayout ws_layout(const lora_mlp_dims* D) {
   part = std::max(part, size_t(proj_splits(T, f)) * T * rp);       // Pd = s Act Ad^T
   part = std::max(part, size_t(proj_splits(T, d)) * T * rp);       // Qd = s dY Bd
   part = std::max(part, size_t(proj_splits(T, f)) * T * 2 * rp);   // Q  = s [dG Bg | dU Bu]
+  part = std::max(part, size_t(dual_slots_bound(T, D->d, D->r, 1)) * T * rp);      // single pass: Qd
+  part = std::max(part, size_t(dual_slots_bound(T, D->f, D->r, 2)) * T * 2 * rp);  // single pass: Q
   L.part = o; o = up256(o + part * 4);
   // double-quantised constants: the fp32 absmax of Wg, Wu and Wd, decoded at each call
   L.am = o;
   if (D->wfmt == LORA_WFMT_4BIT_DQ) o = up256(o + 3 * (f * d / 64) * 4);
+  L.ncnt = dual_shape(D->T, D->d, D->r, 1, kDualMaxGrid).nreg + 2LL * dual_shape(D->T, D->f, D->r, 2, kDualMaxGrid).nreg;
+  L.cnt = o; o = up256(o + static_cast<size_t>(L.ncnt) * 4);
   L.total = o;
   return L;
 }
@@ -561,8 +566,30 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   if (q4) TRY(absmax_for_call(D, W, workspace, WL, st, &am));
 
   float* part = at<float>(workspace, WL.part);
-  // S5a: Qd = s * dY Bd
+  int* cnt = at<int>(workspace, WL.cnt);
+  const bool dual = dual_enabled();
+  // adapter gradients: overwrite semantics -> zero them (and the arrival counters of the
+  // rank-r passes), then accumulate with atomics
   {
+    ZeroList z;
+    z.p[0] = gr->dAg; z.n[0] = static_cast<long long>(r) * d;
+    z.p[1] = gr->dAu; z.n[1] = static_cast<long long>(r) * d;
+    z.p[2] = gr->dBg; z.n[2] = static_cast<long long>(f) * r;
+    z.p[3] = gr->dBu; z.n[3] = static_cast<long long>(f) * r;
+    z.p[4] = gr->dAd; z.n[4] = static_cast<long long>(r) * f;
+    z.p[5] = gr->dBd; z.n[5] = static_cast<long long>(d) * r;
+    z.p[6] = gr->dw;  z.n[6] = gr->dw ? d : 0;
+    z.p[7] = reinterpret_cast<float*>(cnt); z.n[7] = WL.ncnt;  // int zero = float +0 bits
+    PhaseScope ps(st, PH_ZERO);
+    zero_grads_kernel<<<296, 256, 0, st>>>(z);
+    CUDA_TRY(cudaGetLastError());
+  }
+  if (dual) {
+    // S5a + S5c in one read of dY: Qd = s dY Bd, dBd = dY^T Pd
+    const DualProblem pd{dY, d, A->Bd, Pd, rp, gr->dBd};
+    TRY(launch_dual(&pd, 1, T, d, r, s, Qd, rp, part, cnt, status, st, PH_Q_D));
+  } else {
+    // S5a: Qd = s * dY Bd
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], dY, T, d, d, 128));
     TRY(map_mn(&a.maps[1], A->Bd, d, r, r));
@@ -620,8 +647,14 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
     else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
   }
-  // S7a: Q = s * [dG Bg | dU Bu]
-  {
+  if (dual) {
+    // S7a + S7b in one read of dG and dU: Q = s [dG Bg | dU Bu], dBg = dG^T P_g, dBu = dU^T P_u
+    const DualProblem pg[2] = {{dG, f, A->Bg, P, 2 * rp, gr->dBg},
+                               {dU, f, A->Bu, static_cast<const char*>(P) + rp * 2, 2 * rp, gr->dBu}};
+    TRY(launch_dual(pg, 2, T, f, r, s, Q, 2 * rp, part, cnt + dual_shape(T, d, r, 1, kDualMaxGrid).nreg, status, st,
+                    PH_Q_GU));
+  } else {
+    // S7a: Q = s * [dG Bg | dU Bu]
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], dG, T, f, f, 128));
     TRY(map_k(&a.maps[1], dU, T, f, f, 128));
@@ -696,20 +729,6 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // S10: dX = RMSNorm backward (cached rstd)
   TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d, D->residual ? dY : nullptr));
 
-  // adapter gradients: overwrite semantics -> zero, then split-T atomic reductions
-  {
-    ZeroList z;
-    z.p[0] = gr->dAg; z.n[0] = static_cast<long long>(r) * d;
-    z.p[1] = gr->dAu; z.n[1] = static_cast<long long>(r) * d;
-    z.p[2] = gr->dBg; z.n[2] = static_cast<long long>(f) * r;
-    z.p[3] = gr->dBu; z.n[3] = static_cast<long long>(f) * r;
-    z.p[4] = gr->dAd; z.n[4] = static_cast<long long>(r) * f;
-    z.p[5] = gr->dBd; z.n[5] = static_cast<long long>(d) * r;
-    z.p[6] = gr->dw;  z.n[6] = gr->dw ? d : 0;
-    PhaseScope ps(st, PH_ZERO);
-    zero_grads_kernel<<<296, 256, 0, st>>>(z);
-    CUDA_TRY(cudaGetLastError());
-  }
   // norm-weight gradient (trainable-norm variant only): dw_j = sum_t dH_tj x_tj rstd_t
   if (gr->dw) {
     const int rows = static_cast<int>(std::max<long long>(64, (T + 65534) / 65535));
@@ -738,7 +757,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY((launch_gemm<1, 1, 2, EPI_ATOMIC>(a, st, PH_RED_DA_GU)));
   }
   // S7b: dBg = dG^T P_g, dBu = dU^T P_u  ([f x r])
-  {
+  if (!dual) {
     GemmArgs a = new_args(status);
     a.mn3d_a = f % 64 == 0;
     if (a.mn3d_a) {
@@ -760,7 +779,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY((launch_gemm<1, 1, 2, EPI_ATOMIC>(a, st, PH_RED_DB_GU)));
   }
   // S5c: dBd = dY^T Pd  ([d x r])
-  {
+  if (!dual) {
     GemmArgs a = new_args(status);
     a.mn3d_a = d % 64 == 0;
     if (a.mn3d_a) TRY(map_mn3(&a.maps[0], dY, T, d, d, 2));

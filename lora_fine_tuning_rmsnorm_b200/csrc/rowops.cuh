@@ -200,7 +200,7 @@ static __global__ void splitk_finalize_strided_kernel(const float* __restrict__ 
   *reinterpret_cast<uint2*>(out + row * ld_out + col) = o;
 }
 
-constexpr int kZeroMax = 7;
+constexpr int kZeroMax = 8;
 struct ZeroList {
   float* p[kZeroMax];  // NULL entries (n = 0) are skipped
   long long n[kZeroMax];
