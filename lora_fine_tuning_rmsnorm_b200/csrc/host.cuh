@@ -94,17 +94,17 @@ inline int get_encoder() {
   return LORA_OK;
 }
 
-// 2-D bf16 tensor map, 128-byte swizzle: `inner` contiguous elements per row,
+// 2-D bf16 tensor map, 128-byte swizzle (or `swz`): `inner` contiguous elements per row,
 // `outer` rows `ld` elements apart, box of box_inner x box_outer elements.
 inline int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
-             uint32_t box_inner, uint32_t box_outer) {
+             uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   TRY(get_encoder());
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): inner=%llu outer=%llu ld=%llu box=%ux%u",
@@ -438,12 +438,18 @@ inline GemmArgs new_args(int* status) {
 
 // Banded tile order for a dense GEMM: `group_m` row tiles per band (the band's A
 // panels are re-read from L2 by every N tile).  LORA_MLP_RASTER=0 selects the plain
-// M-fastest order instead (tuning comparison).
+// M-fastest order instead, LORA_MLP_BAND=g sets every band to g row tiles (tuning
+// comparisons).
 inline void set_band(GemmArgs& a, int group_m) {
   static const int off = [] {
     const char* e = getenv("LORA_MLP_RASTER");
     return e && e[0] == '0' ? 1 : 0;
   }();
+  static const int forced = [] {
+    const char* e = getenv("LORA_MLP_BAND");
+    return e ? atoi(e) : 0;
+  }();
+  if (forced >= 1) group_m = forced;
   if (off || group_m >= a.tiles_m) return;
   a.raster = 2;
   a.group_m = group_m;
@@ -594,13 +600,26 @@ struct DualShape {
   int qn, R, nrb, nc, nreg, grid, slots;
   long long units;
 };
+// P / B tile geometry for MMA N = qn: row bytes (= the swizzle width), 64-column atoms, swizzle
+inline void dual_tile_geometry(int qn, int* prow, int* patoms, CUtensorMapSwizzle* map_swz, uint32_t* smem_swz) {
+  *prow = qn >= 64 ? 128 : qn * 2;
+  *patoms = qn == 128 ? 2 : 1;
+  *map_swz = *prow == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : (*prow == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+  *smem_swz = *prow == 32 ? kSwz32 : (*prow == 64 ? kSwz64 : kSwz128);
+}
 // Shape of the unit grid on `max_grid` CTAs; slots = the most CTAs that share one
 // (row region, problem), i.e. the partial slots Q needs.
 inline DualShape dual_shape(long long T, int K, int r, int nx, int max_grid) {
   DualShape s{};
   const int rp = round_up(r, 16);
-  s.qn = rp <= 64 ? 64 : 128;
-  s.R = s.qn == 64 ? 4 : 2;  // the Q accumulators (R x qn) and two dB buffers fill 512 TMEM columns
+  // MMA N = the padded rank where a swizzle width fits it exactly (16, 32, 64), else 64 or 128
+  s.qn = rp <= 32 ? rp : (rp <= 64 ? 64 : 128);
+  s.R = 2;  // row blocks per region: the Q accumulators (R x qn) and two dB buffers share TMEM
+  static const int r_knob = [] {
+    const char* e = getenv("LORA_MLP_DUAL_R");  // tuning knob: row blocks per region
+    return e ? atoi(e) : 0;
+  }();
+  if (r_knob >= 1) s.R = std::min(r_knob, 512 / s.qn - 2);
   s.nrb = static_cast<int>((T + 127) / 128);
   s.nc = (K + 127) / 128;
   s.nreg = (s.nrb + s.R - 1) / s.R;
@@ -637,12 +656,24 @@ inline int launch_dual(const DualProblem* pr, int nx, long long T, int K, int r,
   if (s.units <= 0) return LORA_OK;
   if (s.slots > dual_slots_bound(T, K, r, nx))
     return fail(LORA_ERR_UNSUPPORTED, "internal: rank-r pass needs %d partial slots", s.slots);
+  int prow = 0, patoms = 0;
+  CUtensorMapSwizzle map_swz;
+  uint32_t smem_swz = 0;
+  dual_tile_geometry(s.qn, &prow, &patoms, &map_swz, &smem_swz);
   for (int m = 0; m < nx; ++m) {
     TRY(map_k(&a.x[m], pr[m].X, T, K, pr[m].ldx, 128));
-    TRY(map_mn(&a.b[m], pr[m].B, K, r, r));
-    TRY(map_mn(&a.p[m], pr[m].P, T, r, pr[m].ldp));
+    TRY(make_map(&a.b[m], pr[m].B, r, K, r, prow / 2, 128, map_swz));
+    TRY(make_map(&a.p[m], pr[m].P, r, T, pr[m].ldp, prow / 2, 128, map_swz));
     a.dB[m] = pr[m].dB;
   }
+  a.prow = prow;
+  a.patoms = patoms;
+  a.swz = smem_swz;
+  // two accumulators per product when they fit: (R + 2) sets of 2 qn columns
+  a.nsplit = 2 * (s.R + 2) * s.qn <= 512 ? 2 : 1;
+  uint32_t tc = 32;
+  while (tc < static_cast<uint32_t>(a.nsplit * (s.R + 2) * s.qn)) tc <<= 1;
+  a.tmem_cols = tc;
   a.nx = nx;
   a.T = T;
   a.K = K;
@@ -662,10 +693,16 @@ inline int launch_dual(const DualProblem* pr, int nx, long long T, int K, int r,
   a.cnt = cnt;
   a.status = status;
   a.limit_ns = wait_limit_ns();
-  a.stage_bytes = kDualXBytes + static_cast<uint32_t>(s.qn) * 512u;  // X + P + B tiles: the bytes of one stage's copies
-  a.stages = std::min(kDualMaxStages, (kSmemLimit - 1024 - 256) / static_cast<int>(a.stage_bytes));
+  a.stage_bytes = kDualXBytes + 2u * patoms * prow * 128u;  // X + P + B tiles: the bytes of one stage's copies
+  // 4 KB of slack past the barriers: no operand read of the ring's last stage can leave the allocation
+  a.stages = std::min(kDualMaxStages, (kSmemLimit - 1024 - 256 - 4096) / static_cast<int>(a.stage_bytes));
+  static const int stage_cap = [] {
+    const char* e = getenv("LORA_MLP_DUAL_STAGES");  // tuning knob: cap the ring depth
+    return e ? atoi(e) : 0;
+  }();
+  if (stage_cap >= 2) a.stages = std::min(a.stages, stage_cap);
   if (a.stages < 2) return fail(LORA_ERR_UNSUPPORTED, "internal: rank-r stage does not fit");
-  const int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + 256;
+  const int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + 256 + 4096;
   CUDA_TRY(cudaFuncSetAttribute(lowrank_dual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   PhaseScope ps(st, phase);
   lowrank_dual_kernel<<<s.grid, kDualThreads, smem, st>>>(a);

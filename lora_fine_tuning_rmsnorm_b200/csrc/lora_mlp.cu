@@ -468,7 +468,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);  // H is re-read by every N tile: keep it in L2
-    set_band(a, 16 / mt);
+    set_band(a, 8 / mt);
     a.stream_out = 1;
     if (mt == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1, 0, 2>(a, st, PH_GATEUP)));
     else if (pair == 2) TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 2, 1>(a, st, PH_GATEUP)));
@@ -643,7 +643,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
     a.stream_out = 1;
-    set_band(a, 16);
+    set_band(a, 8);
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
     else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
   }
@@ -722,7 +722,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
     a.stream_out = 1;
-    set_band(a, 4);
+    set_band(a, 8);
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_DH)));
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
   }

@@ -20,9 +20,9 @@
 // partial in its slot and the last to arrive (an arrival counter per (region, problem))
 // sums the slots in slot order, so Q does not depend on arrival order.
 //
-// CTA = 6 warps: warp 0 copies X, P and B tiles by TMA into a ring, warp 1 owns TMEM and
-// issues the MMAs from one thread, warps 2..5 drain the accumulators (one TMEM lane
-// quarter each).  Every wait is bounded; the epilogue warps agree on each wait's outcome
+// CTA = 7 warps: warp 0 copies X, P and B tiles by TMA into a ring, warp 1 owns TMEM and
+// issues the Q MMAs from one thread, warp 6 issues the dB MMAs, warps 2..5 drain the
+// accumulators (one TMEM lane quarter each).  Every wait is bounded; the epilogue warps agree on each wait's outcome
 // through a reducing named barrier, so none is left waiting on a warp that gave up.
 #pragma once
 #include "gemm_sm100.cuh"
@@ -30,19 +30,23 @@
 namespace lm {
 
 constexpr int kDualEpiWarps = 4;
-constexpr int kDualThreads = 64 + 32 * kDualEpiWarps;
+constexpr int kDualThreads = 64 + 32 * kDualEpiWarps + 32;  // + the dB MMA warp
 constexpr int kDualMaxGrid = 148;   // CTAs per launch at most (one per SM)
-constexpr int kDualMaxStages = 4;
+constexpr int kDualMaxStages = 6;
 constexpr uint32_t kDualXBytes = 2u * 128u * 128u;  // one [128 rows x 128 columns] bf16 tile of X
 
 struct DualArgs {
   CUtensorMap x[2];  // X of problem m: [T x K], K contiguous, box {64, 128}
-  CUtensorMap b[2];  // B of problem m: [K x r], r contiguous, box {64, 64}
-  CUtensorMap p[2];  // P of problem m: [T x r] (row stride ldp), box {64, 64}
+  CUtensorMap b[2];  // B of problem m: [K x r], r contiguous, box {prow / 2, 128}, prow-byte swizzle
+  CUtensorMap p[2];  // P of problem m: [T x r] (row stride ldp), box {prow / 2, 128}, prow-byte swizzle
   int nx;            // problems (1 or 2)
   long long T;       // rows of X
   int K;             // columns of X
-  int r, rp, qn;     // rank, padded rank (Q columns per problem), MMA N (64 or 128)
+  int r, rp, qn;     // rank, padded rank (Q columns per problem), MMA N (16, 32, 64 or 128)
+  int prow, patoms;  // P / B tiles: bytes per row (32, 64 or 128 = the swizzle width), atoms of 64 columns
+  uint32_t swz;      // their shared-memory swizzle (SmemSwizzle)
+  int nsplit;        // accumulators per product (2: independent MMA chains, summed when drained)
+  uint32_t tmem_cols;
   int R;             // row blocks of 128 per row region
   int nrb, nc, nreg; // row blocks, column groups of 128, row regions
   long long units;   // nreg * nx * nc
@@ -97,12 +101,13 @@ __device__ __forceinline__ DualUnit dual_unit(long long u, int nc, int nx) {
 }
 
 // Shared-memory stage: [X: two 16 KB halves of 64 columns, 128 rows, 128-byte swizzled]
-// [P: qn / 64 chunks of 64 rank columns x 128 rows][B: qn / 64 chunks x 128 K rows].
+// [P: patoms atoms of 128 rows x prow bytes][B: patoms atoms of 128 K rows x prow bytes];
+// the P and B rows are exactly the padded rank wide (N = 16 -> 32-byte rows, 32-byte swizzle).
 static __device__ __noinline__ void dual_producer(const DualArgs& p, uint8_t* tiles, uint32_t full0, uint32_t empty0,
                                                   const WaitCtl& wc, long long u0, long long u1) {
-  const int nstages = p.stages, nc = p.nc, nx = p.nx, R = p.R, nrb = p.nrb, achunks = p.qn / 64;
+  const int nstages = p.stages, nc = p.nc, nx = p.nx, R = p.R, nrb = p.nrb, patoms = p.patoms;
   const uint32_t stage_bytes = p.stage_bytes;
-  const uint32_t pb = static_cast<uint32_t>(p.qn) * 256u;  // bytes of the P (or B) tile
+  const uint32_t atom = static_cast<uint32_t>(p.prow) * 128u;  // one 128-row atom of the P (or B) tile
   int stage = 0;
   uint32_t phase = 0, issued_mask = 0, issued_par = 0;
   bool ok = true;
@@ -121,16 +126,13 @@ static __device__ __noinline__ void dual_producer(const DualArgs& p, uint8_t* ti
       }
       mbar_expect_tx(full, stage_bytes);
       const uint32_t sX = smem_u32(tiles + static_cast<size_t>(stage) * stage_bytes);
-      const uint32_t sP = sX + kDualXBytes, sB = sP + pb;
+      const uint32_t sP = sX + kDualXBytes, sB = sP + patoms * atom;
       const int col = du.c * 128, row = rb * 128;
       tma_load_2d(sX, xm, full, col, row);
       tma_load_2d(sX + 16384, xm, full, col + 64, row);
-      for (int a = 0; a < achunks; ++a) {
-#pragma unroll
-        for (int kh = 0; kh < 2; ++kh) {
-          tma_load_2d(sP + a * 16384 + kh * 8192, pm, full, a * 64, row + kh * 64);
-          tma_load_2d(sB + a * 16384 + kh * 8192, bm, full, a * 64, col + kh * 64);
-        }
+      for (int a = 0; a < patoms; ++a) {
+        tma_load_2d(sP + a * atom, pm, full, a * 64, row);
+        tma_load_2d(sB + a * atom, bm, full, a * 64, col);
       }
       issued_mask |= 1u << stage;
       issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -146,35 +148,49 @@ static __device__ __noinline__ void dual_producer(const DualArgs& p, uint8_t* ti
   }
 }
 
+// MMA issue, split over two threads of different warps that walk the same stages: ROLE 0
+// issues the Q products (and owns the run-level Q hand-off), ROLE 1 the dB products (and
+// the per-unit dB hand-off).  Each commits its MMAs of a stage to the stage's empty
+// barrier, which counts both.  Small-N MMAs cost a roughly fixed issue time each (about
+// 85 cycles at N = 16, measured), so two issuers keep the tensor pipe fed where one could
+// not; four (one per accumulator chain) measured slower than two.
+template <int ROLE>
 static __device__ __noinline__ void dual_mma(const DualArgs& p, uint8_t* tiles, uint32_t full0, uint32_t empty0,
                                              uint32_t dbfull0, uint32_t dbempty0, uint32_t qfull, uint32_t qempty,
                                              uint32_t drain_bar, uint32_t tmem_base, const WaitCtl& wc, long long u0,
                                              long long u1) {
   const int nstages = p.stages, nc = p.nc, nx = p.nx, R = p.R, nrb = p.nrb, qn = p.qn;
-  const uint32_t stage_bytes = p.stage_bytes;
-  const uint32_t pb = static_cast<uint32_t>(qn) * 256u;
+  const uint32_t stage_bytes = p.stage_bytes, swz = p.swz, prow = static_cast<uint32_t>(p.prow);
+  const uint32_t atom = prow * 128u, pbytes = static_cast<uint32_t>(p.patoms) * atom;
+  const uint32_t lbo = p.patoms > 1 ? atom : 0u;  // between 64-column atoms; unused with one atom
   const uint32_t idesc_q = idesc_bf16(128, qn, 0, 1);  // A = X (K-major), B = B (MN-major)
   const uint32_t idesc_b = idesc_bf16(128, qn, 1, 1);  // A = X^T (MN-major), B = P (MN-major)
   const uint32_t tiles_u32 = smem_u32(tiles);
+  // TMEM: Q accumulators (rl, s) at (rl * nsplit + s) * qn, dB accumulators (buf, s) after them
+  const int nsplit = p.nsplit;
+  const uint32_t q_cols = static_cast<uint32_t>(R * nsplit * qn);
+  const uint32_t second = nsplit == 1 ? 1u : 0u;  // a second chain continues the first's sum
+  constexpr int kKind = ROLE;
   int stage = 0;
   uint32_t phase = 0, it = 0, qrun = 0, started = 0;
   bool ok = true, issued_any = false;
   for (long long u = u0; u < u1 && ok; ++u, ++it) {
     const DualUnit du = dual_unit(u, nc, nx);
-    if (u == u0 || du.c == 0) {  // a new run of (region, problem): the Q accumulators are free again
+    const uint32_t buf = it & 1;
+    if (kKind == 0 && (u == u0 || du.c == 0)) {  // a new run of (region, problem): Q accumulators free again
       if (!mbar_wait(qempty, (qrun & 1) ^ 1, wc, kDevTimeoutMma)) {
         ok = false;
         break;
       }
       started = 0;
     }
-    const uint32_t buf = it & 1;
-    if (!mbar_wait(dbempty0 + 8 * buf, ((it >> 1) & 1) ^ 1, wc, kDevTimeoutMma)) {
+    if (kKind == 1 && !mbar_wait(dbempty0 + 8 * buf, ((it >> 1) & 1) ^ 1, wc, kDevTimeoutMma)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    const uint32_t db = tmem_base + static_cast<uint32_t>(R * qn) + buf * qn;
+    const uint32_t db0 = tmem_base + q_cols + buf * nsplit * qn;
+    const uint32_t db1 = db0 + (nsplit - 1) * qn;
     for (int rl = 0; rl < R; ++rl) {
       const int rb = du.reg * R + rl;
       if (rb >= nrb) break;
@@ -184,37 +200,41 @@ static __device__ __noinline__ void dual_mma(const DualArgs& p, uint8_t* tiles, 
       }
       tc_fence_after();
       const uint32_t sX = tiles_u32 + static_cast<uint32_t>(stage) * stage_bytes;
-      const uint32_t sP = sX + kDualXBytes, sB = sP + pb;
-      // Q[rows of block rl] += X_tile B_tile: K = the tile's 128 columns, two halves of 64
-      const uint32_t dq = tmem_base + static_cast<uint32_t>(rl * qn);
-      const uint32_t acc_q = (started >> rl) & 1;
+      const uint32_t sP = sX + kDualXBytes, sB = sP + pbytes;
+      if (kKind == 0) {
+        // Q[rows of block rl] += X_tile B_tile: K = the tile's 128 columns in two halves of 64
+        // (B is MN-major: rows = K, a k-step of 16 rows is 16 * prow bytes), one chain per half
+        const uint32_t dq0 = tmem_base + static_cast<uint32_t>(rl * nsplit * qn);
+        const uint32_t dq1 = dq0 + (nsplit - 1) * qn;
+        const uint32_t st_q = (started >> rl) & 1;
+        const uint64_t qa0 = sdesc_sw128(sX, 16, 1024), qa1 = sdesc_sw128(sX + 16384, 16, 1024);
+        const uint64_t qb0 = sdesc(sB, lbo, 8 * prow, swz), qb1 = sdesc(sB + 64 * prow, lbo, 8 * prow, swz);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint64_t a0 = sdesc_sw128(sX + h * 16384, 16, 1024);
-        const uint64_t b0 = sdesc_sw128(sB + h * 8192, 16384, 1024);
+        for (int j = 0; j < 4; ++j) {
+          mma_bf16(dq0, qa0 + j * (32 >> 4), qb0 + j * prow, idesc_q, j ? 1u : st_q);
+          mma_bf16(dq1, qa1 + j * (32 >> 4), qb1 + j * prow, idesc_q, j ? 1u : (st_q | second));
+        }
+        started |= 1u << rl;
+      } else {
+        // dB[columns of the group] += X_tile^T P_tile: K = the tile's 128 rows, one chain per half
+        const uint64_t ba = sdesc_sw128(sX, 16384, 1024);
+        const uint64_t bb = sdesc(sP, lbo, 8 * prow, swz);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_bf16(dq, a0 + j * (32 >> 4), b0 + j * (2048 >> 4), idesc_q, (h | j) ? 1u : acc_q);
-      }
-      started |= 1u << rl;
-      // dB[columns of the group] += X_tile^T P_tile: K = the tile's 128 rows
-      {
-        const uint64_t a0 = sdesc_sw128(sX, 16384, 1024);
-        const uint64_t b0 = sdesc_sw128(sP, 16384, 1024);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          mma_bf16(db, a0 + j * (2048 >> 4), b0 + j * (2048 >> 4), idesc_b, (rl | j) ? 1u : 0u);
+        for (int j = 0; j < 4; ++j) {
+          mma_bf16(db0, ba + j * (2048 >> 4), bb + j * prow, idesc_b, (rl | j) ? 1u : 0u);
+          mma_bf16(db1, ba + (j + 4) * (2048 >> 4), bb + (j + 4) * prow, idesc_b, (rl | j) ? 1u : second);
+        }
       }
       issued_any = true;
-      mma_commit(empty0 + 8 * stage);  // frees the stage once these MMAs finish
+      mma_commit(empty0 + 8 * stage);  // frees the stage once both issuers' MMAs finish
       if (++stage == nstages) {
         stage = 0;
         phase ^= 1;
       }
     }
     if (!ok) break;
-    mma_commit(dbfull0 + 8 * buf);
-    if (u + 1 == u1 || (u + 1) % nc == 0) {  // the run ends: Q accumulators ready
+    if (kKind == 1) mma_commit(dbfull0 + 8 * buf);
+    if (kKind == 0 && (u + 1 == u1 || (u + 1) % nc == 0)) {  // the run ends: Q accumulators ready
       mma_commit(qfull);
       ++qrun;
     }
@@ -233,6 +253,7 @@ static __device__ __noinline__ void dual_epilogue(const DualArgs& p, uint32_t db
   const int q = warp & 3;  // TMEM lane quarter
   const int etid = threadIdx.x - 64;
   const int nc = p.nc, nx = p.nx, R = p.R, nrb = p.nrb, qn = p.qn, r = p.r, rp = p.rp, K = p.K, ldq = p.ldq;
+  const int nsplit = p.nsplit;
   const long long T = p.T, part_slot = p.part_slot;
   const float scale = p.scale;
   uint16_t* const Q = p.Q;
@@ -251,12 +272,19 @@ static __device__ __noinline__ void dual_epilogue(const DualArgs& p, uint32_t db
     {
       float* const dB = p.dB[du.m];
       const long long kk = static_cast<long long>(du.c) * 128 + 32 * q + lane;
-      const uint32_t t0 = lane_base + static_cast<uint32_t>(R * qn) + buf * qn;
+      const uint32_t t0 = lane_base + static_cast<uint32_t>(R * nsplit * qn) + buf * nsplit * qn;
 #pragma unroll 1
       for (int c0 = 0; c0 < r; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(t0 + c0, v);
         tmem_wait16(v);
+        if (nsplit == 2) {  // the second accumulator (rows 64-127 of each tile)
+          uint32_t w[16];
+          tmem_ld16(t0 + qn + c0, w);
+          tmem_wait16(w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+        }
         if (kk < K) {
           float* o = dB + kk * r + c0;
 #pragma unroll
@@ -292,8 +320,15 @@ static __device__ __noinline__ void dual_epilogue(const DualArgs& p, uint32_t db
 #pragma unroll 1
       for (int c0 = 0; c0 < rp; c0 += 16) {
         uint32_t v[16];
-        tmem_ld16(lane_base + static_cast<uint32_t>(rl * qn + c0), v);
+        tmem_ld16(lane_base + static_cast<uint32_t>(rl * nsplit * qn + c0), v);
         tmem_wait16(v);
+        if (nsplit == 2) {  // the second accumulator (columns 64-127 of each tile)
+          uint32_t w[16];
+          tmem_ld16(lane_base + static_cast<uint32_t>((rl * nsplit + 1) * qn + c0), w);
+          tmem_wait16(w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+        }
         if (t >= T) continue;
         if (n == 1) {  // the whole row of column groups was this CTA's: Q directly
           uint32_t w[8];
@@ -353,8 +388,8 @@ static __global__ void __launch_bounds__(kDualThreads, 1) lowrank_dual_kernel(co
   const uint32_t dbempty0 = dbfull0 + 16;
   const uint32_t qfull = dbempty0 + 16;
   const uint32_t qempty = qfull + 8;
-  const uint32_t drain_bar = qempty + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 7);
+  const uint32_t drain_bar = qempty + 8;  // one per MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -364,7 +399,7 @@ static __global__ void __launch_bounds__(kDualThreads, 1) lowrank_dual_kernel(co
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 2);  // both MMA issuers commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(dbfull0 + 8 * b, 1);
@@ -372,7 +407,7 @@ static __global__ void __launch_bounds__(kDualThreads, 1) lowrank_dual_kernel(co
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, kDualEpiWarps);
-    mbar_init(drain_bar, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(drain_bar + 8 * i, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -384,7 +419,7 @@ static __global__ void __launch_bounds__(kDualThreads, 1) lowrank_dual_kernel(co
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -397,16 +432,21 @@ static __global__ void __launch_bounds__(kDualThreads, 1) lowrank_dual_kernel(co
     if (lane == 0) dual_producer(p, tiles, full0, empty0, wc, u0, u1);
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) dual_mma(p, tiles, full0, empty0, dbfull0, dbempty0, qfull, qempty, drain_bar, tmem_base, wc, u0, u1);
+    if (lane == 0)
+      dual_mma<0>(p, tiles, full0, empty0, dbfull0, dbempty0, qfull, qempty, drain_bar, tmem_base, wc, u0, u1);
     __syncwarp();
-  } else {
+  } else if (warp < 2 + kDualEpiWarps) {
     dual_epilogue(p, dbfull0, dbempty0, qfull, qempty, tmem_base, s_last, wc, u0, u1, U, G);
+  } else {
+    if (lane == 0)
+      dual_mma<1>(p, tiles, full0, empty0, dbfull0, dbempty0, qfull, qempty, drain_bar + 8, tmem_base, wc, u0, u1);
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 

@@ -308,15 +308,24 @@ __device__ __forceinline__ void tmem_wait32(uint32_t (&a)[16], uint32_t (&b)[16]
 // Shared-memory matrix descriptor (sm_100 format): start address >> 4 in bits
 // [0,14), leading-dimension byte offset >> 4 in [16,30), stride-dimension byte
 // offset >> 4 in [32,46), descriptor version 1 in [46,48), base offset 0, swizzle
-// mode in [61,64) (2 = 128-byte swizzle).  Tiles are 1024-byte aligned.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// mode in [61,64): 2 = 128-byte, 4 = 64-byte, 6 = 32-byte swizzle.  A swizzled tile
+// starts on a multiple of its swizzle atom (8 rows of the swizzle width: 1024, 512 or
+// 256 bytes).  For an MN-major operand the rows are K rows of the swizzle width, the
+// leading offset steps between atoms along M/N and the stride offset between groups
+// of 8 K rows; for a K-major operand (128-byte rows of K) the stride offset steps
+// between groups of 8 M/N rows.
+enum SmemSwizzle : uint32_t { kSwz128 = 2, kSwz64 = 4, kSwz32 = 6 };
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t swz) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
   d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
   d |= 1ull << 46;
-  d |= 2ull << 61;
+  d |= static_cast<uint64_t>(swz) << 61;
   return d;
+}
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc(saddr, lbo, sbo, kSwz128);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation:
