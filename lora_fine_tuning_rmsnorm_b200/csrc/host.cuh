@@ -62,15 +62,20 @@ inline bool debug_mode() {
   return v != 0;
 }
 
-// LORA_MLP_DUAL=0 selects the two-pass form of the rank-r gradients (a projection GEMM
-// for Q and a reduction GEMM for dB, each reading the activation gradient) instead of
-// the single-pass kernel; both compute the same quantities.  Read once per process.
-inline bool dual_enabled() {
+// Which rank-r products run in the single-pass streaming kernel (lowrank_dual.cuh) rather
+// than as split-K / split-T GEMMs; both forms compute the same quantities.  LORA_MLP_DUAL:
+//   1 (default): the fused backward passes (Q with dB from one read of dY, of dG / dU) and
+//                the reduction over the wide activation (dAd), where it measured faster;
+//   2: every rank-r product (also P, Pd, dAg / dAu, which measured a few us slower);
+//   0: none (two passes over each activation gradient).
+// Read once per process.
+inline int dual_mode() {
   static int v = [] {
     const char* e = getenv("LORA_MLP_DUAL");
-    return (e && e[0] == '0') ? 0 : 1;
+    if (!e || !e[0]) return 1;
+    return e[0] == '0' ? 0 : (e[0] == '2' ? 2 : 1);
   }();
-  return v != 0;
+  return v;
 }
 
 inline unsigned long long wait_limit_ns() {
@@ -585,101 +590,176 @@ int launch_proj_into(GemmArgs& a, long long T, long long K, int rp, float* part,
 }
 
 
-// ------------------------------------------------- rank-r gradient pass (dual)
-// One problem of lowrank_dual_kernel: X [T x K] (row stride ldx), B [K x r] (row stride
-// r), P [T x r] (row stride ldp), dB [K x r] fp32 (accumulated).
+// ------------------------------------------ rank-r streaming products (lowrank_dual.cuh)
+// One problem: X [T x K] (row stride ldx); the row product's skinny operand S (MN-major
+// [K x r] with row stride r in S[0], or K-major [r x K] rows, row stride K, in S[0] and
+// S[1]); the column product's operand P [T x p_cols] (row stride ldp); its outputs.
 struct DualProblem {
   const void* X;
   long long ldx;
-  const void* B;
+  const void* S[2];
   const void* P;
   long long ldp;
-  float* dB;
+  int p_cols;
+  float* out[2];
 };
+// Which products a launch computes and how their operands and outputs are laid out.
+struct DualSpec {
+  int do_row, do_col;
+  int row_kmajor, nbk;  // K-major row operand from nbk [r x K] matrices (else MN-major [K x r])
+  int col_trans;        // column product written as [r x K] matrices (else [K x r] per problem)
+  int n;                // MMA N: 16 or 32, or a multiple of 64 (MN-major tiles); K-major rows: nbk * rp
+  int qw;               // row-product columns written per problem
+};
+// Q = s [X_m B_m] and dB_m += X_m^T P_m together (the backward of an up-projection)
+inline DualSpec dual_spec_both(int r) {
+  const int rp = round_up(r, 16);
+  const int n = rp <= 32 ? rp : round_up(rp, 64);
+  return DualSpec{1, 1, 0, 1, 0, n, rp};
+}
+// P = s X [A_0; A_1]^T (the forward rank-r projection of nbk adapters sharing X)
+inline DualSpec dual_spec_proj(int r, int nbk) {
+  const int rp = round_up(r, 16);
+  return DualSpec{1, 0, 1, nbk, 0, nbk * rp, nbk * rp};
+}
+// dA_i += (Q[:, i rp : i rp + r])^T X for the nq column blocks of Q (the reductions over T)
+inline DualSpec dual_spec_reduce(int r, int nq) {
+  const int rp = round_up(r, 16);
+  const int w = nq * rp;
+  const int n = w <= 32 ? w : round_up(w, 64);
+  return DualSpec{0, 1, 0, 1, 1, n, 0};
+}
 struct DualShape {
-  int qn, R, nrb, nc, nreg, grid, slots;
+  int R, nrb, nc, nreg, grid, slots;
   long long units;
 };
-// P / B tile geometry for MMA N = qn: row bytes (= the swizzle width), 64-column atoms, swizzle
-inline void dual_tile_geometry(int qn, int* prow, int* patoms, CUtensorMapSwizzle* map_swz, uint32_t* smem_swz) {
-  *prow = qn >= 64 ? 128 : qn * 2;
-  *patoms = qn == 128 ? 2 : 1;
+// MN-major skinny tile geometry for MMA N = n: row bytes (= the swizzle width), atoms of 64
+// columns, swizzle
+inline void dual_tile_geometry(int n, int* prow, int* patoms, CUtensorMapSwizzle* map_swz, uint32_t* smem_swz) {
+  *prow = n >= 64 ? 128 : n * 2;
+  *patoms = n >= 64 ? n / 64 : 1;
   *map_swz = *prow == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : (*prow == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
   *smem_swz = *prow == 32 ? kSwz32 : (*prow == 64 ? kSwz64 : kSwz128);
 }
-// Shape of the unit grid on `max_grid` CTAs; slots = the most CTAs that share one
-// (row region, problem), i.e. the partial slots Q needs.
-inline DualShape dual_shape(long long T, int K, int r, int nx, int max_grid) {
-  DualShape s{};
-  const int rp = round_up(r, 16);
-  // MMA N = the padded rank where a swizzle width fits it exactly (16, 32, 64), else 64 or 128
-  s.qn = rp <= 32 ? rp : (rp <= 64 ? 64 : 128);
-  s.R = 2;  // row blocks per region: the Q accumulators (R x qn) and two dB buffers share TMEM
+// Row blocks per region: 2 while a row product keeps R accumulators in TMEM; a column
+// product alone takes the largest of 16, 8, 4, 2 that still leaves two units per CTA of a
+// full grid (each region adds one fp32 atomic per output element).
+inline int dual_rows(const DualSpec& sp, long long T, int K, int nx) {
   static const int r_knob = [] {
     const char* e = getenv("LORA_MLP_DUAL_R");  // tuning knob: row blocks per region
     return e ? atoi(e) : 0;
   }();
-  if (r_knob >= 1) s.R = std::min(r_knob, 512 / s.qn - 2);
+  const long long nrb = (T + 127) / 128, nc = (K + 127) / 128;
+  int R = 2;
+  if (!sp.do_row) {
+    for (R = 16; R > 2; R /= 2)
+      if ((nrb + R - 1) / R * nx * nc >= 2LL * kDualMaxGrid) break;
+  }
+  if (r_knob >= 1) R = std::max(1, std::min(r_knob, sp.do_row ? 512 / sp.n - 2 : 64));
+  return R;
+}
+// Shape of the unit grid on `max_grid` CTAs; slots = the most CTAs that share one
+// (row region, problem), i.e. the partial slots the row product needs.
+inline DualShape dual_shape(const DualSpec& sp, long long T, int K, int nx, int max_grid) {
+  DualShape s{};
+  s.R = dual_rows(sp, T, K, nx);
   s.nrb = static_cast<int>((T + 127) / 128);
   s.nc = (K + 127) / 128;
   s.nreg = (s.nrb + s.R - 1) / s.R;
   s.units = static_cast<long long>(s.nreg) * nx * s.nc;
   s.grid = static_cast<int>(std::min<long long>(s.units, max_grid));
   s.slots = 1;
-  for (long long k = 0; k < static_cast<long long>(s.nreg) * nx; ++k) {
-    const long long a = dual_owner(k * s.nc, s.units, s.grid);
-    const long long b = dual_owner(k * s.nc + s.nc - 1, s.units, s.grid);
-    s.slots = std::max(s.slots, static_cast<int>(b - a + 1));
+  if (sp.do_row) {
+    for (long long k = 0; k < static_cast<long long>(s.nreg) * nx; ++k) {
+      const long long a = dual_owner(k * s.nc, s.units, s.grid);
+      const long long b = dual_owner(k * s.nc + s.nc - 1, s.units, s.grid);
+      s.slots = std::max(s.slots, static_cast<int>(b - a + 1));
+    }
   }
   return s;
 }
 // Partial slots to reserve whatever the device's SM count: ranges hold at least
 // floor(U / G) units, so a run of nc units meets at most 1 + ceil((nc - 1) / floor(U / G))
 // of them, largest at the largest grid.
-inline int dual_slots_bound(long long T, int K, int r, int nx) {
-  const DualShape s = dual_shape(T, K, r, nx, kDualMaxGrid);
+inline int dual_slots_bound(const DualSpec& sp, long long T, int K, int nx) {
+  if (!sp.do_row) return 0;
+  const DualShape s = dual_shape(sp, T, K, nx, kDualMaxGrid);
   const long long L = std::max<long long>(1, s.units / s.grid);
   return static_cast<int>(1 + (s.nc - 1 + L - 1) / L);
 }
+// Arrival counters a launch uses (zero on entry, left zero).
+inline long long dual_counters(const DualSpec& sp, long long T, int K, int nx) {
+  return sp.do_row ? static_cast<long long>(dual_shape(sp, T, K, nx, kDualMaxGrid).nreg) * nx : 0;
+}
 
-// Q[:, m rp : (m + 1) rp] = scale * X_m B_m and dB_m += X_m^T P_m for the nx problems
-// (Q bf16, row stride ldq).  `part` holds dual_slots_bound(...) * T * ldq floats; `cnt`
-// holds dual_shape(...).nreg * nx ints that are zero on entry (and left zero).
-inline int launch_dual(const DualProblem* pr, int nx, long long T, int K, int r, float scale, void* Q, int ldq,
-                       float* part, int* cnt, int* status, cudaStream_t st, int phase) {
-  if (nx < 1 || nx > 2 || K < 8 || K % 8 || r < 8 || r % 8 || r > 128)
-    return fail(LORA_ERR_UNSUPPORTED, "internal: bad rank-r pass (nx %d, K %d, r %d)", nx, K, r);
+// Runs the products of `sp` over the nx problems.  The row product goes to Q (bf16, row
+// stride ldq; problem m writes columns [m qw, (m + 1) qw), scaled by `scale`); `part` holds
+// dual_slots_bound(...) * T * ldq floats and `cnt` dual_counters(...) zeroed ints.  The
+// column product is added (fp32 atomics) into outputs the caller has zeroed.
+inline int launch_dual(const DualSpec& sp, const DualProblem* pr, int nx, long long T, int K, int r, float scale,
+                       void* Q, int ldq, float* part, int* cnt, int* status, cudaStream_t st, int phase) {
+  const int rp = round_up(r, 16);
+  if (nx < 1 || nx > 2 || K < 8 || K % 8 || r < 8 || r % 8 || r > 128 || sp.n < 16 || sp.n > 256 || sp.n % 16 ||
+      (sp.n > 32 && sp.n % 64 && (sp.do_col || !sp.row_kmajor)) || (sp.row_kmajor && sp.n != sp.nbk * rp) ||
+      (sp.col_trans && nx != 1) || (sp.do_row && (sp.qw % 16 || sp.qw > sp.n || nx * sp.qw > ldq)))
+    return fail(LORA_ERR_UNSUPPORTED, "internal: bad rank-r pass (nx %d, K %d, r %d, n %d)", nx, K, r, sp.n);
   DualArgs a;
   memset(&a, 0, sizeof(a));
-  const int rp = round_up(r, 16);
-  const DualShape s = dual_shape(T, K, r, nx, std::min(sm_count(), kDualMaxGrid));
+  const DualShape s = dual_shape(sp, T, K, nx, std::min(sm_count(), kDualMaxGrid));
   if (s.units <= 0) return LORA_OK;
-  if (s.slots > dual_slots_bound(T, K, r, nx))
+  if (sp.do_row && s.slots > dual_slots_bound(sp, T, K, nx))
     return fail(LORA_ERR_UNSUPPORTED, "internal: rank-r pass needs %d partial slots", s.slots);
   int prow = 0, patoms = 0;
   CUtensorMapSwizzle map_swz;
   uint32_t smem_swz = 0;
-  dual_tile_geometry(s.qn, &prow, &patoms, &map_swz, &smem_swz);
+  dual_tile_geometry(sp.n, &prow, &patoms, &map_swz, &smem_swz);
   for (int m = 0; m < nx; ++m) {
     TRY(map_k(&a.x[m], pr[m].X, T, K, pr[m].ldx, 128));
-    TRY(make_map(&a.b[m], pr[m].B, r, K, r, prow / 2, 128, map_swz));
-    TRY(make_map(&a.p[m], pr[m].P, r, T, pr[m].ldp, prow / 2, 128, map_swz));
-    a.dB[m] = pr[m].dB;
+    if (sp.do_row) {
+      if (sp.row_kmajor) {
+        for (int i = 0; i < sp.nbk; ++i) TRY(map_k(&a.b[m][i], pr[m].S[i], r, K, K, static_cast<uint32_t>(rp)));
+      } else {
+        TRY(make_map(&a.b[m][0], pr[m].S[0], r, K, r, prow / 2, 128, map_swz));
+      }
+    }
+    if (sp.do_col) TRY(make_map(&a.p[m], pr[m].P, pr[m].p_cols, T, pr[m].ldp, prow / 2, 128, map_swz));
+    a.out[m] = pr[m].out[0];
   }
-  a.prow = prow;
-  a.patoms = patoms;
-  a.swz = smem_swz;
-  // two accumulators per product when they fit: (R + 2) sets of 2 qn columns
-  a.nsplit = 2 * (s.R + 2) * s.qn <= 512 ? 2 : 1;
-  uint32_t tc = 32;
-  while (tc < static_cast<uint32_t>(a.nsplit * (s.R + 2) * s.qn)) tc <<= 1;
-  a.tmem_cols = tc;
+  if (sp.col_trans) {
+    a.out[0] = pr[0].out[0];
+    a.out[1] = pr[0].out[1];
+  }
   a.nx = nx;
   a.T = T;
   a.K = K;
   a.r = r;
   a.rp = rp;
-  a.qn = s.qn;
+  a.n = sp.n;
+  a.do_row = sp.do_row;
+  a.do_col = sp.do_col;
+  a.row_kmajor = sp.row_kmajor;
+  a.nbk = sp.nbk;
+  a.qw = sp.qw;
+  a.col_trans = sp.col_trans;
+  a.prow = prow;
+  a.patoms = patoms;
+  a.swz = smem_swz;
+  // TMEM's 512 columns: two row sets (so a run's flush overlaps the next run) and two
+  // accumulators per product (independent MMA chains) where they fit, in that order
+  int sets = 0;
+  a.nsplit = 0;
+  for (int cfg = 0; cfg < 4 && !a.nsplit; ++cfg) {
+    const int rsets = cfg < 2 ? 2 : 1, nsplit = (cfg & 1) ? 1 : 2;
+    sets = (sp.do_row ? rsets * s.R : 0) + (sp.do_col ? 2 : 0);
+    if (nsplit * sets * sp.n <= 512) {
+      a.nsplit = nsplit;
+      a.rsets = rsets;
+    }
+  }
+  if (!a.nsplit) return fail(LORA_ERR_UNSUPPORTED, "internal: rank-r accumulators exceed TMEM");
+  uint32_t tc = 32;
+  while (tc < static_cast<uint32_t>(a.nsplit * sets * sp.n)) tc <<= 1;
+  a.tmem_cols = tc;
   a.R = s.R;
   a.nrb = s.nrb;
   a.nc = s.nc;
@@ -693,7 +773,10 @@ inline int launch_dual(const DualProblem* pr, int nx, long long T, int K, int r,
   a.cnt = cnt;
   a.status = status;
   a.limit_ns = wait_limit_ns();
-  a.stage_bytes = kDualXBytes + 2u * patoms * prow * 128u;  // X + P + B tiles: the bytes of one stage's copies
+  const uint32_t tile = 256u * static_cast<uint32_t>(sp.n);  // one skinny tile: 128 K rows (or 2 x 64 K) x n
+  a.col_off = kDualXBytes;
+  a.row_off = kDualXBytes + (sp.do_col ? tile : 0u);
+  a.stage_bytes = a.row_off + (sp.do_row ? tile : 0u);  // the bytes of one stage's copies
   // 4 KB of slack past the barriers: no operand read of the ring's last stage can leave the allocation
   a.stages = std::min(kDualMaxStages, (kSmemLimit - 1024 - 256 - 4096) / static_cast<int>(a.stage_bytes));
   static const int stage_cap = [] {

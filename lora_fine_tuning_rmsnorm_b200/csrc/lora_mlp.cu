@@ -13,7 +13,7 @@ namespace {
 // --------------------------------------------------------------- layouts
 struct WsLayout {
   size_t status, Q, Qd, dG, dU, dH, part, am, cnt, total;
-  long long ncnt;  // arrival counters of the rank-r gradient passes (down, then gate/up)
+  long long ncnt;  // arrival counters of the rank-r streaming launches (DualLaunch order)
 };
 
 int check_dims(const lora_mlp_dims* D) {
@@ -52,6 +52,33 @@ lora_mlp_ctx_layout ctx_layout(const lora_mlp_dims* D) {
   return L;
 }
 
+// The rank-r streaming launches of one forward + backward (lowrank_dual.cuh), in the
+// order of their arrival counters in the workspace.
+enum DualLaunch { DL_P_GU = 0, DL_P_D, DL_BWD_D, DL_BWD_GU, DL_RED_GU, DL_RED_D, DL_COUNT };
+struct DualPlan {
+  DualSpec sp;
+  int K, nx, ldq;
+};
+DualPlan dual_plan(const lora_mlp_dims* D, int which) {
+  const int r = D->r, rp = rp_of(D);
+  switch (which) {
+    case DL_P_GU: return DualPlan{dual_spec_proj(r, 2), D->d, 1, 2 * rp};    // P  = s H [Ag; Au]^T
+    case DL_P_D: return DualPlan{dual_spec_proj(r, 1), D->f, 1, rp};         // Pd = s Act Ad^T
+    case DL_BWD_D: return DualPlan{dual_spec_both(r), D->d, 1, rp};          // Qd = s dY Bd, dBd
+    case DL_BWD_GU: return DualPlan{dual_spec_both(r), D->f, 2, 2 * rp};     // Q = s [dG Bg | dU Bu], dBg, dBu
+    case DL_RED_GU: return DualPlan{dual_spec_reduce(r, 2), D->d, 1, 0};     // dAg, dAu
+    default: return DualPlan{dual_spec_reduce(r, 1), D->f, 1, 0};            // dAd
+  }
+}
+long long dual_cnt_offset(const lora_mlp_dims* D, int which) {
+  long long o = 0;
+  for (int i = 0; i < which; ++i) {
+    const DualPlan pl = dual_plan(D, i);
+    o += dual_counters(pl.sp, D->T, pl.K, pl.nx);
+  }
+  return o;
+}
+
 WsLayout ws_layout(const lora_mlp_dims* D) {
   const size_t T = D->T, d = D->d, f = D->f, rp = rp_of(D);
   WsLayout L{};
@@ -67,13 +94,15 @@ WsLayout ws_layout(const lora_mlp_dims* D) {
   part = std::max(part, size_t(proj_splits(T, f)) * T * rp);       // Pd = s Act Ad^T
   part = std::max(part, size_t(proj_splits(T, d)) * T * rp);       // Qd = s dY Bd
   part = std::max(part, size_t(proj_splits(T, f)) * T * 2 * rp);   // Q  = s [dG Bg | dU Bu]
-  part = std::max(part, size_t(dual_slots_bound(T, D->d, D->r, 1)) * T * rp);      // single pass: Qd
-  part = std::max(part, size_t(dual_slots_bound(T, D->f, D->r, 2)) * T * 2 * rp);  // single pass: Q
+  for (int i = 0; i < DL_COUNT; ++i) {  // the single-pass kernels' partial slots
+    const DualPlan pl = dual_plan(D, i);
+    part = std::max(part, size_t(dual_slots_bound(pl.sp, D->T, pl.K, pl.nx)) * T * pl.ldq);
+  }
   L.part = o; o = up256(o + part * 4);
   // double-quantised constants: the fp32 absmax of Wg, Wu and Wd, decoded at each call
   L.am = o;
   if (D->wfmt == LORA_WFMT_4BIT_DQ) o = up256(o + 3 * (f * d / 64) * 4);
-  L.ncnt = dual_shape(D->T, D->d, D->r, 1, kDualMaxGrid).nreg + 2LL * dual_shape(D->T, D->f, D->r, 2, kDualMaxGrid).nreg;
+  L.ncnt = dual_cnt_offset(D, DL_COUNT);
   L.cnt = o; o = up256(o + static_cast<size_t>(L.ncnt) * 4);
   L.total = o;
   return L;
@@ -413,7 +442,16 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
 
   // S2: P = s * [H Ag^T | H Au^T]  (rank-r projections, padded to rp columns each)
   float* part = at<float>(workspace, WL.part);
-  {
+  int* cnt = at<int>(workspace, WL.cnt);
+  const int dmode = dual_mode();
+  if (dmode == 2) {
+    CUDA_TRY(cudaMemsetAsync(cnt, 0, static_cast<size_t>(WL.ncnt) * sizeof(int), st));
+    const DualPlan pl = dual_plan(D, DL_P_GU);
+    DualProblem pr{};
+    pr.X = H; pr.ldx = d; pr.S[0] = A->Ag; pr.S[1] = A->Au;
+    TRY(launch_dual(pl.sp, &pr, 1, T, d, r, s, P, 2 * rp, part, cnt + dual_cnt_offset(D, DL_P_GU), status, st,
+                    PH_P_GU));
+  } else {
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], H, T, d, d, 128));
     TRY(map_k(&a.maps[1], A->Ag, r, d, d, rp));
@@ -475,7 +513,12 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     else TRY((launch_gemm<0, 0, 2, EPI_SWIGLU_FWD, 1, 1>(a, st, PH_GATEUP)));
   }
   // S4a: Pd = s * Act Ad^T
-  {
+  if (dmode == 2) {
+    const DualPlan pl = dual_plan(D, DL_P_D);
+    DualProblem pr{};
+    pr.X = Act; pr.ldx = f; pr.S[0] = A->Ad;
+    TRY(launch_dual(pl.sp, &pr, 1, T, f, r, s, Pd, rp, part, cnt + dual_cnt_offset(D, DL_P_D), status, st, PH_P_D));
+  } else {
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], Act, T, f, f, 128));
     TRY(map_k(&a.maps[1], A->Ad, r, f, f, rp));
@@ -567,7 +610,8 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
 
   float* part = at<float>(workspace, WL.part);
   int* cnt = at<int>(workspace, WL.cnt);
-  const bool dual = dual_enabled();
+  const int dmode = dual_mode();
+  const bool dual = dmode >= 1;
   // adapter gradients: overwrite semantics -> zero them (and the arrival counters of the
   // rank-r passes), then accumulate with atomics
   {
@@ -586,8 +630,10 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   }
   if (dual) {
     // S5a + S5c in one read of dY: Qd = s dY Bd, dBd = dY^T Pd
-    const DualProblem pd{dY, d, A->Bd, Pd, rp, gr->dBd};
-    TRY(launch_dual(&pd, 1, T, d, r, s, Qd, rp, part, cnt, status, st, PH_Q_D));
+    DualProblem pr{};
+    pr.X = dY; pr.ldx = d; pr.S[0] = A->Bd; pr.P = Pd; pr.ldp = rp; pr.p_cols = r; pr.out[0] = gr->dBd;
+    TRY(launch_dual(dual_plan(D, DL_BWD_D).sp, &pr, 1, T, d, r, s, Qd, rp, part, cnt + dual_cnt_offset(D, DL_BWD_D),
+                    status, st, PH_Q_D));
   } else {
     // S5a: Qd = s * dY Bd
     GemmArgs a = new_args(status);
@@ -649,10 +695,13 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   }
   if (dual) {
     // S7a + S7b in one read of dG and dU: Q = s [dG Bg | dU Bu], dBg = dG^T P_g, dBu = dU^T P_u
-    const DualProblem pg[2] = {{dG, f, A->Bg, P, 2 * rp, gr->dBg},
-                               {dU, f, A->Bu, static_cast<const char*>(P) + rp * 2, 2 * rp, gr->dBu}};
-    TRY(launch_dual(pg, 2, T, f, r, s, Q, 2 * rp, part, cnt + dual_shape(T, d, r, 1, kDualMaxGrid).nreg, status, st,
-                    PH_Q_GU));
+    DualProblem pg[2] = {};
+    pg[0].X = dG; pg[0].ldx = f; pg[0].S[0] = A->Bg; pg[0].P = P; pg[0].ldp = 2 * rp; pg[0].p_cols = r;
+    pg[0].out[0] = gr->dBg;
+    pg[1].X = dU; pg[1].ldx = f; pg[1].S[0] = A->Bu; pg[1].P = static_cast<const char*>(P) + rp * 2;
+    pg[1].ldp = 2 * rp; pg[1].p_cols = r; pg[1].out[0] = gr->dBu;
+    TRY(launch_dual(dual_plan(D, DL_BWD_GU).sp, pg, 2, T, f, r, s, Q, 2 * rp, part,
+                    cnt + dual_cnt_offset(D, DL_BWD_GU), status, st, PH_Q_GU));
   } else {
     // S7a: Q = s * [dG Bg | dU Bu]
     GemmArgs a = new_args(status);
@@ -741,7 +790,12 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // (M = d or f, MN-major A), columns the rank (N = r, MN-major narrow B).
   const int rbn = r <= 64 ? 64 : 128;
   // S9: dAg = Q_g^T H, dAu = Q_u^T H   ([r x d], written transposed from [d x r] tiles)
-  {
+  if (dmode == 2) {
+    DualProblem pr{};
+    pr.X = H; pr.ldx = d; pr.P = Q; pr.ldp = 2 * rp; pr.p_cols = 2 * rp; pr.out[0] = gr->dAg; pr.out[1] = gr->dAu;
+    TRY(launch_dual(dual_plan(D, DL_RED_GU).sp, &pr, 1, T, d, r, 1.0f, nullptr, 0, part, nullptr, status, st,
+                    PH_RED_DA_GU));
+  } else {
     GemmArgs a = new_args(status);
     a.mn3d_a = d % 64 == 0;
     if (a.mn3d_a) TRY(map_mn3(&a.maps[0], H, T, d, d, 2));
@@ -793,7 +847,12 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_RED_DB_D)));
   }
   // S6b: dAd = Qd^T Act  ([r x f], written transposed from [f x r] tiles)
-  {
+  if (dual) {
+    DualProblem pr{};
+    pr.X = Act; pr.ldx = f; pr.P = Qd; pr.ldp = rp; pr.p_cols = rp; pr.out[0] = gr->dAd;
+    TRY(launch_dual(dual_plan(D, DL_RED_D).sp, &pr, 1, T, f, r, 1.0f, nullptr, 0, part, nullptr, status, st,
+                    PH_RED_DA_D));
+  } else {
     GemmArgs a = new_args(status);
     a.mn3d_a = f % 64 == 0;
     if (a.mn3d_a) TRY(map_mn3(&a.maps[0], Act, T, f, f, 2));

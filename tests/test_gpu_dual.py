@@ -1,6 +1,8 @@
-"""The single-pass rank-r gradient kernel (Q = s X B and dB = X^T P from one read of the
-activation gradient X, for the down branch and for gate/up together) against the fp64
-oracle, on shapes chosen for its work split:
+"""The single-pass rank-r streaming kernel against the fp64 oracle.  By default it computes
+Q = s X B together with dB = X^T P from one read of the activation gradient X (the down
+branch, and gate/up together) and the reduction dAd = Qd^T Act; with LORA_MLP_DUAL=2 it
+also computes the forward projections P, Pd (the row product alone, K-major operand) and
+dAg, dAu (the column product alone, written transposed).  Shapes chosen for its work split:
 
 * several CTAs per (row region, problem), so Q goes through the fp32 partial slots and is
   summed by the last CTA to arrive (arrival order varies from run to run: the result may
@@ -10,8 +12,9 @@ oracle, on shapes chosen for its work split:
 * two calls in a row on one workspace (the arrival counters are left at zero).
 
 The workspace and outputs start poisoned (NaN / 0xFF).  The two-pass form
-(LORA_MLP_DUAL=0: a projection GEMM and a reduction GEMM) runs the small MLP suite in a
-fresh process, since the library reads that setting once."""
+(LORA_MLP_DUAL=0: a projection GEMM and a reduction GEMM) and the all-products form
+(LORA_MLP_DUAL=2) run the small MLP suite and these shapes in fresh processes, since the
+library reads that setting once."""
 import os
 import subprocess
 import sys
@@ -56,8 +59,9 @@ def test_rank_r_pass_parity(cuda_ok, shape):
     compare(pb, R)
 
 
-def test_two_pass_form(cuda_ok):
-    env = dict(os.environ, LORA_MLP_DUAL="0")
+@pytest.mark.parametrize("mode", ["0", "2"], ids=["two_pass", "all_products"])
+def test_other_forms(cuda_ok, mode):
+    env = dict(os.environ, LORA_MLP_DUAL=mode)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         "tests/test_gpu_lora_mlp.py::test_fwd_bwd_parity_small",
                         "tests/test_gpu_dual.py::test_rank_r_pass_parity"], cwd=ROOT, env=env,
