@@ -601,7 +601,7 @@ struct DualProblem {
   const void* P;
   long long ldp;
   int p_cols;
-  float* out[2];
+  float* out[3];
 };
 // Which products a launch computes and how their operands and outputs are laid out.
 struct DualSpec {
@@ -622,7 +622,7 @@ inline DualSpec dual_spec_proj(int r, int nbk) {
   const int rp = round_up(r, 16);
   return DualSpec{1, 0, 1, nbk, 0, nbk * rp, nbk * rp};
 }
-// dA_i += (Q[:, i rp : i rp + r])^T X for the nq column blocks of Q (the reductions over T)
+// dA_i += (Q[:, i rp : i rp + r])^T X for the nq (<= 3) column blocks of Q (the reductions over T)
 inline DualSpec dual_spec_reduce(int r, int nq) {
   const int rp = round_up(r, 16);
   const int w = nq * rp;
@@ -725,10 +725,8 @@ inline int launch_dual(const DualSpec& sp, const DualProblem* pr, int nx, long l
     if (sp.do_col) TRY(make_map(&a.p[m], pr[m].P, pr[m].p_cols, T, pr[m].ldp, prow / 2, 128, map_swz));
     a.out[m] = pr[m].out[0];
   }
-  if (sp.col_trans) {
-    a.out[0] = pr[0].out[0];
-    a.out[1] = pr[0].out[1];
-  }
+  if (sp.col_trans)
+    for (int i = 0; i < 3; ++i) a.out[i] = pr[0].out[i];
   a.nx = nx;
   a.T = T;
   a.K = K;

@@ -32,8 +32,25 @@ lora_qkv_ctx_layout qkv_ctx_layout(const lora_qkv_dims* D) {
   return L;
 }
 
+// Rank-r streaming launches of the Q/K/V backward (lowrank_dual.cuh): Q_q with dB_q, then
+// Q_k, Q_v with dB_k, dB_v (two problems sharing K = nkv), then dA_q, dA_k, dA_v in one
+// read of H.  Their arrival counters follow one another in the workspace.
+struct QkvDual {
+  DualSpec sp;
+  int K, nx;
+  long long cnt_off;
+};
+QkvDual qkv_dual(const lora_qkv_dims* D, int which) {
+  const DualSpec both = dual_spec_both(D->r);
+  const long long c0 = dual_counters(both, D->T, D->nq, 1);
+  if (which == 0) return QkvDual{both, D->nq, 1, 0};
+  if (which == 1) return QkvDual{both, D->nkv, 2, c0};
+  return QkvDual{dual_spec_reduce(D->r, 3), D->d, 1, c0 + dual_counters(both, D->T, D->nkv, 2)};
+}
+
 struct QkvWsLayout {
-  size_t status, Q, dH, part, total;
+  size_t status, Q, dH, part, cnt, total;
+  long long ncnt;
 };
 QkvWsLayout qkv_ws_layout(const lora_qkv_dims* D) {
   const size_t T = D->T, d = D->d, rp = round_up(D->r, 16);
@@ -45,7 +62,13 @@ QkvWsLayout qkv_ws_layout(const lora_qkv_dims* D) {
   size_t part = 0;
   for (long long K : {static_cast<long long>(D->d), static_cast<long long>(D->nq), static_cast<long long>(D->nkv)})
     part = std::max(part, size_t(proj_splits(T, K)) * T * rp);
+  for (int i = 0; i < 2; ++i) {  // the single-pass kernels' partial slots (Q rows of 3 rp)
+    const QkvDual q = qkv_dual(D, i);
+    part = std::max(part, size_t(dual_slots_bound(q.sp, D->T, q.K, q.nx)) * T * 3 * rp);
+  }
   L.part = o; o = up256(o + part * 4);
+  L.ncnt = qkv_dual(D, 2).cnt_off;
+  L.cnt = o; o = up256(o + static_cast<size_t>(L.ncnt) * 4);
   L.total = o;
   return L;
 }
@@ -62,16 +85,21 @@ int check_o_dims(const lora_o_dims* D) {
 }
 
 struct OWsLayout {
-  size_t status, Q, part, total;
+  size_t status, Q, part, cnt, total;
+  long long ncnt;
 };
 OWsLayout o_ws_layout(const lora_o_dims* D) {
   const size_t T = D->T, rp = round_up(D->r, 16);
+  const DualSpec both = dual_spec_both(D->r);  // Q = s dY Bo with dBo = dY^T P, one read of dY
   OWsLayout L{};
   size_t o = 0;
   L.status = o; o = 256;
   L.Q = o; o = up256(o + T * rp * 2);        // s dY Bo
   size_t part = std::max(size_t(proj_splits(T, D->n_in)), size_t(proj_splits(T, D->n_out))) * T * rp;
+  part = std::max(part, size_t(dual_slots_bound(both, D->T, D->n_out, 1)) * T * rp);
   L.part = o; o = up256(o + part * 4);
+  L.ncnt = dual_counters(both, D->T, D->n_out, 1);
+  L.cnt = o; o = up256(o + static_cast<size_t>(L.ncnt) * 4);
   L.total = o;
   return L;
 }
@@ -181,8 +209,38 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
   const int nx[3] = {D->nq, D->nkv, D->nkv};
   const int qbn = rp <= 64 ? 64 : 128;
   TRY(begin_call(status, st));
+  int* cnt = at<int>(workspace, WL.cnt);
+  const bool dual = dual_mode() >= 1;
+  // adapter gradients: overwrite semantics -> zero them (and the arrival counters), then
+  // accumulate with atomics
+  {
+    ZeroList z{};
+    for (int x = 0; x < 3; ++x) {
+      z.p[2 * x] = dAx[x]; z.n[2 * x] = static_cast<long long>(r) * d;
+      z.p[2 * x + 1] = dBx[x]; z.n[2 * x + 1] = static_cast<long long>(nx[x]) * r;
+    }
+    z.p[6] = reinterpret_cast<float*>(cnt); z.n[6] = WL.ncnt;  // int zero = float +0 bits
+    PhaseScope ps(st, PH_ZERO);
+    zero_grads_kernel<<<296, 256, 0, st>>>(z);
+    CUDA_TRY(cudaGetLastError());
+  }
+  if (dual) {
+    // Q_x = s dZ_x B_x into columns [x rp, x rp + rp) of Q [T x 3rp] with dB_x = dZ_x^T P_x,
+    // one read of each dZ_x: q alone, then k and v (same width) together
+    DualProblem pr[3] = {};
+    for (int x = 0; x < 3; ++x) {
+      pr[x].X = dZ[x]; pr[x].ldx = nx[x]; pr[x].S[0] = Bx[x];
+      pr[x].P = P + static_cast<size_t>(x) * rp * 2; pr[x].ldp = 3 * rp; pr[x].p_cols = r;
+      pr[x].out[0] = dBx[x];
+    }
+    const QkvDual q0 = qkv_dual(D, 0), q1 = qkv_dual(D, 1);
+    TRY(launch_dual(q0.sp, &pr[0], 1, T, D->nq, r, D->scale, Q, 3 * rp, part, cnt + q0.cnt_off, status, st,
+                    PH_QKV_LOWRANK));
+    TRY(launch_dual(q1.sp, &pr[1], 2, T, D->nkv, r, D->scale, Q + static_cast<size_t>(rp) * 2, 3 * rp, part,
+                    cnt + q1.cnt_off, status, st, PH_QKV_LOWRANK));
+  }
   // Q_x = s dZ_x B_x into columns [x rp, x rp + rp) of Q [T x 3rp]
-  for (int x = 0; x < 3; ++x) {
+  for (int x = 0; x < 3 && !dual; ++x) {
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], dZ[x], T, nx[x], nx[x], 128));
     TRY(map_mn(&a.maps[1], Bx[x], nx[x], r, r));
@@ -220,19 +278,18 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_QKV_DH)));
   }
   TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));
-  {
-    ZeroList z{};
-    for (int x = 0; x < 3; ++x) {
-      z.p[2 * x] = dAx[x]; z.n[2 * x] = static_cast<long long>(r) * d;
-      z.p[2 * x + 1] = dBx[x]; z.n[2 * x + 1] = static_cast<long long>(nx[x]) * r;
-    }
-    PhaseScope ps(st, PH_ZERO);
-    zero_grads_kernel<<<296, 256, 0, st>>>(z);
-    CUDA_TRY(cudaGetLastError());
-  }
   const int rbn = r <= 64 ? 64 : 128;
+  const bool dual_da = dual && qkv_dual(D, 2).sp.n <= 256;  // 3 rp columns fit one MMA (r <= 80)
+  if (dual_da) {
+    // dA_q, dA_k, dA_v = [Q_q | Q_k | Q_v]^T H in one read of H  ([r x d] each)
+    DualProblem pr{};
+    pr.X = H; pr.ldx = d; pr.P = Q; pr.ldp = 3 * rp; pr.p_cols = 3 * rp;
+    for (int x = 0; x < 3; ++x) pr.out[x] = dAx[x];
+    TRY(launch_dual(qkv_dual(D, 2).sp, &pr, 1, T, d, r, 1.0f, nullptr, 0, part, nullptr, status, st,
+                    PH_QKV_LOWRANK));
+  }
   // dA_x = Q_x^T H  ([r x d], written transposed from [d x r] tiles)
-  for (int x = 0; x < 3; ++x) {
+  for (int x = 0; x < 3 && !dual_da; ++x) {
     GemmArgs a = new_args(status);
     a.mn3d_a = d % 64 == 0;
     if (a.mn3d_a) TRY(map_mn3(&a.maps[0], H, T, d, d, 2));
@@ -246,7 +303,7 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_QKV_LOWRANK)));
   }
   // dB_x = dZ_x^T P_x  ([n_x x r])
-  for (int x = 0; x < 3; ++x) {
+  for (int x = 0; x < 3 && !dual; ++x) {
     GemmArgs a = new_args(status);
     a.mn3d_a = nx[x] % 64 == 0;
     if (a.mn3d_a) TRY(map_mn3(&a.maps[0], dZ[x], T, nx[x], nx[x], 2));
@@ -333,8 +390,24 @@ int lora_o_bwd(const lora_o_dims* D, const void* dY, const void* X, const void* 
   float* part = at<float>(workspace, WL.part);
   void* Q = at<char>(workspace, WL.Q);
   TRY(begin_call(status, st));
-  // Q = s dY Bo
-  {
+  int* cnt = at<int>(workspace, WL.cnt);
+  const bool dual = dual_mode() >= 1;
+  {  // overwrite semantics: zero the gradients (and the arrival counters), then accumulate
+    ZeroList z{};
+    z.p[0] = dAo; z.n[0] = static_cast<long long>(r) * n_in;
+    z.p[1] = dBo; z.n[1] = static_cast<long long>(n_out) * r;
+    z.p[2] = reinterpret_cast<float*>(cnt); z.n[2] = WL.ncnt;  // int zero = float +0 bits
+    PhaseScope ps(st, PH_ZERO);
+    zero_grads_kernel<<<148, 256, 0, st>>>(z);
+    CUDA_TRY(cudaGetLastError());
+  }
+  if (dual) {
+    // Q = s dY Bo with dBo = dY^T P, one read of dY
+    DualProblem pr{};
+    pr.X = dY; pr.ldx = n_out; pr.S[0] = Bo; pr.P = ctx; pr.ldp = rp; pr.p_cols = r; pr.out[0] = dBo;
+    TRY(launch_dual(dual_spec_both(r), &pr, 1, T, n_out, r, D->scale, Q, rp, part, cnt, status, st, PH_O_LOWRANK));
+  } else {
+    // Q = s dY Bo
     GemmArgs a = new_args(status);
     TRY(map_k(&a.maps[0], dY, T, n_out, n_out, 128));
     TRY(map_mn(&a.maps[1], Bo, n_out, r, r));
@@ -369,14 +442,6 @@ int lora_o_bwd(const lora_o_dims* D, const void* dY, const void* X, const void* 
     if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_BF16, 2>(a, st, PH_O_DX)));
     else TRY((launch_gemm<0, 1, 1, EPI_BF16>(a, st, PH_O_DX)));
   }
-  {
-    ZeroList z{};
-    z.p[0] = dAo; z.n[0] = static_cast<long long>(r) * n_in;
-    z.p[1] = dBo; z.n[1] = static_cast<long long>(n_out) * r;
-    PhaseScope ps(st, PH_ZERO);
-    zero_grads_kernel<<<148, 256, 0, st>>>(z);
-    CUDA_TRY(cudaGetLastError());
-  }
   const int rbn = r <= 64 ? 64 : 128;
   // dAo = Q^T X  ([r x n_in], written transposed from [n_in x r] tiles)
   {
@@ -393,7 +458,7 @@ int lora_o_bwd(const lora_o_dims* D, const void* dY, const void* X, const void* 
     TRY((launch_gemm<1, 1, 1, EPI_ATOMIC>(a, st, PH_O_LOWRANK)));
   }
   // dBo = dY^T P  ([n_out x r])
-  {
+  if (!dual) {
     GemmArgs a = new_args(status);
     a.mn3d_a = n_out % 64 == 0;
     if (a.mn3d_a) TRY(map_mn3(&a.maps[0], dY, T, n_out, n_out, 2));

@@ -58,7 +58,7 @@ struct DualArgs {
   int row_kmajor, nbk;  // the row product's operand is K-major from nbk maps (else MN-major)
   int qw;               // row-product columns written per problem: problem m owns [m qw, (m + 1) qw)
   int col_trans;        // column product: 0 -> out[m] is [K x r]; 1 -> accumulator column c goes to
-                        // row c % rp of the [r x K] matrix out[c / rp] (problem 0 only)
+                        // row c % rp of the [r x K] matrix out[c / rp] (problem 0 only, up to 3)
   int prow, patoms;     // MN-major skinny tiles: bytes per row (32, 64, 128 = the swizzle width),
                         // 64-column atoms
   uint32_t swz;         // their shared-memory swizzle (SmemSwizzle)
@@ -69,7 +69,7 @@ struct DualArgs {
   int nrb, nc, nreg;    // row blocks, column groups of 128, row regions
   long long units;      // nreg * nx * nc
   float scale;          // applied to the row product only
-  float* out[2];        // column-product outputs, fp32, accumulated with atomics (zeroed by the caller)
+  float* out[3];        // column-product outputs, fp32, accumulated with atomics (zeroed by the caller)
   uint16_t* Q;          // row-product output, bf16 [T x ldq]
   int ldq;
   float* part;          // fp32 partials [slots][T][ldq]
@@ -368,7 +368,7 @@ static __device__ __noinline__ void dual_epilogue(const DualArgs& p, uint32_t cf
             const float x2 = __shfl_sync(0xffffffffu, __uint_as_float(v[e]), src + 2);
             const float x3 = __shfl_sync(0xffffffffu, __uint_as_float(v[e]), src + 3);
             const int c = c0 + e, o = c / rp, j = c - o * rp;
-            if ((lane & 3) == (e & 3) && j < r && o < 2 && kb < K) {
+            if ((lane & 3) == (e & 3) && j < r && o < 3 && kb < K) {
               float* dst = p.out[o];
               if (dst) atomicAdd(reinterpret_cast<float4*>(dst + static_cast<long long>(j) * K + kb),
                                  make_float4(x0, x1, x2, x3));

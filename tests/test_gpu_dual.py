@@ -13,8 +13,9 @@ dAg, dAu (the column product alone, written transposed).  Shapes chosen for its 
 
 The workspace and outputs start poisoned (NaN / 0xFF).  The two-pass form
 (LORA_MLP_DUAL=0: a projection GEMM and a reduction GEMM) and the all-products form
-(LORA_MLP_DUAL=2) run the small MLP suite and these shapes in fresh processes, since the
-library reads that setting once."""
+(LORA_MLP_DUAL=2) run the small MLP, Q/K/V and o_proj suites and these shapes in fresh
+processes, since the library reads that setting once.  The Q/K/V and o_proj backward use
+the kernel too (Q with dB per branch; dA_q, dA_k, dA_v from one read of H)."""
 import os
 import subprocess
 import sys
@@ -64,7 +65,9 @@ def test_other_forms(cuda_ok, mode):
     env = dict(os.environ, LORA_MLP_DUAL=mode)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         "tests/test_gpu_lora_mlp.py::test_fwd_bwd_parity_small",
-                        "tests/test_gpu_dual.py::test_rank_r_pass_parity"], cwd=ROOT, env=env,
+                        "tests/test_gpu_dual.py::test_rank_r_pass_parity",
+                        "tests/test_gpu_qkv.py::test_qkv_parity_small",
+                        "tests/test_gpu_attn.py::test_o_proj_parity_small"], cwd=ROOT, env=env,
                        capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
     assert " passed" in r.stdout
