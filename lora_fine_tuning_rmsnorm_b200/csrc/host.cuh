@@ -65,8 +65,9 @@ inline bool debug_mode() {
 // Which rank-r products run in the single-pass streaming kernel (lowrank_dual.cuh) rather
 // than as split-K / split-T GEMMs; both forms compute the same quantities.  LORA_MLP_DUAL:
 //   1 (default): the fused backward passes (Q with dB from one read of dY, of dG / dU) and
-//                the reduction over the wide activation (dAd), where it measured faster;
-//   2: every rank-r product (also P, Pd, dAg / dAu, which measured a few us slower);
+//                the reductions over T (dAg / dAu, dAd), where it measured faster;
+//   2: every rank-r product (also the forward projections P, Pd, which measured a few us
+//      slower than the split-K GEMM);
 //   0: none (two passes over each activation gradient).
 // Read once per process.
 inline int dual_mode() {
@@ -641,20 +642,18 @@ inline void dual_tile_geometry(int n, int* prow, int* patoms, CUtensorMapSwizzle
   *map_swz = *prow == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : (*prow == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
   *smem_swz = *prow == 32 ? kSwz32 : (*prow == 64 ? kSwz64 : kSwz128);
 }
-// Row blocks per region: 2 while a row product keeps R accumulators in TMEM; a column
-// product alone takes the largest of 16, 8, 4, 2 that still leaves two units per CTA of a
-// full grid (each region adds one fp32 atomic per output element).
+// Row blocks per region: 2 while a row product keeps R accumulators in TMEM; 8 for a
+// column product alone (each region adds one fp32 atomic per output element; at the 8B
+// shape R = 8 measured faster than 4 and 16 for both reductions over T).
 inline int dual_rows(const DualSpec& sp, long long T, int K, int nx) {
   static const int r_knob = [] {
     const char* e = getenv("LORA_MLP_DUAL_R");  // tuning knob: row blocks per region
     return e ? atoi(e) : 0;
   }();
-  const long long nrb = (T + 127) / 128, nc = (K + 127) / 128;
-  int R = 2;
-  if (!sp.do_row) {
-    for (R = 16; R > 2; R /= 2)
-      if ((nrb + R - 1) / R * nx * nc >= 2LL * kDualMaxGrid) break;
-  }
+  (void)T;
+  (void)K;
+  (void)nx;
+  int R = sp.do_row ? 2 : 8;
   if (r_knob >= 1) R = std::max(1, std::min(r_knob, sp.do_row ? 512 / sp.n - 2 : 64));
   return R;
 }

@@ -790,7 +790,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
   // (M = d or f, MN-major A), columns the rank (N = r, MN-major narrow B).
   const int rbn = r <= 64 ? 64 : 128;
   // S9: dAg = Q_g^T H, dAu = Q_u^T H   ([r x d], written transposed from [d x r] tiles)
-  if (dmode == 2) {
+  if (dual) {
     DualProblem pr{};
     pr.X = H; pr.ldx = d; pr.P = Q; pr.ldp = 2 * rp; pr.p_cols = 2 * rp; pr.out[0] = gr->dAg; pr.out[1] = gr->dAu;
     TRY(launch_dual(dual_plan(D, DL_RED_GU).sp, &pr, 1, T, d, r, 1.0f, nullptr, 0, part, nullptr, status, st,
