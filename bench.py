@@ -228,12 +228,13 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ timing
-def timed(step, steps, stream, clk=None, label=None):
+def timed(step, steps, stream, clk=None, label=None, phases=False):
     """Events around `steps` calls of step() on `stream` (after a synchronize); returns
-    total ms and the library's per-phase times of those calls."""
+    total ms and, with `phases`, the library's per-phase times of those calls (their
+    events are off otherwise, so a plain timed loop carries none)."""
     import torch
     from lora_fine_tuning_rmsnorm_b200 import ops
-    ops.timing_enable(True)
+    ops.timing_enable(phases)
     ops.timing_collect()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -247,9 +248,17 @@ def timed(step, steps, stream, clk=None, label=None):
     torch.cuda.synchronize()
     if ctx:
         ctx.__exit__(None, None, None)
-    ph = ops.timing_collect()
+    ph = ops.timing_collect() if phases else {}
     ops.timing_enable(False)
     return e0.elapsed_time(e1), ph
+
+
+def timed_with_phases(step, steps, stream, clk=None, label=None):
+    """The timed loop (no phase events; clocks sampled), then the same number of steps
+    again with the phase events on for the per-kernel breakdown."""
+    ms, _ = timed(step, steps, stream, clk, label)
+    _, ph = timed(step, steps, stream, phases=True)
+    return ms, ph
 
 
 def dominant(phases, name, flops_per_step, steps, peak):
@@ -284,7 +293,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     pb = Problem(s1, synth.make_inputs_bits(s1))
     for _ in range(3):
         pb.step()
-    ms, ph = timed(pb.step, steps, stream, clk, "config_1b")
+    ms, ph = timed_with_phases(pb.step, steps, stream, clk, "config_1b")
     rec("config_1b", f"LoRA-MLP fwd+bwd, Llama-3.2-1B MLP shape: T={s1.T} d={s1.d} f={s1.f} r={s1.r} alpha=16",
         s1.T, configs.algorithmic_flops(s1), ms, ph, "gemm_gate_up_swiglu",
         4.0 * s1.T * s1.d * s1.f + 4.0 * s1.T * s1.r * s1.f)
@@ -294,7 +303,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     pb8.use_4bit(load_codebook(), drop_bf16=False)
     for _ in range(3):
         pb8.step()
-    ms, ph = timed(pb8.step, steps, stream, clk, "config_4bit")
+    ms, ph = timed_with_phases(pb8.step, steps, stream, clk, "config_4bit")
     rec("config_4bit", f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape with 4-bit frozen W (block 64): T={s8.T} d={s8.d} "
         f"f={s8.f} r={s8.r} alpha=16", s8.T, configs.algorithmic_flops(s8), ms, ph, "gemm_gate_up_swiglu",
         4.0 * s8.T * s8.d * s8.f + 4.0 * s8.T * s8.r * s8.f, dtype=dtype_for("8b-4bit"))
@@ -302,7 +311,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     pb8.use_4bit(load_codebook(), double_quant=True)
     for _ in range(3):
         pb8.step()
-    ms, ph = timed(pb8.step, steps, stream, clk, "config_4bit_dq")
+    ms, ph = timed_with_phases(pb8.step, steps, stream, clk, "config_4bit_dq")
     rec("config_4bit_dq", f"LoRA-MLP fwd+bwd, Llama-3-8B MLP shape with 4-bit frozen W, double-quantised block "
         f"constants: T={s8.T} d={s8.d} f={s8.f} r={s8.r} alpha=16", s8.T, configs.algorithmic_flops(s8), ms, ph,
         "gemm_gate_up_swiglu", 4.0 * s8.T * s8.d * s8.f + 4.0 * s8.T * s8.r * s8.f,
@@ -312,7 +321,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     qp = QkvProblem(sq)
     for _ in range(3):
         qp.step()
-    ms, ph = timed(qp.step, steps, stream, clk, "qkv")
+    ms, ph = timed_with_phases(qp.step, steps, stream, clk, "qkv")
     rec("qkv", f"LoRA Q/K/V projections fwd+bwd, Llama-3-8B attention shape: T={sq.T} d={sq.d} nq={sq.nq} "
         f"nkv={sq.nkv} r={sq.r} alpha=16", sq.T, configs.qkv_algorithmic_flops(sq), ms, ph, "qkv_gemm",
         2.0 * sq.T * sq.d * (sq.nq + 2 * sq.nkv))
@@ -322,7 +331,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     op = OProblem(so)
     for _ in range(3):
         op.step()
-    ms, ph = timed(op.step, steps, stream, clk, "o_proj")
+    ms, ph = timed_with_phases(op.step, steps, stream, clk, "o_proj")
     rec("o_proj", f"LoRA o_proj fwd+bwd, Llama-3-8B shape: T={so.T} n_in={so.n_in} n_out={so.n_out} r={so.r} "
         "alpha=16", so.T, configs.o_algorithmic_flops(so), ms, ph, "o_gemm", 2.0 * so.T * so.n_in * so.n_out)
     del op
@@ -331,7 +340,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     rp = RopeProblem(sr)
     for _ in range(3):
         rp.step()
-    ms, ph = timed(rp.step, steps, stream, clk, "rope")
+    ms, ph = timed_with_phases(rp.step, steps, stream, clk, "rope")
     rb = configs.rope_bytes(sr)
     rms, rn = ph.get("rope", (0.0, 0))
     gbs = rb / (rms / rn / 1e3) / 1e9 if rn else None
@@ -349,7 +358,7 @@ def sub_records(args, pb8, bits8, clk, pk):
     cp = CeProblem(sc)
     for _ in range(3):
         cp.step()
-    ms, ph = timed(cp.step, steps, stream, clk, "ce")
+    ms, ph = timed_with_phases(cp.step, steps, stream, clk, "ce")
     rec("ce", f"fused LM-head cross-entropy fwd+bwd, Llama-3-8B head: T={sc.T} d={sc.d} V={sc.V} "
         f"(vocabulary chunk 32768 in the backward)", sc.T, configs.ce_algorithmic_flops(sc), ms, ph,
         "ce_gemm_lse", 2.0 * sc.T * sc.d * sc.V)
@@ -396,9 +405,12 @@ def ours_arm(args, rank, world, local_rank):
 
     # ---- device-resident timed region
     barrier()
-    ms, phases = timed(step, args.steps, stream, clk, "main")
+    ms, _ = timed(step, args.steps, stream, clk, "main")
     barrier()
     ms = ldist.max_over_ranks(ms, dev)
+    # per-kernel breakdown: the same number of steps again with the library's phase events
+    # on (outside the timed region; every rank takes the same steps)
+    _, phases = timed(step, args.steps, stream, phases=True)
     value = world * shape.T * args.steps / (ms / 1e3)
 
     # ---- end-to-end through the C ABI with host buffers (pinned): every step copies its
@@ -543,7 +555,7 @@ def extras(args):
     def timed_steps(pb):
         for _ in range(args.warmup):
             pb.step()
-        ms, ph = timed(pb.step, args.steps, stream)
+        ms, ph = timed_with_phases(pb.step, args.steps, stream)
         return ms / args.steps, ph
 
     plain = Problem(shape, bits)
@@ -589,7 +601,7 @@ def sweep(args):
         pb = Problem(s, synth.make_inputs_bits(s))
         for _ in range(args.warmup):
             pb.step()
-        ms, ph = timed(pb.step, args.steps, stream)
+        ms, ph = timed_with_phases(pb.step, args.steps, stream)
         ms /= args.steps
         gemm = sum(ph.get(k, (0.0, 0))[0] for k in GEMM_PHASES) / args.steps
         other = sum(v[0] for k, v in ph.items() if k not in GEMM_PHASES) / args.steps
