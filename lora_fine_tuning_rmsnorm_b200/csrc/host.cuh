@@ -528,7 +528,12 @@ inline int pick_mt(long long T, int pair, int bn, long long N, double gain) {
 }
 
 // Expected MT = 2 gains by GEMM kind (see pick_mt).
-constexpr double kMtGain4bit = 0.8, kMtGainCe = 0.85, kMtGainBf16Swiglu = 1.02;
+constexpr double kMtGain4bit = 0.8, kMtGainCe = 0.85, kMtGainBf16Swiglu = 1.02, kMtGainBf16 = 1.02;
+// bf16 GEMMs with a long K (down: K = f, dH: K = 2f, the cross-entropy's dH: K = the
+// vocabulary chunk): the epilogue is a small part of a unit, fetching B once per two M tiles
+// pays (8B shape: down 0.80 -> 0.71 ms, dH 1.59 -> 1.40 ms; the dAct GEMM, K = d with the
+// SwiGLU' epilogue, measured 13 % slower and keeps kMtGainBf16)
+constexpr double kMtGainBf16LongK = 0.8;
 
 // Rank-r projection out[T x cols] (bf16) = scale * sum of K-split fp32 partials.
 // The GEMM args must already hold maps/segments/M/N/bn/tiles and NACC columns.

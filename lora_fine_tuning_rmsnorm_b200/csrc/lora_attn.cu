@@ -270,11 +270,14 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     }
     TRY(map_k(&a.maps[6], Q, T, 3 * rp, 3 * rp, 128));
     for (int x = 0; x < 3; ++x) set_seg(a, 3 + x, 6, x * rp, 7 + x, 0, -1, 0, rp);
+    // K = nq + 2 nkv (+ 3 rp): long enough that B fetched once per two M tiles pays
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, d, kMtGainBf16LongK) : 1;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
-    set_band(a, 4);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_QKV_DH)));
+    set_band(a, mt == 2 ? 2 : 4);
+    if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 0, 2>(a, st, PH_QKV_DH)));
+    else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_QKV_DH)));
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_QKV_DH)));
   }
   TRY(launch_rms_bwd(st, dH, X, rms_w, rstd, dX, T, d));

@@ -167,12 +167,14 @@ int lora_ce_bwd(const lora_ce_dims* D, const void* H, const void* W, const int32
       if (a.mn3d_b) TRY(map_mn3(&a.maps[1], Wc, N, d, d, bn / pair / 64));
       else TRY(map_mn(&a.maps[1], Wc, N, d, d));
       set_seg(a, 0, 0, 0, 1, 0, -1, 0, N);
+      const int mt = pair == 2 ? pick_mt(T, pair, bn, d, kMtGainBf16LongK) : 1;  // K = the chunk
       a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-      a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
+      a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
       a.out[0] = dH; a.ld_out = d;
       a.out_add = v0 > 0;
-      set_band(a, 4);
-      if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_CE_DH)));
+      set_band(a, mt == 2 ? 2 : 4);
+      if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 0, 2>(a, st, PH_CE_DH)));
+      else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_CE_DH)));
       else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_CE_DH)));
     }
   }

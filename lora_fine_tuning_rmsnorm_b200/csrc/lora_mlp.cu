@@ -561,13 +561,15 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     TRY(map_k(&a.maps[3], A->Bd, d, r, r, bn / pair));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, f);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, d, kMtGainBf16LongK) : 1;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
     if (D->residual) { a.in[0] = X; a.ld_in = d; }  // Y = X + ...
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_DOWN)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 0, 2>(a, st, PH_DOWN)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_DOWN)));
     else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_DOWN)));
   }
   return end_call(status, st);
@@ -684,13 +686,15 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     }
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, f, kMtGainBf16) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (f + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2, 0, 0, 2>(a, st, PH_DACT)));
+    else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2>(a, st, PH_DACT)));
     else TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD>(a, st, PH_DACT)));
   }
   if (dual) {
@@ -767,12 +771,14 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, f);
     set_seg(a, 2, 4, 0, 5, 0, -1, 0, rp);
     set_seg(a, 3, 4, rp, 6, 0, -1, 0, rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, d, kMtGainBf16LongK) : 1;
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (d + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_DH)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 0, 2>(a, st, PH_DH)));
+    else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_DH)));
     else TRY((launch_gemm<0, 1, 1, EPI_F32>(a, st, PH_DH)));
   }
   // S10: dX = RMSNorm backward (cached rstd)
