@@ -4,6 +4,7 @@ run of the asynchronous, non-debug path and the status query outside debug mode.
 
     python -m tests.gpu_worker mlp8b OUT.npz      # 8B-shaped fwd+bwd, as bench.py runs it
     python -m tests.gpu_worker stall OUT.npz      # a GEMM whose waits run out, then a normal one
+    python -m tests.gpu_worker graph OUT.npz      # fwd+bwd captured in a CUDA graph and replayed
 """
 import os
 import sys
@@ -46,5 +47,41 @@ def stall(out_path):
              A=Ab, B=Bb)
 
 
+def graph(out_path):
+    """The MLP and Q/K/V fwd+bwd called eagerly, then captured once into one CUDA graph on a
+    side torch stream and replayed twice: outputs of the eager calls and of the replays."""
+    import torch
+    from lora_fine_tuning_rmsnorm_b200 import ops, synth
+    from lora_fine_tuning_rmsnorm_b200.runner import QkvProblem, Problem
+    mlp = Problem(synth.Shape(T=1000, d=256, f=640, r=16, alpha=16.0))
+    qkv = QkvProblem(synth.QkvShape(T=600, d=256, nq=256, nkv=64, r=16))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        mlp.step(stream=s)
+        qkv.step(stream=s)
+
+    def snapshot():
+        torch.cuda.synchronize()
+        out = {"mlp_Y": mlp.Y, "mlp_dX": mlp.dX, **{"mlp_" + k: v for k, v in mlp.g.items()},
+               "qkv_dX": qkv.dX, **{"qkv_" + k: v for k, v in qkv.out.items()},
+               **{"qkv_g_" + k: v for k, v in qkv.g.items()}}
+        return {k: v.float().cpu().numpy().copy() for k, v in out.items()}
+
+    with torch.cuda.stream(s):
+        step()
+    eager = snapshot()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for k in range(2):
+        g.replay()
+    replay = snapshot()
+    code = ops.status(mlp.ws)
+    np.savez(out_path, status=np.int32(code), **{"eager_" + k: v for k, v in eager.items()},
+             **{"replay_" + k: v for k, v in replay.items()})
+
+
 if __name__ == "__main__":
-    {"mlp8b": mlp8b, "stall": stall}[sys.argv[1]](sys.argv[2])
+    {"mlp8b": mlp8b, "stall": stall, "graph": graph}[sys.argv[1]](sys.argv[2])
