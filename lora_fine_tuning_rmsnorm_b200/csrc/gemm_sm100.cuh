@@ -34,12 +34,14 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kMaxStages = 8;
 constexpr int kMaxSegs = 6;
-constexpr int kMaxMaps = 10;
+constexpr int kMaxMaps = 12;
 constexpr int kEpiWarps = 8;  // two warps per TMEM lane quarter, alternating 16-column chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kDqWarps = 8;  // 4-bit weights: warps that expand codes into bf16 B tiles
 constexpr int kDqGroups = 2;  // ... in groups that take alternate stages
 constexpr int kCodeRing = 8;  // 4-bit weights: entries of the code ring (codes + absmax of one stage)
+// Epilogue staging for TMA stores: per epilogue warp, three [32 rows x 16 columns] bf16 tiles
+constexpr int kEpiStageBytes = 3 * 32 * 16 * 2;
 // Code-ring entries for MT M tiles per unit (two tiles per unit leave less shared memory)
 __host__ __device__ constexpr int code_ring(int mt) { return mt == 2 ? 4 : kCodeRing; }
 // 4-bit CTAs add the dequant warps and one warp that fills the code ring
@@ -128,6 +130,9 @@ struct GemmArgs {
   int test_no_loads;      // test of the bounded waits: the producer copies nothing and arms no
                           // barrier, so the MMA's first wait runs out (single-CTA tiles only)
   int out_add;            // EPI_F32: add into the fp32 output instead of overwriting it
+  int epi_tma;            // EPI_SWIGLU_FWD / _BWD: the outputs (G, U, Act / dG, dU) leave through shared
+                          // memory by TMA stores (maps from out_map0: bf16 [M x N], box {16, 32}, no swizzle)
+  int out_map0;
   // cross-entropy epilogues (rows = tokens, columns = vocabulary entries ce_col0 + n)
   const int* ce_labels;   // label of each row; outside [0, ce_V) = left out of the loss
   const float* ce_lse;    // EPI_CE_DZ: logsumexp of each row (from the forward)
@@ -504,7 +509,8 @@ __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
 template <int NACC, int EPI, int PAIR, int MT>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0, uint32_t tempty0,
-                                              uint32_t tmem_base, const WaitCtl& wc, uint32_t rank) {
+                                              uint32_t tmem_base, const WaitCtl& wc, uint32_t rank,
+                                              uint8_t* stage_out) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int q = warp & 3;             // TMEM lane quarter this warp may access
   const int c0 = ((warp - 2) >> 2) * 16;  // first 16-column chunk of this warp; stride 32
@@ -526,6 +532,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   const int* const ce_count = p.ce_count;
   const float ce_g = p.ce_g;
   const int ce_col0 = p.ce_col0, ce_V = p.ce_V;
+  const int epi_tma = p.epi_tma;
+  const CUtensorMap* const out_maps = p.maps + p.out_map0;
+  const uint32_t stg = smem_u32(stage_out) + static_cast<uint32_t>(warp - 2) * kEpiStageBytes;  // this warp's
   uint32_t it = 0;
   for (int t = unit0; t < total; t += nunits, ++it) {
     int mt, nt, ks;
@@ -599,6 +608,45 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
           }
         }
       }
+    } else if (EPI == EPI_SWIGLU_FWD && epi_tma) {
+      // The warp's 32 rows x 16 columns of G, U and Act go to its staging tiles, then out by
+      // three TMA stores (whole 32-byte rows of the box per write instead of a 16-byte piece of
+      // 32 different rows per store instruction); boxes are clipped at the tensor's end.
+      const int row0 = m0 + 32 * q;
+#pragma unroll 1
+      for (int c = c0; c < bn; c += 32) {
+        uint32_t rg[16], ru[16];
+        tmem_ld16(tbase + c, rg);
+        tmem_ld16(tbase + bn + c, ru);
+        tmem_wait32(rg, ru);
+        const int n = n0 + c;
+        if (lane == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging tiles
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pg[4], pu[4], pa[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float g0 = __uint_as_float(rg[8 * h + 2 * j]), g1 = __uint_as_float(rg[8 * h + 2 * j + 1]);
+            const float u0 = __uint_as_float(ru[8 * h + 2 * j]), u1 = __uint_as_float(ru[8 * h + 2 * j + 1]);
+            pg[j] = pack_bf16x2(g0, g1);
+            pu[j] = pack_bf16x2(u0, u1);
+            pa[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+          }
+          const uint32_t o = stg + static_cast<uint32_t>(lane) * 32u + 16u * h;
+          st_shared_v4(o, pg);
+          st_shared_v4(o + 1024u, pu);
+          st_shared_v4(o + 2048u, pa);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < M && n < N) {
+          tma_store_2d(out_maps + 0, stg, n, row0);
+          tma_store_2d(out_maps + 1, stg + 1024u, n, row0);
+          tma_store_2d(out_maps + 2, stg + 2048u, n, row0);
+          bulk_commit();
+        }
+      }
     } else if (EPI == EPI_SWIGLU_FWD) {
 #pragma unroll 1
       for (int c = c0; c < bn; c += 32) {
@@ -646,6 +694,44 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         uint32_t r[16];
         tmem_ld16(tbase + c, r);
         tmem_wait16(r);
+        if (epi_tma) {
+          // dG and dU of the warp's 32 rows x 16 columns leave by two TMA stores (see SwiGLU fwd)
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t gw[4] = {gv[h].x, gv[h].y, gv[h].z, gv[h].w};
+            const uint32_t uw[4] = {uv[h].x, uv[h].y, uv[h].z, uv[h].w};
+            uint32_t pdg[4], pdu[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float dg[2], du[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const float g = e ? bf16hi(gw[j]) : bf16lo(gw[j]);
+                const float u = e ? bf16hi(uw[j]) : bf16lo(uw[j]);
+                const float da = __uint_as_float(r[8 * h + 2 * j + e]);
+                const float sg = sigmoid_f(g);
+                du[e] = da * g * sg;
+                dg[e] = da * u * sg * (1.0f + g * (1.0f - sg));
+              }
+              pdg[j] = pack_bf16x2(dg[0], dg[1]);
+              pdu[j] = pack_bf16x2(du[0], du[1]);
+            }
+            const uint32_t o = stg + static_cast<uint32_t>(lane) * 32u + 16u * h;
+            st_shared_v4(o, pdg);
+            st_shared_v4(o + 1024u, pdu);
+          }
+          fence_async_smem();
+          __syncwarp();
+          const int row0 = m0 + 32 * q;
+          if (lane == 0 && row0 < M && n < N) {
+            tma_store_2d(out_maps + 0, stg, n, row0);
+            tma_store_2d(out_maps + 1, stg + 1024u, n, row0);
+            bulk_commit();
+          }
+          continue;
+        }
         if (!row_ok) continue;
         const long long off = row * ld_out + n;
 #pragma unroll
@@ -786,6 +872,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       else mbar_arrive_cluster(mapa_shared(tempty0 + 8 * buf, 0));  // the MMA issuer's barrier
     }
   }
+  if ((EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) && epi_tma && lane == 0) bulk_wait0();  // before the CTA exits
 }
 
 // 4-bit code-ring producer (one thread of the code warp): for every stage of a 4-bit
@@ -1006,7 +1093,8 @@ static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = tiles + static_cast<size_t>(p.stages) * p.stage_bytes;  // Q4: code ring
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (Q4 ? static_cast<size_t>(code_ring(MT)) * p.cr_bytes : 0));
+  uint8_t* stage_out = ring + (Q4 ? static_cast<size_t>(code_ring(MT)) * p.cr_bytes : 0);  // epilogue staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage_out + (p.epi_tma ? kEpiWarps * kEpiStageBytes : 0));
   const int S = p.stages;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * S;
@@ -1071,7 +1159,7 @@ static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const 
       gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE, Q4, MT>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc, dq0);
     __syncwarp();
   } else if (warp < 2 + kEpiWarps) {
-    gemm_epilogue<NACC, EPI, PAIR, MT>(p, tfull0, tempty0, tmem_base, wc, rank);
+    gemm_epilogue<NACC, EPI, PAIR, MT>(p, tfull0, tempty0, tmem_base, wc, rank, stage_out);
   } else if (Q4 && warp < 2 + kEpiWarps + kDqWarps) {
     gemm_dequant<B_MN, NACC, FUSE, PAIR, MT>(p, tiles, ring, empty0, crfull0, crempty0, dq0, tab, wc, rank);
   } else if (Q4) {

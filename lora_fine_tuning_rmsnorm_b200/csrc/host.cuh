@@ -256,7 +256,8 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   a.stage_bytes = (a.stage_bytes + 1023) & ~1023u;
   const int extra = Q4 ? 2560 : 256;  // barriers (+ the 4-bit code table)
   const int ring = Q4 ? code_ring(MT) * static_cast<int>(a.cr_bytes) : 0;
-  const int avail = kSmemLimit - 1024 - extra - ring;
+  const int stg = a.epi_tma ? kEpiWarps * kEpiStageBytes : 0;  // epilogue staging for TMA stores
+  const int avail = kSmemLimit - 1024 - extra - ring - stg;
   a.stages = std::min(kMaxStages, avail / static_cast<int>(a.stage_bytes));
   static const int stage_cap = [] {
     const char* e = getenv("LORA_MLP_MAX_STAGES");  // tuning knob: cap the TMA ring depth
@@ -272,7 +273,7 @@ int launch_gemm(GemmArgs& a, cudaStream_t st, int phase) {
   while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
   if (tc > 512) return fail(LORA_ERR_UNSUPPORTED, "internal: TMEM columns %d > 512", cols);
   a.tmem_cols = tc;
-  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + ring + extra;
+  int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + ring + stg + extra;
   // more than half of TMEM per CTA: keep one CTA per SM so allocation never waits
   if (tc > 256) smem = std::max(smem, kSmemLimit / 2 + 4096);
   a.limit_ns = wait_limit_ns();
@@ -461,6 +462,29 @@ inline void set_band(GemmArgs& a, int group_m) {
   a.group_m = group_m;
 }
 
+// The SwiGLU forward epilogue's outputs (bf16 [rows x cols], row stride ld) written by TMA
+// stores from shared-memory staging: maps at a.maps[first .. first + 2].  LORA_MLP_EPI_TMA=0
+// keeps the per-thread stores (tuning comparison).
+inline bool epilogue_tma_enabled() {
+  static const int on = [] {
+    const char* e = getenv("LORA_MLP_EPI_TMA");
+    return e && e[0] == '0' ? 0 : 1;
+  }();
+  return on != 0;
+}
+inline int set_epilogue_tma(GemmArgs& a, int first, std::initializer_list<const void*> outs, long long rows,
+                            long long cols, long long ld) {
+  if (!epilogue_tma_enabled()) return LORA_OK;
+  if (first < 0 || first + static_cast<int>(outs.size()) > kMaxMaps)
+    return fail(LORA_ERR_UNSUPPORTED, "internal: bad epilogue maps");
+  int i = first;
+  for (const void* p : outs)
+    TRY(make_map_raw(&a.maps[i++], p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cols, rows, ld, 16, 32));
+  a.epi_tma = 1;
+  a.out_map0 = first;
+  return LORA_OK;
+}
+
 inline void set_hints(GemmArgs& a, int a_hint, int b_hint) {
   for (int s = 0; s < a.nseg; ++s) {
     a.seg[s].a_hint = a_hint;
@@ -528,7 +552,13 @@ inline int pick_mt(long long T, int pair, int bn, long long N, double gain) {
 }
 
 // Expected MT = 2 gains by GEMM kind (see pick_mt).
-constexpr double kMtGain4bit = 0.8, kMtGainCe = 0.85, kMtGainBf16Swiglu = 1.02, kMtGainBf16 = 1.02;
+constexpr double kMtGain4bit = 0.8, kMtGainCe = 0.85, kMtGainBf16 = 1.02;
+// bf16 gate/up with its SwiGLU outputs leaving by TMA stores: MT = 2 measured 1.74 -> 1.45 ms at
+// the 8B shape (with per-thread stores the exposed epilogue cancelled the gain: 1.73 ms)
+constexpr double kMtGainBf16Swiglu = 0.8;
+// bf16 dAct (SwiGLU' epilogue): MT = 2 measured slower (0.91 -> 1.08 ms) even with dG, dU leaving by
+// TMA stores, since its per-thread loads of G, U stay exposed; it keeps MT = 1 unless forced
+constexpr double kMtGainBf16Dact = 1.02;
 // bf16 GEMMs with a long K (down: K = f, dH: K = 2f, the cross-entropy's dH: K = the
 // vocabulary chunk): the epilogue is a small part of a unit, fetching B once per two M tiles
 // pays (8B shape: down 0.80 -> 0.71 ms, dH 1.59 -> 1.40 ms; the dAct GEMM, K = d with the

@@ -501,10 +501,13 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     TRY(map_k(&a.maps[5], A->Bu, f, r, r, 128));
     set_seg(a, 0, 0, 0, 1, 0, 2, 0, d);
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
-    const int mt = pair == 2 ? pick_mt(T, pair, 128, f, kMtGainBf16Swiglu) : 1;
+    // MT = 2 leaves one accumulator set, so the epilogue no longer hides behind the next
+    // unit's main loop: it then writes G, U, Act by TMA stores from shared-memory staging
+    const int mt = pair == 2 ? pick_mt(T, pair, 128, f, epilogue_tma_enabled() ? kMtGainBf16Swiglu : 1.02) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
+    if (mt == 2) TRY(set_epilogue_tma(a, 6, {G, U, Act}, T, f, f));
     set_hints(a, HINT_EVICT_LAST, HINT_NONE);  // H is re-read by every N tile: keep it in L2
     set_band(a, 8 / mt);
     a.stream_out = 1;
@@ -686,11 +689,12 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     }
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
-    const int mt = pair == 2 ? pick_mt(T, pair, bn, f, kMtGainBf16) : 1;
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, f, kMtGainBf16Dact) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + bn - 1) / bn;
     a.in[0] = G; a.in[1] = U; a.ld_in = f;
     a.out[0] = dG; a.out[1] = dU; a.ld_out = f;
+    if (mt == 2) TRY(set_epilogue_tma(a, 4, {dG, dU}, T, f, f));
     a.stream_out = 1;
     set_band(a, 8 / mt);
     if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_SWIGLU_BWD, 2, 0, 0, 2>(a, st, PH_DACT)));
