@@ -130,8 +130,8 @@ struct GemmArgs {
   int test_no_loads;      // test of the bounded waits: the producer copies nothing and arms no
                           // barrier, so the MMA's first wait runs out (single-CTA tiles only)
   int out_add;            // EPI_F32: add into the fp32 output instead of overwriting it
-  int epi_tma;            // EPI_SWIGLU_FWD / _BWD: the outputs (G, U, Act / dG, dU) leave through shared
-                          // memory by TMA stores (maps from out_map0: bf16 [M x N], box {16, 32}, no swizzle)
+  int epi_tma;            // the outputs (SwiGLU: G, U, Act / dG, dU; bf16, fp32 (NACC = 1) and CE dZ: out[0])
+                          // leave through shared memory by TMA stores; maps from out_map0, box {16, 32}, no swizzle
   int out_map0;
   // cross-entropy epilogues (rows = tokens, columns = vocabulary entries ce_col0 + n)
   const int* ce_labels;   // label of each row; outside [0, ce_V) = left out of the loss
@@ -553,7 +553,54 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
     const bool row_ok = row < M;
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (MT * NACC * bn) + h * (NACC * bn);
 
-    if (EPI == EPI_F32 || EPI == EPI_BF16) {
+    if ((EPI == EPI_F32 || EPI == EPI_BF16) && NACC == 1 && epi_tma) {
+      // The warp's 32 rows x 16 columns leave by one TMA store (fp32 with out_add: a TMA
+      // add-reduction into the old values) from its staging tile
+      const int row0 = m0 + 32 * q;
+#pragma unroll 1
+      for (int c = c0; c < bn; c += 32) {
+        uint32_t r[16];
+        tmem_ld16(tbase + c, r);
+        tmem_wait16(r);
+        const int n = n0 + c;
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        if (EPI == EPI_F32) {
+          const uint32_t o = stg + static_cast<uint32_t>(lane) * 64u;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint32_t w[4] = {__float_as_uint(__uint_as_float(r[4 * h]) * alpha),
+                                   __float_as_uint(__uint_as_float(r[4 * h + 1]) * alpha),
+                                   __float_as_uint(__uint_as_float(r[4 * h + 2]) * alpha),
+                                   __float_as_uint(__uint_as_float(r[4 * h + 3]) * alpha)};
+            st_shared_v4(o + 16u * h, w);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float v8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(r[8 * h + e]) * alpha;
+            if (in0 && row_ok && n + 8 * h < N) {  // residual input (bf16, same layout as the output)
+              const uint4 xv = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in0) +
+                                                                   row * ld_in + n + 8 * h));
+              v8[0] += bf16lo(xv.x); v8[1] += bf16hi(xv.x); v8[2] += bf16lo(xv.y); v8[3] += bf16hi(xv.y);
+              v8[4] += bf16lo(xv.z); v8[5] += bf16hi(xv.z); v8[6] += bf16lo(xv.w); v8[7] += bf16hi(xv.w);
+            }
+            const uint32_t w[4] = {pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]), pack_bf16x2(v8[4], v8[5]),
+                                   pack_bf16x2(v8[6], v8[7])};
+            st_shared_v4(stg + static_cast<uint32_t>(lane) * 32u + 16u * h, w);
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < M && n < N) {
+          if (EPI == EPI_F32 && out_add) tma_reduce_add_2d(out_maps, stg, n, row0);
+          else tma_store_2d(out_maps, stg, n, row0);
+          bulk_commit();
+        }
+      }
+    } else if (EPI == EPI_F32 || EPI == EPI_BF16) {
 #pragma unroll 1
       for (int a = 0; a < NACC; ++a) {
 #pragma unroll 1
@@ -843,6 +890,34 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         uint32_t r[16];
         tmem_ld16(tbase + c, r);
         tmem_wait16(r);
+        if (epi_tma) {  // dZ of the warp's 32 rows x 16 columns leaves by one TMA store
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float dz[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int k = 8 * h + 2 * j + e;
+                const float pr = exp2f(fmaf(__uint_as_float(r[k]), kLog2e, -l2));
+                dz[e] = gs * (pr - (ce_col0 + n + k == lab ? 1.f : 0.f));
+              }
+              w[j] = pack_bf16x2(dz[0], dz[1]);
+            }
+            st_shared_v4(stg + static_cast<uint32_t>(lane) * 32u + 16u * h, w);
+          }
+          fence_async_smem();
+          __syncwarp();
+          const int row0 = m0 + 32 * q;
+          if (lane == 0 && row0 < M) {
+            tma_store_2d(out_maps, stg, n, row0);
+            bulk_commit();
+          }
+          continue;
+        }
         if (!row_ok) continue;
         uint16_t* o = static_cast<uint16_t*>(out0) + row * ld_out + n;
 #pragma unroll
@@ -872,7 +947,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       else mbar_arrive_cluster(mapa_shared(tempty0 + 8 * buf, 0));  // the MMA issuer's barrier
     }
   }
-  if ((EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) && epi_tma && lane == 0) bulk_wait0();  // before the CTA exits
+  if (epi_tma && lane == 0) bulk_wait0();  // the TMA stores are done before the CTA exits
 }
 
 // 4-bit code-ring producer (one thread of the code warp): for every stage of a 4-bit

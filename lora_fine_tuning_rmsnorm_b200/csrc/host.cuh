@@ -462,9 +462,10 @@ inline void set_band(GemmArgs& a, int group_m) {
   a.group_m = group_m;
 }
 
-// The SwiGLU forward epilogue's outputs (bf16 [rows x cols], row stride ld) written by TMA
-// stores from shared-memory staging: maps at a.maps[first .. first + 2].  LORA_MLP_EPI_TMA=0
-// keeps the per-thread stores (tuning comparison).
+// Epilogue outputs ([rows x cols] bf16 or fp32, row stride ld) written by TMA stores from
+// shared-memory staging, for GEMMs run with MT = 2 (one accumulator set: the epilogue no longer
+// hides behind the next unit's main loop): maps at a.maps[first ...].  LORA_MLP_EPI_TMA=0 keeps
+// the per-thread stores (tuning comparison).
 inline bool epilogue_tma_enabled() {
   static const int on = [] {
     const char* e = getenv("LORA_MLP_EPI_TMA");
@@ -473,13 +474,14 @@ inline bool epilogue_tma_enabled() {
   return on != 0;
 }
 inline int set_epilogue_tma(GemmArgs& a, int first, std::initializer_list<const void*> outs, long long rows,
-                            long long cols, long long ld) {
+                            long long cols, long long ld, bool fp32 = false) {
   if (!epilogue_tma_enabled()) return LORA_OK;
   if (first < 0 || first + static_cast<int>(outs.size()) > kMaxMaps)
     return fail(LORA_ERR_UNSUPPORTED, "internal: bad epilogue maps");
   int i = first;
   for (const void* p : outs)
-    TRY(make_map_raw(&a.maps[i++], p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cols, rows, ld, 16, 32));
+    TRY(make_map_raw(&a.maps[i++], p, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     fp32 ? 4 : 2, cols, rows, ld, 16, 32));
   a.epi_tma = 1;
   a.out_map0 = first;
   return LORA_OK;

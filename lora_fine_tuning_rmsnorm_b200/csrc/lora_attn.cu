@@ -275,6 +275,7 @@ int lora_qkv_bwd(const lora_qkv_dims* D, const void* dQ, const void* dK, const v
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
+    if (mt == 2) TRY(set_epilogue_tma(a, 10, {dH}, T, d, d, true));
     set_band(a, mt == 2 ? 2 : 4);
     if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 0, 2>(a, st, PH_QKV_DH)));
     else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_QKV_DH)));

@@ -150,6 +150,7 @@ int lora_ce_bwd(const lora_ce_dims* D, const void* H, const void* W, const int32
       a.M = static_cast<int>(T); a.N = N; a.bn = bn;
       a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (N + bn - 1) / bn;
       a.out[0] = dZ; a.ld_out = chunk;
+      if (mt == 2) TRY(set_epilogue_tma(a, 2, {dZ}, T, N, chunk));
       a.ce_labels = labels; a.ce_lse = lse; a.ce_count = D->reduction == LORA_CE_MEAN ? n_valid : nullptr;
       a.ce_g = dloss; a.ce_col0 = v0; a.ce_V = V;
       if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_CE_DZ, 2, 0, 0, 2>(a, st, PH_CE_DZ)));
@@ -171,7 +172,8 @@ int lora_ce_bwd(const lora_ce_dims* D, const void* H, const void* W, const int32
       a.M = static_cast<int>(T); a.N = d; a.bn = bn;
       a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
       a.out[0] = dH; a.ld_out = d;
-      a.out_add = v0 > 0;
+      a.out_add = v0 > 0;  // with TMA stores: an fp32 add-reduction into the previous chunks' sum
+      if (mt == 2) TRY(set_epilogue_tma(a, 2, {dH}, T, d, d, true));
       set_band(a, mt == 2 ? 2 : 4);
       if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 0, 2>(a, st, PH_CE_DH)));
       else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2>(a, st, PH_CE_DH)));

@@ -569,6 +569,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = d;
     if (D->residual) { a.in[0] = X; a.ld_in = d; }  // Y = X + ...
+    if (mt == 2) TRY(set_epilogue_tma(a, 4, {Y}, T, d, d));
     a.stream_out = 1;
     set_band(a, 8 / mt);
     if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 0, 2>(a, st, PH_DOWN)));
@@ -779,6 +780,7 @@ int lora_mlp_bwd(const lora_mlp_dims* D, const void* dY, const void* X, const vo
     a.M = static_cast<int>(T); a.N = d; a.bn = bn;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (d + bn - 1) / bn;
     a.out[0] = dH; a.ld_out = d;
+    if (mt == 2) TRY(set_epilogue_tma(a, 7, {dH}, T, d, d, true));
     a.stream_out = 1;
     set_band(a, 8 / mt);
     if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_F32, 2, 0, 0, 2>(a, st, PH_DH)));
