@@ -473,6 +473,9 @@ inline bool epilogue_tma_enabled() {
   }();
   return on != 0;
 }
+// MT = 2 gain for a short-K bf16 GEMM whose epilogue only stores (gate/up, the Q/K/V and
+// o_proj GEMMs): worth it when the stores leave by TMA (see kMtGainBf16Swiglu), not otherwise.
+inline double mt_gain_bf16_stores() { return epilogue_tma_enabled() ? 0.8 : 1.02; }
 inline int set_epilogue_tma(GemmArgs& a, int first, std::initializer_list<const void*> outs, long long rows,
                             long long cols, long long ld, bool fp32 = false) {
   if (!epilogue_tma_enabled()) return LORA_OK;

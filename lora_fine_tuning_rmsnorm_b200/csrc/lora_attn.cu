@@ -170,12 +170,15 @@ int lora_qkv_fwd(const lora_qkv_dims* D, const void* X, const void* rms_w, const
     TRY(map_k(&a.maps[3], Bx[x], nx[x], r, r, bn / pair));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, d);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, nx[x], mt_gain_bf16_stores()) : 1;
     a.M = static_cast<int>(T); a.N = nx[x]; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (nx[x] + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (nx[x] + bn - 1) / bn;
     a.out[0] = Ox[x]; a.ld_out = nx[x];
+    if (mt == 2) TRY(set_epilogue_tma(a, 4, {Ox[x]}, T, nx[x], nx[x]));
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_QKV_GEMM)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 0, 2>(a, st, PH_QKV_GEMM)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_QKV_GEMM)));
     else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_QKV_GEMM)));
   }
   return end_call(status, st);
@@ -371,12 +374,15 @@ int lora_o_fwd(const lora_o_dims* D, const void* X, const void* Wo, const void* 
     TRY(map_k(&a.maps[3], Bo, n_out, r, r, bn / pair));
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, n_in);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, n_out, mt_gain_bf16_stores()) : 1;
     a.M = static_cast<int>(T); a.N = n_out; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (n_out + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (n_out + bn - 1) / bn;
     a.out[0] = Y; a.ld_out = n_out;
+    if (mt == 2) TRY(set_epilogue_tma(a, 4, {Y}, T, n_out, n_out));
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_O_GEMM)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2, 0, 0, 2>(a, st, PH_O_GEMM)));
+    else if (pair == 2) TRY((launch_gemm<0, 0, 1, EPI_BF16, 2>(a, st, PH_O_GEMM)));
     else TRY((launch_gemm<0, 0, 1, EPI_BF16>(a, st, PH_O_GEMM)));
   }
   return end_call(status, st);
@@ -438,12 +444,15 @@ int lora_o_bwd(const lora_o_dims* D, const void* dY, const void* X, const void* 
     }
     set_seg(a, 0, 0, 0, 1, 0, -1, 0, n_out);
     set_seg(a, 1, 2, 0, 3, 0, -1, 0, rp);
+    const int mt = pair == 2 ? pick_mt(T, pair, bn, n_in, mt_gain_bf16_stores()) : 1;
     a.M = static_cast<int>(T); a.N = n_in; a.bn = bn;
-    a.tiles_m = static_cast<int>((T + BM * pair - 1) / (BM * pair)); a.tiles_n = (n_in + bn - 1) / bn;
+    a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (n_in + bn - 1) / bn;
     a.out[0] = dX; a.ld_out = n_in;
+    if (mt == 2) TRY(set_epilogue_tma(a, 4, {dX}, T, n_in, n_in));
     a.stream_out = 1;
-    set_band(a, 8);
-    if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_BF16, 2>(a, st, PH_O_DX)));
+    set_band(a, 8 / mt);
+    if (mt == 2) TRY((launch_gemm<0, 1, 1, EPI_BF16, 2, 0, 0, 2>(a, st, PH_O_DX)));
+    else if (pair == 2) TRY((launch_gemm<0, 1, 1, EPI_BF16, 2>(a, st, PH_O_DX)));
     else TRY((launch_gemm<0, 1, 1, EPI_BF16>(a, st, PH_O_DX)));
   }
   const int rbn = r <= 64 ? 64 : 128;

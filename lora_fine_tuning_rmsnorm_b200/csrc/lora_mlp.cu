@@ -503,7 +503,7 @@ int lora_mlp_fwd(const lora_mlp_dims* D, const void* X, const void* rms_w, const
     set_seg(a, 1, 3, 0, 4, 0, 5, -rp, 2 * rp);
     // MT = 2 leaves one accumulator set, so the epilogue no longer hides behind the next
     // unit's main loop: it then writes G, U, Act by TMA stores from shared-memory staging
-    const int mt = pair == 2 ? pick_mt(T, pair, 128, f, epilogue_tma_enabled() ? kMtGainBf16Swiglu : 1.02) : 1;
+    const int mt = pair == 2 ? pick_mt(T, pair, 128, f, mt_gain_bf16_stores()) : 1;
     a.M = static_cast<int>(T); a.N = f; a.bn = 128;
     a.tiles_m = static_cast<int>((T + BM * pair * mt - 1) / (BM * pair * mt)); a.tiles_n = (f + 127) / 128;
     a.out[0] = G; a.out[1] = U; a.out[2] = Act; a.ld_out = f;
