@@ -451,10 +451,15 @@ def ours_arm(args, rank, world, local_rank):
     if rank != 0:
         return
     T, d, f, r = shape.T, shape.d, shape.f, shape.r
-    # dominant kernel: the gate/up GEMM with the LoRA B-term and the SwiGLU epilogue
-    dom = "gemm_gate_up_swiglu"
+    # dominant kernel: the dense GEMM with the most time per step (gate/up and dH are within a
+    # few per cent of each other at the 8B shape), with its algorithmic FLOPs per launch
+    gemm_flops_per_launch = {"gemm_gate_up_swiglu": 4.0 * T * d * f + 4.0 * T * r * f,
+                             "gemm_down": 2.0 * T * d * f + 2.0 * T * r * d,
+                             "gemm_dact_swiglu_bwd": 2.0 * T * d * f + 2.0 * T * r * f,
+                             "gemm_dH": 4.0 * T * d * f + 4.0 * T * r * d}
+    dom = max(GEMM_PHASES, key=lambda k: phases.get(k, (0.0, 0))[0])
     dom_ms, dom_n = phases.get(dom, (0.0, 0))
-    dom_flops = 4.0 * T * d * f + 4.0 * T * r * f
+    dom_flops = gemm_flops_per_launch[dom]
     dom_tflops = dom_flops / (dom_ms / dom_n / 1e3) / 1e12 if dom_n else None
     flops = configs.algorithmic_flops(shape)
     step_ms = ms / args.steps
