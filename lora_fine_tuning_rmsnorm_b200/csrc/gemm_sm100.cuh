@@ -533,6 +533,12 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
   const float ce_g = p.ce_g;
   const int ce_col0 = p.ce_col0, ce_V = p.ce_V;
   const int epi_tma = p.epi_tma;
+  // whole 16-column pieces of a row go out (come in) as one 32-byte access when aligned
+  const bool v8_out = ld_out % 16 == 0 && ((reinterpret_cast<uintptr_t>(out0) | reinterpret_cast<uintptr_t>(out1) |
+                                            reinterpret_cast<uintptr_t>(out2)) & 31) == 0;
+  const bool v8_in = ld_in % 16 == 0 && ((reinterpret_cast<uintptr_t>(in0) | reinterpret_cast<uintptr_t>(in1)) & 31) == 0;
+  const bool v8_f32 = v8_out && ld_out % 8 == 0 && split_stride % 8 == 0 && out_acc_col % 8 == 0;
+  const bool v8_bf16 = v8_out && out_acc_col % 16 == 0 && (!in0 || v8_in);
   const CUtensorMap* const out_maps = p.maps + p.out_map0;
   const uint32_t stg = smem_u32(stage_out) + static_cast<uint32_t>(warp - 2) * kEpiStageBytes;  // this warp's
   uint32_t it = 0;
@@ -613,6 +619,22 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
           if (EPI == EPI_F32) {
             float* o = static_cast<float*>(out0) + ks * split_stride + row * ld_out +
                        a * out_acc_col + n;
+            if (v8_f32 && n + 16 <= N) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(__uint_as_float(r[8 * h + e]) * alpha);
+                if (out_add) {
+                  uint32_t old[8];
+                  ld_global_v8(o + 8 * h, old, 1);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) + __uint_as_float(old[e]));
+                }
+                st_global_v8(o + 8 * h, w, stream_out);
+              }
+              continue;
+            }
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               if (n + 4 * h < N) {
@@ -629,6 +651,25 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             }
           } else {
             uint16_t* o = static_cast<uint16_t*>(out0) + row * ld_out + a * out_acc_col + n;
+            if (v8_bf16 && n + 16 <= N) {
+              float v16[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v16[e] = __uint_as_float(r[e]) * alpha;
+              if (in0) {  // residual input (bf16, same layout as the output) added in fp32
+                uint32_t x8[8];
+                ld_global_v8(static_cast<const uint16_t*>(in0) + row * ld_in + n, x8, 0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  v16[2 * j] += bf16lo(x8[j]);
+                  v16[2 * j + 1] += bf16hi(x8[j]);
+                }
+              }
+              uint32_t w[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(v16[2 * j], v16[2 * j + 1]);
+              st_global_v8(o, w, stream_out);
+              continue;
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               if (n + 8 * h < N) {
@@ -704,6 +745,21 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         const int n = n0 + c;
         if (!row_ok) continue;
         const long long off = row * ld_out + n;
+        if (v8_out && n + 16 <= N) {
+          uint32_t g8[8], u8[8], a8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float g0 = __uint_as_float(rg[2 * j]), g1 = __uint_as_float(rg[2 * j + 1]);
+            const float u0 = __uint_as_float(ru[2 * j]), u1 = __uint_as_float(ru[2 * j + 1]);
+            g8[j] = pack_bf16x2(g0, g1);
+            u8[j] = pack_bf16x2(u0, u1);
+            a8[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+          }
+          st_global_v8(static_cast<uint16_t*>(out0) + off, g8, stream_out);
+          st_global_v8(static_cast<uint16_t*>(out1) + off, u8, stream_out);
+          st_global_v8(static_cast<uint16_t*>(out2) + off, a8, stream_out);
+          continue;
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (n + 8 * h >= N) continue;
@@ -726,6 +782,14 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
       for (int c = c0; c < bn; c += 32) {
         const int n = n0 + c;
         uint4 gv[2], uv[2];
+        if (v8_in && row_ok && n + 16 <= N) {
+          uint32_t g8[8], u8[8];
+          const long long off = row * ld_in + n;
+          ld_global_v8(static_cast<const uint16_t*>(in0) + off, g8, 1);
+          ld_global_v8(static_cast<const uint16_t*>(in1) + off, u8, 1);
+          gv[0] = make_uint4(g8[0], g8[1], g8[2], g8[3]); gv[1] = make_uint4(g8[4], g8[5], g8[6], g8[7]);
+          uv[0] = make_uint4(u8[0], u8[1], u8[2], u8[3]); uv[1] = make_uint4(u8[4], u8[5], u8[6], u8[7]);
+        } else {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (row_ok && n + 8 * h < N) {
@@ -737,6 +801,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
             gv[h] = make_uint4(0, 0, 0, 0);
             uv[h] = make_uint4(0, 0, 0, 0);
           }
+        }
         }
         uint32_t r[16];
         tmem_ld16(tbase + c, r);
@@ -781,12 +846,11 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         }
         if (!row_ok) continue;
         const long long off = row * ld_out + n;
+        uint32_t pdg[8], pdu[8];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (n + 8 * h >= N) continue;
           const uint32_t gw[4] = {gv[h].x, gv[h].y, gv[h].z, gv[h].w};
           const uint32_t uw[4] = {uv[h].x, uv[h].y, uv[h].z, uv[h].w};
-          uint32_t pdg[4], pdu[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float dg[2], du[2];
@@ -799,11 +863,22 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
               du[e] = da * g * sg;
               dg[e] = da * u * sg * (1.0f + g * (1.0f - sg));
             }
-            pdg[j] = pack_bf16x2(dg[0], dg[1]);
-            pdu[j] = pack_bf16x2(du[0], du[1]);
+            pdg[4 * h + j] = pack_bf16x2(dg[0], dg[1]);
+            pdu[4 * h + j] = pack_bf16x2(du[0], du[1]);
           }
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out0) + off + 8 * h), make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]), stream_out);
-          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out1) + off + 8 * h), make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]), stream_out);
+        }
+        if (v8_out && n + 16 <= N) {
+          st_global_v8(static_cast<uint16_t*>(out0) + off, pdg, stream_out);
+          st_global_v8(static_cast<uint16_t*>(out1) + off, pdu, stream_out);
+          continue;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (n + 8 * h >= N) continue;
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out0) + off + 8 * h),
+                 make_uint4(pdg[4 * h], pdg[4 * h + 1], pdg[4 * h + 2], pdg[4 * h + 3]), stream_out);
+          st_out(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out1) + off + 8 * h),
+                 make_uint4(pdu[4 * h], pdu[4 * h + 1], pdu[4 * h + 2], pdu[4 * h + 3]), stream_out);
         }
       }
     } else if (EPI == EPI_ATOMIC) {
@@ -920,23 +995,25 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
         }
         if (!row_ok) continue;
         uint16_t* o = static_cast<uint16_t*>(out0) + row * ld_out + n;
+        uint32_t w[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (n + 8 * h >= N) continue;
-          uint32_t w[4];
+        for (int j = 0; j < 8; ++j) {
+          float dz[2];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float dz[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int k = 8 * h + 2 * j + e;
-              const float pr = exp2f(fmaf(__uint_as_float(r[k]), kLog2e, -l2));
-              dz[e] = gs * (pr - (ce_col0 + n + k == lab ? 1.f : 0.f));
-            }
-            w[j] = pack_bf16x2(dz[0], dz[1]);
+          for (int e = 0; e < 2; ++e) {
+            const int k = 2 * j + e;
+            const float pr = exp2f(fmaf(__uint_as_float(r[k]), kLog2e, -l2));
+            dz[e] = gs * (pr - (ce_col0 + n + k == lab ? 1.f : 0.f));
           }
-          st_out(reinterpret_cast<uint4*>(o + 8 * h), make_uint4(w[0], w[1], w[2], w[3]), stream_out);
+          w[j] = pack_bf16x2(dz[0], dz[1]);
         }
+        if (v8_out && n + 16 <= N) {
+          st_global_v8(o, w, stream_out);
+          continue;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (n + 8 * h < N) st_out(reinterpret_cast<uint4*>(o + 8 * h), make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]), stream_out);
       }
     }
     }  // M tiles of the unit

@@ -136,6 +136,31 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[
 }
 // Orders this thread's generic-proxy shared-memory writes before later async-proxy reads (TMA).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 32-byte global store / load of one thread (sm_100 256-bit vector access); the address is
+// 32-byte aligned.  `streaming` marks the store evict-first (.cs).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8], int streaming) {
+  if (streaming)
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  else
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+// `streaming` marks the load evict-first (.cs): data read once.
+__device__ __forceinline__ void ld_global_v8(const void* p, uint32_t (&w)[8], int streaming) {
+  if (streaming)
+    asm volatile("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p)
+                 : "memory");
+  else
+    asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p)
+                 : "memory");
+}
 // 2-D tiled bulk tensor load global -> shared, completion counted in bytes on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
                                             int32_t x, int32_t y) {
