@@ -132,6 +132,8 @@ struct GemmArgs {
   int out_add;            // EPI_F32: add into the fp32 output instead of overwriting it
   int epi_tma;            // the outputs (SwiGLU: G, U, Act / dG, dU; bf16, fp32 (NACC = 1) and CE dZ: out[0])
                           // leave through shared memory by TMA stores; maps from out_map0, box {16, 32}, no swizzle
+  int epi_drain;          // with epi_tma, MT = 2, bf16 out (N tile 256) or SwiGLU fwd (N tile 128): the
+                          // epilogue empties TMEM into registers first (see gemm_epilogue)
   int out_map0;
   // cross-entropy epilogues (rows = tokens, columns = vocabulary entries ce_col0 + n)
   const int* ce_labels;   // label of each row; outside [0, ce_V) = left out of the loss
@@ -507,7 +509,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ float sigmoid_f(float g) { return rcp_approx(1.0f + __expf(-g)); }
 __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
-template <int NACC, int EPI, int PAIR, int MT>
+template <int NACC, int EPI, int PAIR, int MT, int Q4>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0, uint32_t tempty0,
                                               uint32_t tmem_base, const WaitCtl& wc, uint32_t rank,
                                               uint8_t* stage_out) {
@@ -552,6 +554,116 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, uint32_t tfull0
     if (!ok) break;
     tc_fence_after();
     const int n0 = nt * bn;
+    if constexpr (MT == 2 && !Q4 && ((EPI == EPI_BF16 && NACC == 1) || (EPI == EPI_SWIGLU_FWD && NACC == 2))) {
+      if (epi_tma && p.epi_drain) {
+        // With one accumulator set, the next unit's main loop waits for this epilogue.  So the
+        // warp reads its share of the accumulators out of TMEM into registers, rounded to bf16
+        // and packed two to a word, and releases TMEM before it converts and stores them: the
+        // stores then run under the next main loop.  epi_drain 2 holds both M tiles (2 x 64
+        // words a lane); 1 holds the second only and sends the first out straight from TMEM.
+        // A chunk is 16 columns: bf16 out has 8 a tile (N tile 256); SwiGLU has 4 of G and 4 of
+        // U a tile (N tile 128 each), and Act = silu(G) U is formed from the rounded G and U.
+        constexpr int kChunks = EPI == EPI_BF16 ? 8 : 4;
+        const int full = p.epi_drain == 2;
+        // the packed words of chunk i of tile h (G's 8 words, then U's 8 for SwiGLU)
+        auto read_chunk = [&](int h, int i, uint32_t (&w)[2][8]) {
+          const int m0 = (mt * 2 + h) * BM * PAIR + static_cast<int>(rank) * BM;
+          const long long row = static_cast<long long>(m0) + 32 * q + lane;
+          const uint32_t tbase =
+              tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * (MT * NACC * bn) + h * (NACC * bn);
+#pragma unroll
+          for (int a = 0; a < (EPI == EPI_BF16 ? 1 : 2); ++a) {
+            const int c = a * bn + c0 + 32 * i;
+            uint32_t r[16];
+            tmem_ld16(tbase + c, r);
+            tmem_wait16(r);
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = EPI == EPI_BF16 ? __uint_as_float(r[e]) * alpha : __uint_as_float(r[e]);
+            if (EPI == EPI_BF16 && in0) {  // residual input (bf16, same layout as the output) added in fp32
+              const int n = n0 + c;
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh)
+                if (row < M && n + 8 * hh < N) {
+                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in0) +
+                                                                       row * ld_in + n + 8 * hh));
+                  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    v[8 * hh + 2 * k] += bf16lo(xw[k]);
+                    v[8 * hh + 2 * k + 1] += bf16hi(xw[k]);
+                  }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[a][k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+          }
+        };
+        // chunk i of tile h through the staging tiles and out by TMA stores
+        auto emit_chunk = [&](int h, int i, const uint32_t (&w)[2][8]) {
+          const int row0 = (mt * 2 + h) * BM * PAIR + static_cast<int>(rank) * BM + 32 * q;
+          const int n = n0 + c0 + 32 * i;
+          if (lane == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging
+          __syncwarp();
+          const uint32_t o = stg + static_cast<uint32_t>(lane) * 32u;
+          if (EPI == EPI_SWIGLU_FWD) {
+            uint32_t pa[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              pa[k] = pack_bf16x2(silu_f(bf16lo(w[0][k])) * bf16lo(w[1][k]), silu_f(bf16hi(w[0][k])) * bf16hi(w[1][k]));
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t a4[4] = {pa[4 * hh], pa[4 * hh + 1], pa[4 * hh + 2], pa[4 * hh + 3]};
+              st_shared_v4(o + 2048u + 16u * hh, a4);
+            }
+          }
+#pragma unroll
+          for (int a = 0; a < (EPI == EPI_BF16 ? 1 : 2); ++a)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t w4[4] = {w[a][4 * hh], w[a][4 * hh + 1], w[a][4 * hh + 2], w[a][4 * hh + 3]};
+              st_shared_v4(o + 1024u * a + 16u * hh, w4);
+            }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M && n < N) {
+            tma_store_2d(out_maps + 0, stg, n, row0);
+            if (EPI == EPI_SWIGLU_FWD) {
+              tma_store_2d(out_maps + 1, stg + 1024u, n, row0);
+              tma_store_2d(out_maps + 2, stg + 2048u, n, row0);
+            }
+            bulk_commit();
+          }
+        };
+        uint32_t hold[2][kChunks][2][8];
+        if (full) {
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i) read_chunk(0, i, hold[0][i]);
+        } else {
+#pragma unroll 1
+          for (int i = 0; i < kChunks; ++i) {
+            uint32_t w[2][8];
+            read_chunk(0, i, w);
+            emit_chunk(0, i, w);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) read_chunk(1, i, hold[1][i]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR == 1) mbar_arrive(tempty0 + 8 * buf);
+          else mbar_arrive_cluster(mapa_shared(tempty0 + 8 * buf, 0));  // the MMA issuer's barrier
+        }
+        if (full) {
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i) emit_chunk(0, i, hold[0][i]);
+        }
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) emit_chunk(1, i, hold[1][i]);
+        continue;
+      }
+    }
 #pragma unroll 1
     for (int h = 0; h < MT; ++h) {  // the unit's M tiles, each with its own accumulator set
     const int m0 = (mt * MT + h) * BM * PAIR + static_cast<int>(rank) * BM;
@@ -1311,7 +1423,7 @@ static __global__ void __launch_bounds__(gemm_threads(Q4), 1) gemm_kernel(const 
       gemm_mma<A_MN, B_MN, NACC, PAIR, FUSE, Q4, MT>(p, tiles, full0, empty0, tfull0, tempty0, drain_bar, tmem_base, wc, dq0);
     __syncwarp();
   } else if (warp < 2 + kEpiWarps) {
-    gemm_epilogue<NACC, EPI, PAIR, MT>(p, tfull0, tempty0, tmem_base, wc, rank, stage_out);
+    gemm_epilogue<NACC, EPI, PAIR, MT, Q4>(p, tfull0, tempty0, tmem_base, wc, rank, stage_out);
   } else if (Q4 && warp < 2 + kEpiWarps + kDqWarps) {
     gemm_dequant<B_MN, NACC, FUSE, PAIR, MT>(p, tiles, ring, empty0, crfull0, crempty0, dq0, tab, wc, rank);
   } else if (Q4) {

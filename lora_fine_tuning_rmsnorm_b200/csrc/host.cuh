@@ -485,6 +485,16 @@ inline int set_epilogue_tma(GemmArgs& a, int first, std::initializer_list<const 
   for (const void* p : outs)
     TRY(make_map_raw(&a.maps[i++], p, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                      fp32 ? 4 : 2, cols, rows, ld, 16, 32));
+  static const int drain_mode = [] {
+    // tuning knob: 0 = convert straight from TMEM, 1 = hold the second M tile, 2 = hold both
+    const char* e = getenv("LORA_MLP_EPI_DRAIN");
+    const int v = e ? atoi(e) : 2;
+    return v >= 0 && v <= 2 ? v : 2;
+  }();
+  // empty TMEM into registers first: one bf16 output with N tile 256, or the SwiGLU forward's
+  // three outputs with N tile 128 (the kernel takes it only with two M tiles per unit)
+  const bool drainable = !fp32 && (outs.size() == 3 ? a.bn == 128 : outs.size() == 1 && a.bn == 256);
+  a.epi_drain = drainable ? drain_mode : 0;
   a.epi_tma = 1;
   a.out_map0 = first;
   return LORA_OK;
