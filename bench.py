@@ -415,7 +415,7 @@ def ours_arm(args, rank, world, local_rank):
 
     # ---- end-to-end through the C ABI with host buffers (pinned): every step copies its
     # inputs in and its results (Y, dX, gradients) out inside the timed region; the copies
-    # are double-buffered on a second stream and overlap the neighbouring steps' compute
+    # are double-buffered, one stream per direction, and overlap the neighbouring steps' compute
     hX = bf16_tensor(bits["X"], "cpu", pin=True)
     hdY = bf16_tensor(bits["dY"], "cpu", pin=True)
     pipe = HostPipeline(pb, hX, hdY, reduce=ldist.allreduce_grads if world > 1 else None)
@@ -432,6 +432,7 @@ def ours_arm(args, rank, world, local_rank):
     pipe.start()
     for i in range(args.steps):
         pipe.step(i, args.steps)
+    pipe.finish()
     f1.record(pipe.xs)
     torch.cuda.synchronize(dev)
     if win:

@@ -96,11 +96,14 @@ class HostPipeline:
     """Training-step driver for inputs and results in pinned HOST memory.
 
     Every step copies its X and dY host -> device, runs lora_mlp_fwd + lora_mlp_bwd,
-    and copies Y, dX and the packed adapter gradients device -> host.  The copies
-    run on a second stream and are double-buffered, so step i's results go back and
-    step i+2's inputs come in while step i+1 computes.  `reduce` (optional) is called
-    on the packed gradient buffer on the compute stream after each backward (the
-    data-parallel all-reduce).
+    and copies Y, dX and the packed adapter gradients device -> host.  The copies are
+    double-buffered, one stream per direction (`xs` inputs in, `ss` results out, so the
+    two directions of the host link run at the same time): step i's results go back and
+    step i+2's inputs come in while step i+1 computes.  Events order the buffers: a step
+    computes once its inputs are in (`ready`) and the results of the step before it in the
+    same buffer are out (`stored`); its buffer is refilled once it has computed (`done`).
+    `reduce` (optional) is called on the packed gradient buffer on the compute stream after
+    each backward (the data-parallel all-reduce).
     """
 
     def __init__(self, pb: "Problem", hX: torch.Tensor, hdY: torch.Tensor, reduce=None):
@@ -110,6 +113,7 @@ class HostPipeline:
         dev = pb.Y.device
         self.cs = torch.cuda.current_stream(dev)
         self.xs = torch.cuda.Stream(dev)
+        self.ss = torch.cuda.Stream(dev)
         self.bufs = []
         for _ in range(2):
             flat, views = ldist.flat_grads(s.d, s.f, s.r, device=dev)
@@ -117,7 +121,7 @@ class HostPipeline:
                                   Y=torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev),
                                   dX=torch.empty(s.T, s.d, dtype=torch.bfloat16, device=dev), flat=flat,
                                   grads=ops.make_grads(*(views[k] for k in GRADS)),
-                                  ready=torch.cuda.Event(), done=torch.cuda.Event()))
+                                  ready=torch.cuda.Event(), done=torch.cuda.Event(), stored=torch.cuda.Event()))
         self.hY = torch.empty(s.T, s.d, dtype=torch.bfloat16, pin_memory=True)
         self.hdX = torch.empty(s.T, s.d, dtype=torch.bfloat16, pin_memory=True)
         self.hflat = torch.empty(self.bufs[0]["flat"].numel(), dtype=torch.float32, pin_memory=True)
@@ -138,19 +142,27 @@ class HostPipeline:
         """Run step i; with n_steps given, inputs are not prefetched past the last step."""
         pb, b = self.pb, self.bufs[i % 2]
         self.cs.wait_event(b["ready"])
+        self.cs.wait_event(b["stored"])  # step i - 2's results have left this buffer
         ops.lora_mlp_fwd(pb.dims, b["X"], pb.t["w"], pb.weights, pb.adapters, b["Y"], pb.ctx, pb.ws, self.cs)
         ops.lora_mlp_bwd(pb.dims, b["dY"], b["X"], pb.t["w"], pb.weights, pb.adapters, pb.ctx, b["dX"],
                          b["grads"], pb.ws, self.cs)
         if self.reduce is not None:
             self.reduce(b["flat"])
         b["done"].record(self.cs)
-        self.xs.wait_event(b["done"])
-        with torch.cuda.stream(self.xs):
+        self.ss.wait_event(b["done"])
+        with torch.cuda.stream(self.ss):
             self.hY.copy_(b["Y"], non_blocking=True)
             self.hdX.copy_(b["dX"], non_blocking=True)
             self.hflat.copy_(b["flat"], non_blocking=True)
+            b["stored"].record(self.ss)
         if n_steps is None or i + 2 < n_steps:
+            self.xs.wait_event(b["done"])
             self._load(b)  # inputs of step i + 2 (after this step's compute has read them)
+
+    def finish(self):
+        """Make the input stream wait for the results' copies: an event recorded on `xs`
+        afterwards completes after every step's copies and compute."""
+        self.xs.wait_stream(self.ss)
 
 
 QKV_GRADS = ("dAq", "dBq", "dAk", "dBk", "dAv", "dBv")

@@ -109,8 +109,8 @@ def test_fwd_bwd_parity_llama3_8b(cuda_ok):
 
 
 def test_host_pipeline_matches_device_step(cuda_ok):
-    """Host-buffer driver (double-buffered copies on a second stream) returns the same
-    Y, dX and gradients as the device-resident step."""
+    """Host-buffer driver (double-buffered copies, one stream per direction) returns the
+    same Y, dX and gradients as the device-resident step."""
     from lora_fine_tuning_rmsnorm_b200 import dist as ldist
     from lora_fine_tuning_rmsnorm_b200.runner import HostPipeline, bf16_tensor
     shape = synth.Shape(T=384, d=256, f=512, r=16)
@@ -120,6 +120,7 @@ def test_host_pipeline_matches_device_step(cuda_ok):
     pipe.start()
     for i in range(3):
         pipe.step(i, 3)
+    pipe.finish()
     torch.cuda.synchronize()
     assert torch.equal(pipe.hY, pb.Y.cpu()) and torch.equal(pipe.hdX, pb.dX.cpu())
     _, views = ldist.flat_grads(shape.d, shape.f, shape.r)
